@@ -1,0 +1,263 @@
+"""Plain float64 CPU oracle for Star Attention's two-phase attention (test infrastructure).
+
+Only tests, the smoke check and the benchmark's CPU-baseline leg may call this
+module. It is deliberately slow and direct: numpy matrix products and an
+explicit visibility mask, no tiling, no online softmax, no fusion.
+
+Notation (the Star Attention pages' terms): the context of L tokens is cut into
+n = ceil(L / B) blocks b_0 .. b_{n-1} of B tokens (the last one may be short);
+b_0 is the anchor block. Heads follow grouped-query attention: q-head h reads
+kv-head h // (Hq / Hkv). Scores are s(t, j) = scale * <q_t, k_j>; the
+log-sum-exp (LSE) of a row is ln sum_j exp(s(t, j)) over its visible keys.
+
+Readings where the pages are silent (each is listed in the design notes):
+  * softmax scale 1/sqrt(d) unless the caller gives one;
+  * the Phase-2 "scalar" each block returns is the natural-log LSE of its
+    scaled logits, and the "vector" is its softmax-normalised output;
+  * the anchor's keys and values are b_0's own (inputs are already projected,
+    so anchor tokens carry b_0's positions); anchor rows are not outputs;
+  * query token j sees the whole context and query tokens 0..j; a decoded token
+    sees everything cached before it and itself;
+  * contiguous GQA grouping h -> h // (Hq / Hkv).
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Sequence, Tuple
+
+import numpy as np
+
+F64 = np.float64
+_ROW_CHUNK = 1024
+
+
+def default_scale(head_dim: int) -> float:
+    """Softmax scale when the caller passes none: 1/sqrt(d), the standard
+    scaled-dot-product choice (the pages do not state one)."""
+    return 1.0 / math.sqrt(head_dim)
+
+
+def kv_head_of(h: int, num_q_heads: int, num_kv_heads: int) -> int:
+    """GQA mapping: q-head h reads kv-head h // G with G = Hq / Hkv."""
+    return h // (num_q_heads // num_kv_heads)
+
+
+def block_plan(ctx_len: int, block_size: int) -> List[Tuple[int, int]]:
+    """Context blocking (hotaipapers.com page, Phase 1 paragraph: the context is
+    split into blocks). Returns [start, end) of b_0 .. b_{n-1}, n = ceil(L/B);
+    the last block may be shorter than B."""
+    n = -(-ctx_len // block_size)
+    return [(i * block_size, min(ctx_len, (i + 1) * block_size)) for i in range(n)]
+
+
+def phase1_visible(t, j, block_size: int):
+    """Phase-1 visibility of key position j to query position t (broadcasts).
+
+    Causal attention over [anchor = b_0 ; b_i] for the block b_i holding t
+    (hotaipapers.com page, Phase 1 paragraph: a copy of the first block is put
+    in front of every other block; rebuttal to EMsM, "Size of Anchor Block":
+    the anchor is as large as a block and Phase 1 is causal). So j is visible
+    when j <= t and j lies either in the anchor b_0 or in t's own block. For
+    t in b_0 both conditions name the same block: plain causal attention.
+    """
+    t = np.asarray(t)
+    j = np.asarray(j)
+    return (j <= t) & ((j < block_size) | (j // block_size == t // block_size))
+
+
+def attend(q, k, v, scale: float, allowed=None) -> Tuple[np.ndarray, np.ndarray]:
+    """Softmax attention of rows q [R, d] over keys k, v [N, d], in float64.
+
+    This is one host's local attention in Phase 2 (hotaipapers.com page, Phase 2
+    paragraph): it returns the output vector o [R, d] and the scalar
+    lse [R] = ln sum_j exp(s_j) over the keys where `allowed` [R, N] is true.
+    A row that sees no key returns o = 0 and lse = -inf.
+    """
+    q = np.asarray(q, dtype=F64)
+    k = np.asarray(k, dtype=F64)
+    v = np.asarray(v, dtype=F64)
+    s = scale * (q @ k.T)
+    if allowed is not None:
+        s = np.where(allowed, s, -np.inf)
+    m = s.max(axis=1) if s.shape[1] else np.full(s.shape[0], -np.inf)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    e = np.exp(s - m_safe[:, None])
+    l = e.sum(axis=1)
+    empty = l == 0
+    l_safe = np.where(empty, 1.0, l)
+    o = (e @ v) / l_safe[:, None]
+    lse = m_safe + np.log(l_safe)
+    o[empty] = 0.0
+    lse[empty] = -np.inf
+    return o, lse
+
+
+def lse_merge(o_parts, lse_parts) -> Tuple[np.ndarray, np.ndarray]:
+    """Query-host aggregation of per-block partials (hotaipapers.com page,
+    Phase 2 paragraph: each host sends one vector and one scalar and the query
+    host combines them into global attention).
+
+    With partials (o_s, lse_s), s = 1..S, over disjoint key sets, the exact
+    attention over their union is
+        lse = M + ln sum_s exp(lse_s - M),   M = max_s lse_s
+        o   = sum_s exp(lse_s - lse) * o_s
+    Partials with lse_s = -inf (no visible key) weigh nothing.
+    o_parts: [S, ..., d], lse_parts: [S, ...].
+    """
+    o_parts = np.asarray(o_parts, dtype=F64)
+    lse_parts = np.asarray(lse_parts, dtype=F64)
+    M = lse_parts.max(axis=0)
+    M_safe = np.where(np.isfinite(M), M, 0.0)
+    w = np.exp(lse_parts - M_safe)
+    W = w.sum(axis=0)
+    empty = W == 0
+    W_safe = np.where(empty, 1.0, W)
+    lse = M_safe + np.log(W_safe)
+    o = (w[..., None] * o_parts).sum(axis=0) / W_safe[..., None]
+    lse = np.where(empty, -np.inf, lse)
+    o = np.where(empty[..., None], 0.0, o)
+    return o, lse
+
+
+def phase1_head(q, k, v, block_size: int, scale: float, rows: Sequence[int] = None):
+    """Phase 1 for one (batch, q-head): q [L, d] and its kv-head's k, v [L, d].
+
+    Each block b_i runs causal attention over [anchor = b_0 ; b_i] and keeps
+    only its own rows (hotaipapers.com page, Phase 1 paragraph). For the rows of
+    b_i the candidate keys are b_0 and b_i (every key `phase1_visible` can
+    allow); the mask then applies the definition exactly.
+    Returns o [R, d], lse [R] for `rows` (default: all L rows, in order).
+    """
+    L, d = q.shape[0], q.shape[1]
+    rows = np.arange(L) if rows is None else np.asarray(rows, dtype=np.int64)
+    o_out = np.zeros((len(rows), d), dtype=F64)
+    lse_out = np.zeros(len(rows), dtype=F64)
+    for start, end in block_plan(L, block_size):
+        sel = np.nonzero((rows >= start) & (rows < end))[0]
+        if sel.size == 0:
+            continue
+        if start == 0:
+            cand = np.arange(0, end)
+        else:
+            cand = np.concatenate([np.arange(0, block_size), np.arange(start, end)])
+        kc = np.asarray(k[cand], dtype=F64)
+        vc = np.asarray(v[cand], dtype=F64)
+        for c0 in range(0, sel.size, _ROW_CHUNK):
+            idx = sel[c0:c0 + _ROW_CHUNK]
+            t = rows[idx]
+            allowed = phase1_visible(t[:, None], cand[None, :], block_size)
+            o, lse = attend(q[t], kc, vc, scale, allowed)
+            o_out[idx] = o
+            lse_out[idx] = lse
+    return o_out, lse_out
+
+
+def phase1(q, k, v, block_size: int, scale: float = None):
+    """Phase 1 over whole tensors: q [b, L, Hq, d], k, v [b, L, Hkv, d].
+    Returns o [b, L, Hq, d] and lse [b, Hq, L] in float64."""
+    b, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    scale = default_scale(d) if scale is None else scale
+    o = np.zeros((b, L, Hq, d), dtype=F64)
+    lse = np.zeros((b, Hq, L), dtype=F64)
+    for bi in range(b):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            oh, lh = phase1_head(q[bi, :, h], k[bi, :, g], v[bi, :, g], block_size, scale)
+            o[bi, :, h] = oh
+            lse[bi, h] = lh
+    return o, lse
+
+
+def phase2_query_head(q, k_ctx, v_ctx, k_qry, v_qry, scale: float):
+    """Phase-2 query tokens by the definition: sequence-global attention
+    (abstract: query and response tokens attend to all prior cached tokens).
+    Query token j sees all L context keys and query keys 0..j.
+    q [Lq, d]; k_ctx, v_ctx [L, d]; k_qry, v_qry [Lq, d]. Returns o [Lq, d], lse [Lq].
+    """
+    L = k_ctx.shape[0]
+    Lq = q.shape[0]
+    keys = np.concatenate([np.asarray(k_ctx, F64), np.asarray(k_qry, F64)])
+    vals = np.concatenate([np.asarray(v_ctx, F64), np.asarray(v_qry, F64)])
+    c = np.arange(L + Lq)[None, :]
+    j = np.arange(Lq)[:, None]
+    allowed = (c < L) | (c - L <= j)
+    return attend(q, keys, vals, scale, allowed)
+
+
+def phase2_query_head_blockwise(q, k_ctx, v_ctx, k_qry, v_qry, block_size: int, scale: float):
+    """Phase-2 query tokens the way the pages compute them (hotaipapers.com page,
+    Phase 2 paragraph): every context block b_i returns (o_i, lse_i) of the query
+    over its own keys, the query host adds its own causal partial over the query
+    tokens' KV, and the partials are merged with `lse_merge`."""
+    L = k_ctx.shape[0]
+    Lq = q.shape[0]
+    o_parts, lse_parts = [], []
+    for start, end in block_plan(L, block_size):
+        o, lse = attend(q, k_ctx[start:end], v_ctx[start:end], scale)
+        o_parts.append(o)
+        lse_parts.append(lse)
+    causal = np.arange(Lq)[None, :] <= np.arange(Lq)[:, None]
+    o, lse = attend(q, k_qry, v_qry, scale, causal)
+    o_parts.append(o)
+    lse_parts.append(lse)
+    return lse_merge(np.stack(o_parts), np.stack(lse_parts))
+
+
+def phase2_query(q_qry, k_qry, v_qry, k_ctx, v_ctx, scale: float = None):
+    """Phase-2 query over whole tensors: q_qry [b, Lq, Hq, d], k_qry, v_qry
+    [b, Lq, Hkv, d], k_ctx, v_ctx [b, L, Hkv, d]. Returns o [b, Lq, Hq, d],
+    lse [b, Hq, Lq]. The query tokens' KV become cache rows 0..Lq-1."""
+    b, Lq, Hq, d = q_qry.shape
+    Hkv = k_ctx.shape[2]
+    scale = default_scale(d) if scale is None else scale
+    o = np.zeros((b, Lq, Hq, d), dtype=F64)
+    lse = np.zeros((b, Hq, Lq), dtype=F64)
+    for bi in range(b):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            oh, lh = phase2_query_head(q_qry[bi, :, h], k_ctx[bi, :, g], v_ctx[bi, :, g],
+                                       k_qry[bi, :, g], v_qry[bi, :, g], scale)
+            o[bi, :, h] = oh
+            lse[bi, h] = lh
+    return o, lse
+
+
+def phase2_decode_head(q, k_ctx, v_ctx, k_cache, v_cache, k_new, v_new, scale: float):
+    """One decode step for one (batch, q-head) (hotaipapers.com page, Phase 2
+    paragraph: the query host appends the new token's KV to its cache, and the
+    token attends globally). The token sees every context key, the cached query
+    and earlier decode keys (k_cache [n, d]) and its own new key.
+    q, k_new, v_new [d]. Returns o [d], lse (a float)."""
+    keys = np.concatenate([np.asarray(k_ctx, F64), np.asarray(k_cache, F64),
+                           np.asarray(k_new, F64)[None, :]])
+    vals = np.concatenate([np.asarray(v_ctx, F64), np.asarray(v_cache, F64),
+                           np.asarray(v_new, F64)[None, :]])
+    o, lse = attend(np.asarray(q, F64)[None, :], keys, vals, scale)
+    return o[0], lse[0]
+
+
+def phase2_decode(q_t, k_t, v_t, k_ctx, v_ctx, k_cache, v_cache, cache_len: int,
+                  scale: float = None):
+    """One decode step over whole tensors: q_t [b, 1, Hq, d], k_t, v_t
+    [b, 1, Hkv, d], caches [b, cap, Hkv, d] holding `cache_len` valid rows.
+    Returns o [b, 1, Hq, d], lse [b, Hq, 1] and copies of the caches with the new
+    token's KV appended at row cache_len."""
+    b, _, Hq, d = q_t.shape
+    Hkv = k_ctx.shape[2]
+    scale = default_scale(d) if scale is None else scale
+    o = np.zeros((b, 1, Hq, d), dtype=F64)
+    lse = np.zeros((b, Hq, 1), dtype=F64)
+    for bi in range(b):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            oh, lh = phase2_decode_head(q_t[bi, 0, h], k_ctx[bi, :, g], v_ctx[bi, :, g],
+                                        k_cache[bi, :cache_len, g], v_cache[bi, :cache_len, g],
+                                        k_t[bi, 0, g], v_t[bi, 0, g], scale)
+            o[bi, 0, h] = oh
+            lse[bi, h, 0] = lh
+    k_cache_new = np.array(k_cache, dtype=F64, copy=True)
+    v_cache_new = np.array(v_cache, dtype=F64, copy=True)
+    k_cache_new[:, cache_len] = np.asarray(k_t, F64)[:, 0]
+    v_cache_new[:, cache_len] = np.asarray(v_t, F64)[:, 0]
+    return o, lse, k_cache_new, v_cache_new
