@@ -1,0 +1,444 @@
+"""Benchmark of the Star Attention two-phase hot path on B200.
+
+One step = the whole path for one attention layer of the workload: Phase 1 over
+the context, Phase 2 for the query tokens, then every decode step (append +
+split-KV partials + merge). Inputs are seeded synthetic tensors already resident
+in HBM when timing starts. Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl star|reference]
+
+Multi-GPU runs (torchrun, one process per GPU) execute independent replicas of
+the workload (the path has no data-path exchange on one node's problem; each
+rank draws its own seeded inputs): weak scaling, timed as the max over ranks.
+`--impl reference` times the CPU oracle instead, on bounded samples of the same
+workload, extrapolated to the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "Phase-1 context tok/s & TFLOP/s; Phase-2 decode KV GB/s vs HBM peak"
+DEFAULT_WORKLOAD = "llama8b-32k"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p["bf16_tflops_sustained"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power = [], [], []
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        under = [s for s, p in zip(sm, power) if p > 0.35 * max(power or [1])] or sm
+        return {"sm_mhz": statistics.median(under) if under else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------ the GPU arm
+class Step:
+    """One whole hot-path pass over resident inputs, with CUDA events per phase."""
+
+    def __init__(self, w, x, device):
+        import block_sparse_attention_phase_b200 as sa
+        self.sa = sa
+        self.w, self.x = w, x
+        self.layer = sa.StarAttentionLayer(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                           w.ctx_len, w.block_size, w.cache_capacity, device=device)
+        b, L, hq, d = w.batch, w.ctx_len, w.num_q_heads, w.head_dim
+        self.o_ctx = torch.empty((b, L, hq, d), dtype=torch.bfloat16, device=device)
+        self.lse_ctx = torch.empty((b, hq, L), dtype=torch.float32, device=device)
+        self.o_q = torch.empty((b, w.query_len, hq, d), dtype=torch.bfloat16, device=device)
+        self.lse_q = torch.empty((b, hq, w.query_len), dtype=torch.float32, device=device)
+        self.o_dec = torch.empty((w.decode_steps, b, 1, hq, d), dtype=torch.bfloat16, device=device)
+        self.lse_dec = torch.empty((w.decode_steps, b, hq, 1), dtype=torch.float32, device=device)
+        self.flush = torch.empty(workloads.l2_flush_bytes(), dtype=torch.uint8, device=device)
+        self.events = None
+
+    def run(self, record: bool = False):
+        w, x, layer = self.w, self.x, self.layer
+        ev = []
+        self.flush.fill_(1)  # evict L2 between steps (buffer > 126 MB L2)
+
+        def mark():
+            if record:
+                e = torch.cuda.Event(enable_timing=True)
+                e.record()
+                ev.append(e)
+
+        mark()
+        layer.prefill(x["q_ctx"], x["k_ctx"], x["v_ctx"], o=self.o_ctx, lse=self.lse_ctx)
+        mark()
+        layer.query(x["q_qry"], x["k_qry"], x["v_qry"], o=self.o_q, lse=self.lse_q)
+        mark()
+        for t in range(w.decode_steps):
+            layer.decode(x["q_dec"][t], x["k_dec"][t], x["v_dec"][t], o=self.o_dec[t],
+                         lse=self.lse_dec[t])
+            mark()
+        if record:
+            self.events = ev
+
+    def phase_times_ms(self):
+        ev = self.events
+        p1 = ev[0].elapsed_time(ev[1])
+        q = ev[1].elapsed_time(ev[2])
+        dec = [ev[2 + t].elapsed_time(ev[3 + t]) for t in range(self.w.decode_steps)]
+        return p1, q, dec
+
+
+def decode_cold_ms(step: Step, reps: int = 1):
+    """Each decode call timed alone after an L2 flush (events on the launching stream)."""
+    w, x, layer = step.w, step.x, step.layer
+    layer.prefill(x["q_ctx"], x["k_ctx"], x["v_ctx"], o=step.o_ctx, lse=step.lse_ctx)
+    layer.query(x["q_qry"], x["k_qry"], x["v_qry"], o=step.o_q, lse=step.lse_q)
+    times = []
+    for t in range(w.decode_steps):
+        step.flush.fill_(2)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        layer.decode(x["q_dec"][t], x["k_dec"][t], x["v_dec"][t], o=step.o_dec[t],
+                     lse=step.lse_dec[t])
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return times
+
+
+def e2e_run(step: Step, steps: int):
+    """The same step through the public API with host buffers: pinned host -> device
+    copies of every input, the step, and device -> host copies of every output, all
+    inside the timed region."""
+    x = step.x
+    host_in = {k: v.cpu().pin_memory() for k, v in x.items()}
+    outs = [step.o_ctx, step.lse_ctx, step.o_q, step.lse_q, step.o_dec, step.lse_dec]
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        for k, v in host_in.items():
+            x[k].copy_(v, non_blocking=True)
+        step.run(record=False)
+        for o, h in zip(outs, host_out):
+            h.copy_(o, non_blocking=True)
+    t1.record()
+    t1.synchronize()
+    return t0.elapsed_time(t1) / steps, h2d, d2h
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def oracle_sample(w, x_cpu=None, min_seconds: float = 10.0, max_seconds: float = 30.0):
+    """Time the oracle (as it stands) on a bounded sample of the workload and
+    extrapolate to the whole step. Sample: Phase 1 for the last block of q-head 0,
+    Phase 2 for the query tokens of q-head 0, one decode step of q-head 0.
+    Returns (step_seconds_estimate, description, threads)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    gen = workloads.make_inputs(w, device="cpu") if x_cpu is None else x_cpu
+    L, B, d = w.ctx_len, w.block_size, w.head_dim
+    n = w.num_blocks
+    start = (n - 1) * B
+    q = gen["q_ctx"][0, :, 0].float().numpy()
+    k = gen["k_ctx"][0, :, 0].float().numpy()
+    v = gen["v_ctx"][0, :, 0].float().numpy()
+    rows = np.arange(start, L)
+    nb = L - start
+    sample_pairs = nb * (nb + 1) // 2 + (nb * B if n > 1 else 0)
+    total_pairs = w.phase1_flops() / (4.0 * d)
+    qq = gen["q_qry"][0, :, 0].float().numpy()
+    kq = gen["k_qry"][0, :, 0].float().numpy()
+    vq = gen["v_qry"][0, :, 0].float().numpy()
+    qd = gen["q_dec"][0, 0, 0, 0].float().numpy()
+    kd = gen["k_dec"][0, 0, 0, 0].float().numpy()
+    vd = gen["v_dec"][0, 0, 0, 0].float().numpy()
+    t_p1, t_q, t_d, reps = 0.0, 0.0, 0.0, 0
+    t_all = time.perf_counter()
+    while True:
+        a = time.perf_counter()
+        oracle.phase1_head(q, k, v, B, w.softmax_scale, rows)
+        b_ = time.perf_counter()
+        oracle.phase2_query_head(qq, k, v, kq, vq, w.softmax_scale)
+        c = time.perf_counter()
+        oracle.phase2_decode_head(qd, k, v, kq, vq, kd, vd, w.softmax_scale)
+        e = time.perf_counter()
+        t_p1 += b_ - a
+        t_q += c - b_
+        t_d += e - c
+        reps += 1
+        el = e - t_all
+        if el >= min_seconds or el + el / reps > max_seconds:
+            break
+    t_p1, t_q, t_d = t_p1 / reps, t_q / reps, t_d / reps
+    heads = w.batch * w.num_q_heads
+    est = t_p1 * total_pairs / sample_pairs + t_q * heads + t_d * heads * w.decode_steps
+    desc = (f"oracle float64 on one q-head: Phase-1 rows of the last block ({nb} rows), the "
+            f"{w.query_len} query rows and one decode row, {reps} repetition(s); extrapolated to "
+            f"the whole step by score pairs (Phase 1) and by heads x steps (Phase 2)")
+    return est, desc, threads
+
+
+# ------------------------------------------------------------------ main
+def setup_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def run_reference(args, w, world, rank):
+    """CPU oracle arm: rank 0 only; each step is one bounded sample."""
+    if rank != 0:
+        return 0
+    gen = workloads.make_inputs(w, device="cpu")
+    per_step = []
+    threads = 1
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        est, desc, threads = oracle_sample(w, gen, min_seconds=args.ref_seconds,
+                                           max_seconds=3 * args.ref_seconds)
+        if i >= args.warmup:
+            per_step.append(est)
+    step_s = statistics.median(per_step)
+    value = w.batch * w.ctx_len / step_s
+    line = {
+        "metric": METRIC, "impl": "reference", "value": value, "unit": "tok/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, **w.describe()},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.BY_NAME))
+    ap.add_argument("--impl", default="star", choices=["star", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = setup_dist(args)
+    w = workloads.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w, world, rank)
+
+    import block_sparse_attention_phase_b200 as sa
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    x = workloads.make_inputs(w, device=device, seed=w.seed + rank)
+    step = Step(w, x, device)
+    peaks = load_peaks()
+
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    launches0 = sa.launch_count()
+    p1_ms, q_ms, dec_ms = [], [], []
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step.run(record=True)
+        p1_ms.append(step.events)  # read after the timed region
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = sa.launch_count() - launches0
+    clk = clocks.stop()
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world, device)
+
+    phases = []
+    for evs in p1_ms:
+        step.events = evs
+        phases.append(step.phase_times_ms())
+    p1_list = [p[0] for p in phases]
+    q_list = [p[1] for p in phases]
+    dec_all = [t for p in phases for t in p[2]]
+
+    ms_per_step = elapsed_ms / args.steps
+    tokens = w.batch * w.ctx_len
+    value = world * tokens * args.steps / (elapsed_ms / 1e3)
+
+    flops = w.phase1_flops()
+    p1_avg = statistics.mean(p1_list)
+    p1_tflops = flops / (p1_avg / 1e3) / 1e12
+    kv_bytes = [w.decode_kv_bytes(t) for t in range(w.decode_steps)]
+    dec_avg = statistics.mean(dec_all)
+    dec_gbs = statistics.mean(kv_bytes) / (dec_avg / 1e3) / 1e9
+    cold = decode_cold_ms(step)
+    dec_cold_avg = statistics.mean(cold)
+    dec_cold_gbs = statistics.mean(kv_bytes) / (dec_cold_avg / 1e3) / 1e9
+
+    rl_p1 = {"bound": "tensor", "kernel": "phase1", "achieved": p1_tflops,
+             "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+             "frac": p1_tflops / peaks["bf16_tflops_sustained"],
+             "frac_of_burst": p1_tflops / peaks["bf16_tflops"],
+             "peak_kind": f"bf16 sustained ({peaks['source']})", "traffic": None,
+             "algorithmic_per_launch": flops, "avg_launch_ms": p1_avg}
+    rl_dec = {"bound": "hbm", "kernel": "phase2_decode (partials + merge)", "achieved": dec_cold_gbs,
+              "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dec_cold_gbs / peaks["hbm_gbs"],
+              "peak_kind": f"HBM copy ({peaks['source']})", "traffic": None,
+              "algorithmic_per_launch": statistics.mean(kv_bytes), "avg_launch_ms": dec_cold_avg,
+              "in_step_gbs": dec_gbs, "in_step_avg_launch_ms": dec_avg}
+    dominant = rl_p1 if p1_avg >= sum(dec_all) / args.steps else rl_dec
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = e2e_run(step, steps=min(args.steps, 3))
+        e2e_ms = max_over_ranks(e2e_ms, world, device)
+        e2e = {"value": world * tokens / (e2e_ms / 1e3), "unit": "tok/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        est, desc, threads = oracle_sample(w)
+        cpu = {"value": tokens / est, "unit": "tok/s", "cores": threads, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads,
+                       "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                       "ctx_len": w.ctx_len, "block_size": w.block_size,
+                       "query_len": w.query_len, "decode_steps": w.decode_steps,
+                       "planted_pairs": w.planted_pairs, "parallelism": f"replicas{world}",
+                       "l2": "256 MiB write before every step; every decode step reads "
+                             f"{w.decode_kv_bytes(0) / 1e6:.1f} MB of KV"},
+            "phase1": {"ms": p1_avg, "tok_s": tokens / (p1_avg / 1e3), "tflops": p1_tflops,
+                       "frac_sustained": rl_p1["frac"], "frac_burst": rl_p1["frac_of_burst"]},
+            "query": {"ms": statistics.mean(q_list)},
+            "decode": {"ms_per_token_in_step": dec_avg, "gbs_in_step": dec_gbs,
+                       "ms_per_token_cold": dec_cold_avg, "gbs_cold": dec_cold_gbs,
+                       "frac_hbm_cold": dec_cold_gbs / peaks["hbm_gbs"]},
+            "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac",
+                                                  "traffic")},
+            "roofline_kernel": dominant["kernel"],
+            "rooflines": {"phase1": rl_p1, "decode": rl_dec},
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+            "peaks": peaks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,298 @@
+"""Star Attention two-phase attention on B200 (sm_100a): Python binding.
+
+A thin ctypes layer over the C-ABI library libstarattn.so (include/star_attn.h).
+It only marshals arguments: it checks tensor dtypes/shapes, allocates outputs
+with torch (device memory is PyTorch's job here), and passes raw pointers and
+the current CUDA stream. Every step of the attention runs in the library's
+CUDA kernels; there is no fallback of any kind. If the library is missing the
+import of an entry point raises.
+
+Entry points mirror the C names:
+    phase1(q, k, v, block_size)                      -> (o, lse)
+    phase2_query(q, k, v, k_ctx, v_ctx, k_cache, v_cache, block_size) -> (o, lse)
+    phase2_decode(q, k, v, k_ctx, v_ctx, k_cache, v_cache, cache_len, block_size) -> (o, lse)
+    lse_merge(o_parts, lse_parts)                    -> (o, lse)
+and StarAttentionLayer bundles them with the caches and workspace of one layer.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libstarattn.so")
+
+STAR_PHASE1, STAR_PHASE2_QUERY, STAR_PHASE2_DECODE = 1, 2, 3
+STATUS_NAMES = {0: "STAR_OK", 1: "STAR_ERR_INVALID_ARG", 2: "STAR_ERR_UNSUPPORTED",
+                3: "STAR_ERR_WORKSPACE", 4: "STAR_ERR_CACHE_FULL", 5: "STAR_ERR_CUDA",
+                6: "STAR_ERR_TIMEOUT"}
+
+# Every symbol the header declares; tests check that the library exports them all.
+EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase2_query",
+            "star_attn_phase2_decode", "star_attn_lse_merge", "star_attn_simple_phase1",
+            "star_attn_simple_phase2", "star_attn_get_device_status",
+            "star_attn_selftest_wait_timeout", "star_attn_launch_count", "star_attn_status_string",
+            "star_attn_version"]
+
+
+class StarAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("ctx_len", ctypes.c_int64), ("block_size", ctypes.c_int64),
+                ("softmax_scale", ctypes.c_float)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libstarattn.so (built in-tree by block_sparse_attention_phase_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m block_sparse_attention_phase_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    SP = ctypes.POINTER(Shape)
+    sig = {
+        "star_attn_workspace_bytes": (SZ, [SP, I32, I64]),
+        "star_attn_phase1": (I32, [SP, P, P, P, P, P, P]),
+        "star_attn_phase2_query": (I32, [SP, P, P, P, I64, P, P, P, P, I64, P, P, P, SZ, P]),
+        "star_attn_phase2_decode": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P, SZ, P]),
+        "star_attn_lse_merge": (I32, [P, P, I32, I32, I64, I32, I32, P, P, P]),
+        "star_attn_simple_phase1": (I32, [SP, P, P, P, P, P, P]),
+        "star_attn_simple_phase2": (I32, [SP, P, I64, P, P, P, P, I64, I64, I32, P, P, P]),
+        "star_attn_get_device_status": (I32, [P]),
+        "star_attn_selftest_wait_timeout": (I32, [ctypes.c_uint64, P]),
+        "star_attn_launch_count": (ctypes.c_uint64, []),
+        "star_attn_status_string": (ctypes.c_char_p, [I32]),
+        "star_attn_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise StarAttnError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _bf16(t: torch.Tensor, name: str, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor, got {tuple(t.shape)}")
+
+
+def make_shape(batch, num_q_heads, num_kv_heads, head_dim, ctx_len, block_size,
+               softmax_scale: Optional[float] = None) -> Shape:
+    return Shape(batch, num_q_heads, num_kv_heads, head_dim, ctx_len, block_size,
+                 0.0 if softmax_scale is None else float(softmax_scale))
+
+
+def workspace_bytes(shape: Shape, phase: int, rows: int = 1) -> int:
+    return int(lib().star_attn_workspace_bytes(ctypes.byref(shape), phase, rows))
+
+
+def _ctx_shape(q, k, block_size, scale) -> Shape:
+    b, L, hq, d = q.shape
+    return make_shape(b, hq, k.shape[2], d, L, block_size, scale)
+
+
+def phase1(q, k, v, block_size: int, scale: Optional[float] = None, o=None, lse=None,
+           want_lse: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Anchor-prefixed blockwise-local causal attention over the context.
+    q [b, L, Hq, d], k/v [b, L, Hkv, d] bf16 -> o [b, L, Hq, d] bf16, lse [b, Hq, L] fp32."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bf16(t, n, 4)
+    shape = _ctx_shape(q, k, block_size, scale)
+    b, L, hq, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((b, hq, L), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_phase1(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                  _ptr(lse), _stream()), "star_attn_phase1")
+    return o, lse
+
+
+def _ws(shape: Shape, phase: int, rows: int, device, workspace):
+    need = workspace_bytes(shape, phase, rows)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    return workspace
+
+
+def phase2_query(q, k, v, k_ctx, v_ctx, k_cache, v_cache, block_size: int,
+                 scale: Optional[float] = None, o=None, lse=None, workspace=None):
+    """Query tokens: q [b, Lq, Hq, d], k/v [b, Lq, Hkv, d]; context KV [b, L, Hkv, d];
+    caches [b, cap, Hkv, d] (rows 0..Lq-1 are written). Returns (o, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (k_ctx, "k_ctx"), (v_ctx, "v_ctx"),
+                 (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _bf16(t, n, 4)
+    b, lq, hq, d = q.shape
+    shape = make_shape(b, hq, k_ctx.shape[2], d, k_ctx.shape[1], block_size, scale)
+    workspace = _ws(shape, STAR_PHASE2_QUERY, lq, q.device, workspace)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((b, hq, lq), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_phase2_query(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), lq, _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(k_cache), _ptr(v_cache), k_cache.shape[1], _ptr(o), _ptr(lse), _ptr(workspace),
+        workspace.numel(), _stream()), "star_attn_phase2_query")
+    return o, lse
+
+
+def phase2_decode(q, k, v, k_ctx, v_ctx, k_cache, v_cache, cache_len: int, block_size: int,
+                  scale: Optional[float] = None, o=None, lse=None, workspace=None):
+    """One decode step: q [b, 1, Hq, d], k/v [b, 1, Hkv, d]; the token's KV is appended at
+    cache row cache_len and it attends to context + cache rows 0..cache_len."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (k_ctx, "k_ctx"), (v_ctx, "v_ctx"),
+                 (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _bf16(t, n, 4)
+    b, _, hq, d = q.shape
+    shape = make_shape(b, hq, k_ctx.shape[2], d, k_ctx.shape[1], block_size, scale)
+    workspace = _ws(shape, STAR_PHASE2_DECODE, 1, q.device, workspace)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((b, hq, 1), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_phase2_decode(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_cache),
+        _ptr(v_cache), int(cache_len), k_cache.shape[1], _ptr(o), _ptr(lse), _ptr(workspace),
+        workspace.numel(), _stream()), "star_attn_phase2_decode")
+    return o, lse
+
+
+def lse_merge(o_parts: torch.Tensor, lse_parts: torch.Tensor):
+    """o_parts [S, b, T, H, d] fp32, lse_parts [S, b, H, T] fp32 -> (o bf16 [b, T, H, d], lse)."""
+    S, b, T, H, d = o_parts.shape
+    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
+        raise TypeError("partials must be float32")
+    o_parts = o_parts.contiguous()
+    lse_parts = lse_parts.contiguous()
+    o = torch.empty((b, T, H, d), dtype=torch.bfloat16, device=o_parts.device)
+    lse = torch.empty((b, H, T), dtype=torch.float32, device=o_parts.device)
+    _check(lib().star_attn_lse_merge(_ptr(o_parts), _ptr(lse_parts), S, b, T, H, d, _ptr(o),
+                                     _ptr(lse), _stream()), "star_attn_lse_merge")
+    return o, lse
+
+
+def simple_phase1(q, k, v, block_size: int, scale: Optional[float] = None):
+    """Cross-check kernel (one warp per row) for Phase 1; same contract as phase1()."""
+    shape = _ctx_shape(q, k, block_size, scale)
+    b, L, hq, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((b, hq, L), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_simple_phase1(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                         _ptr(lse), _stream()), "star_attn_simple_phase1")
+    return o, lse
+
+
+def simple_phase2(q, k_ctx, v_ctx, k_cache, v_cache, block_size: int, visible_base: int,
+                  causal: bool, scale: Optional[float] = None):
+    """Cross-check kernel for Phase 2: row r sees all context keys and cache rows
+    0..visible_base + (r if causal else 0). The cache must already hold those rows."""
+    b, rows, hq, d = q.shape
+    shape = make_shape(b, hq, k_ctx.shape[2], d, k_ctx.shape[1], block_size, scale)
+    o = torch.empty_like(q)
+    lse = torch.empty((b, hq, rows), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_simple_phase2(
+        ctypes.byref(shape), _ptr(q), rows, _ptr(k_ctx), _ptr(v_ctx), _ptr(k_cache),
+        _ptr(v_cache), k_cache.shape[1], visible_base, 1 if causal else 0, _ptr(o), _ptr(lse),
+        _stream()), "star_attn_simple_phase2")
+    return o, lse
+
+
+def device_status() -> int:
+    """Synchronise the current stream and return (and clear) the device status."""
+    return int(lib().star_attn_get_device_status(_stream()))
+
+
+def selftest_wait_timeout(wait_ns: int = 20_000_000) -> None:
+    _check(lib().star_attn_selftest_wait_timeout(int(wait_ns), _stream()),
+           "star_attn_selftest_wait_timeout")
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process."""
+    return int(lib().star_attn_launch_count())
+
+
+def version() -> str:
+    return lib().star_attn_version().decode()
+
+
+class StarAttentionLayer:
+    """One attention layer's Star Attention state on one GPU: the context KV from
+    Phase 1, the query-local cache, and the Phase-2 workspace (allocated once).
+
+        layer = StarAttentionLayer(batch, Hq, Hkv, d, ctx_len, block_size, cache_capacity)
+        o_ctx = layer.prefill(q, k, v)          # Phase 1; keeps k, v as the context KV
+        o_q = layer.query(q_q, k_q, v_q)        # Phase 2, query tokens
+        o_t = layer.decode(q_t, k_t, v_t)       # Phase 2, one decode step (repeat)
+    """
+
+    def __init__(self, batch, num_q_heads, num_kv_heads, head_dim, ctx_len, block_size,
+                 cache_capacity, device="cuda", scale: Optional[float] = None):
+        self.shape = make_shape(batch, num_q_heads, num_kv_heads, head_dim, ctx_len, block_size,
+                                scale)
+        self.block_size = block_size
+        self.scale = scale
+        self.k_cache = torch.empty((batch, cache_capacity, num_kv_heads, head_dim),
+                                   dtype=torch.bfloat16, device=device)
+        self.v_cache = torch.empty_like(self.k_cache)
+        self.cache_len = 0
+        self.k_ctx = self.v_ctx = None
+        self.ws_decode = torch.empty(max(256, workspace_bytes(self.shape, STAR_PHASE2_DECODE)),
+                                     dtype=torch.uint8, device=device)
+        self.ws_query = None
+
+    def prefill(self, q, k, v, o=None, lse=None):
+        self.k_ctx, self.v_ctx = k, v
+        self.cache_len = 0
+        return phase1(q, k, v, self.block_size, self.scale, o=o, lse=lse)
+
+    def query(self, q, k, v, o=None, lse=None):
+        lq = q.shape[1]
+        need = workspace_bytes(self.shape, STAR_PHASE2_QUERY, lq)
+        if self.ws_query is None or self.ws_query.numel() < need:
+            self.ws_query = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+        out = phase2_query(q, k, v, self.k_ctx, self.v_ctx, self.k_cache, self.v_cache,
+                           self.block_size, self.scale, o=o, lse=lse, workspace=self.ws_query)
+        self.cache_len = lq
+        return out
+
+    def decode(self, q, k, v, o=None, lse=None):
+        out = phase2_decode(q, k, v, self.k_ctx, self.v_ctx, self.k_cache, self.v_cache,
+                            self.cache_len, self.block_size, self.scale, o=o, lse=lse,
+                            workspace=self.ws_decode)
+        self.cache_len += 1
+        return out

@@ -1,0 +1,90 @@
+// Exact merge of split-KV attention partials (the query host's aggregation in
+// Star Attention's Phase 2: hotaipapers.com page, Phase 2 paragraph — every
+// block returns one vector and one scalar).
+//
+// For one output row with partials (o_s, lse_s):
+//   M = max_s lse_s,  W = sum_s exp(lse_s - M),  lse = M + ln W,
+//   o = sum_s exp(lse_s - M) o_s / W
+// A split whose lse_s is -inf (it saw no key) contributes nothing.
+// One warp per (batch, token, head); lanes own D/32 consecutive elements, so
+// every partial row is read with one coalesced 128-/256-byte access.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "star_internal.h"
+
+namespace star {
+namespace {
+
+constexpr int kWarps = 8;
+
+template <int D>
+__global__ void __launch_bounds__(kWarps * 32) merge_kernel(
+    const float* __restrict__ o_parts, const float* __restrict__ lse_parts, int32_t S, int32_t b,
+    int64_t T, int32_t H, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  const int64_t rows = static_cast<int64_t>(b) * T * H;
+  if (row >= rows) return;
+  const int h = static_cast<int>(row % H);
+  const int64_t t = (row / H) % T;
+  const int bb = static_cast<int>(row / (static_cast<int64_t>(H) * T));
+  // lse_parts[s][bb][h][t]; o_parts[s][bb][t][h][:]
+  const int64_t lse_stride = static_cast<int64_t>(b) * H * T;
+  const int64_t lse_off = (static_cast<int64_t>(bb) * H + h) * T + t;
+  const int64_t o_stride = static_cast<int64_t>(b) * T * H * D;
+  const int64_t o_off = ((static_cast<int64_t>(bb) * T + t) * H + h) * D + lane * E;
+
+  float M = -INFINITY;
+  for (int sidx = lane; sidx < S; sidx += 32) M = fmaxf(M, lse_parts[sidx * lse_stride + lse_off]);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+
+  float W = 0.f;
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  if (M != -INFINITY) {
+    for (int sidx = 0; sidx < S; ++sidx) {
+      const float ls = lse_parts[sidx * lse_stride + lse_off];
+      const float w = expf(ls - M);  // exp(-inf) = 0 for an empty split
+      W += w;
+      const float* src = o_parts + sidx * o_stride + o_off;
+      if constexpr (E == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src);
+        acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(src);
+        acc[0] += w * x.x; acc[1] += w * x.y;
+      }
+    }
+  }
+  const float inv = W > 0.f ? 1.f / W : 0.f;
+  __nv_bfloat16* dst = o + ((static_cast<int64_t>(bb) * T + t) * H + h) * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; ++e) dst[e] = __float2bfloat16_rn(acc[e] * inv);
+  if (lse && lane == 0) lse[lse_off] = W > 0.f ? M + logf(W) : -INFINITY;
+}
+
+}  // namespace
+
+cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int32_t n_splits,
+                         int32_t b, int64_t tokens, int32_t heads, int32_t d, void* o,
+                         float* lse, cudaStream_t st) {
+  const int64_t rows = static_cast<int64_t>(b) * tokens * heads;
+  if (rows == 0) return cudaSuccess;
+  const dim3 grid(static_cast<unsigned>((rows + kWarps - 1) / kWarps));
+  auto* oo = static_cast<__nv_bfloat16*>(o);
+  if (d == 128)
+    merge_kernel<128><<<grid, kWarps * 32, 0, st>>>(o_parts, lse_parts, n_splits, b, tokens,
+                                                    heads, oo, lse);
+  else
+    merge_kernel<64><<<grid, kWarps * 32, 0, st>>>(o_parts, lse_parts, n_splits, b, tokens,
+                                                   heads, oo, lse);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace star

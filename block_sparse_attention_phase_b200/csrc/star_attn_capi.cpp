@@ -1,0 +1,261 @@
+// C-ABI layer: argument validation, Phase-2 split planning, workspace sizing and
+// launch sequencing. Nothing here computes attention; every step of the path
+// runs in the kernels of the .cu files.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/star_attn.h"
+#include "star_internal.h"
+
+namespace star {
+namespace {
+
+constexpr int kSMs = 148;              // B200
+constexpr int kDecodeCtasPerSM = 2;
+constexpr int64_t kMinChunk = 64;      // one TMA tile of keys
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+star_status_t resolve(const star_attn_shape_t* in, Shape* out) {
+  if (!in) return STAR_ERR_INVALID_ARG;
+  if (in->batch < 1 || in->num_q_heads < 1 || in->num_kv_heads < 1 || in->ctx_len < 1 ||
+      in->block_size < 1)
+    return STAR_ERR_INVALID_ARG;
+  if (in->num_q_heads % in->num_kv_heads != 0) return STAR_ERR_INVALID_ARG;
+  if (!(in->softmax_scale == in->softmax_scale)) return STAR_ERR_INVALID_ARG;  // NaN
+  if (in->head_dim != 64 && in->head_dim != 128) return STAR_ERR_UNSUPPORTED;
+  const int G = in->num_q_heads / in->num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return STAR_ERR_UNSUPPORTED;
+  if (in->ctx_len > (int64_t{1} << 31) - 1) return STAR_ERR_UNSUPPORTED;  // TMA coordinates
+  out->b = in->batch;
+  out->hq = in->num_q_heads;
+  out->hkv = in->num_kv_heads;
+  out->d = in->head_dim;
+  out->L = in->ctx_len;
+  out->B = in->block_size < in->ctx_len ? in->block_size : in->ctx_len;
+  out->scale = in->softmax_scale > 0.f ? in->softmax_scale
+                                       : static_cast<float>(1.0 / std::sqrt(double(in->head_dim)));
+  return STAR_OK;
+}
+
+star_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? STAR_OK : STAR_ERR_CUDA; }
+
+SplitPlan make_plan(const Shape& s, int64_t target_ctas) {
+  SplitPlan p;
+  const int64_t n = s.n_blocks();
+  const int64_t units = static_cast<int64_t>(s.b) * s.hkv;
+  int64_t per_unit = target_ctas / units - 1;  // context splits wanted per (batch, kv-head)
+  int64_t spb = per_unit / n;
+  if (spb < 1) spb = 1;
+  int64_t chunk = (s.B + spb - 1) / spb;
+  if (chunk < kMinChunk) {
+    chunk = kMinChunk;
+    spb = (s.B + chunk - 1) / chunk;
+  }
+  p.spb = static_cast<int32_t>(spb);
+  p.chunk = chunk;
+  p.n_ctx = static_cast<int32_t>(n * spb);
+  p.n_splits = p.n_ctx + 1;
+  return p;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+std::atomic<uint64_t> g_launches{0};
+
+}  // namespace
+
+void count_launch(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+SplitPlan decode_plan(const Shape& s) { return make_plan(s, int64_t{kSMs} * kDecodeCtasPerSM); }
+
+SplitPlan query_plan(const Shape& s, int64_t lq) {
+  (void)lq;
+  return make_plan(s, int64_t{kSMs} * kDecodeCtasPerSM);
+}
+
+size_t partial_bytes(const Shape& s, const SplitPlan& p, int64_t rows) {
+  const size_t per = static_cast<size_t>(p.n_splits) * s.b * rows * s.hq;
+  return align256(per * s.d * sizeof(float)) + align256(per * sizeof(float));
+}
+
+}  // namespace star
+
+using star::Shape;
+
+extern "C" {
+
+STAR_ATTN_API uint64_t star_attn_launch_count(void) {
+  return star::g_launches.load(std::memory_order_relaxed);
+}
+
+STAR_ATTN_API const char* star_attn_version(void) { return "star-attn-b200 0.1 (sm_100a)"; }
+
+STAR_ATTN_API const char* star_attn_status_string(star_status_t st) {
+  switch (st) {
+    case STAR_OK: return "ok";
+    case STAR_ERR_INVALID_ARG: return "invalid argument";
+    case STAR_ERR_UNSUPPORTED: return "unsupported shape";
+    case STAR_ERR_WORKSPACE: return "workspace missing or too small";
+    case STAR_ERR_CACHE_FULL: return "query-local cache full";
+    case STAR_ERR_CUDA: return "CUDA error";
+    case STAR_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+STAR_ATTN_API size_t star_attn_workspace_bytes(const star_attn_shape_t* shape, int32_t phase,
+                                               int64_t rows) {
+  Shape s;
+  if (star::resolve(shape, &s) != STAR_OK) return 0;
+  switch (phase) {
+    case STAR_PHASE1: return 0;
+    case STAR_PHASE2_QUERY:
+      if (rows < 1) return 0;
+      return star::partial_bytes(s, star::query_plan(s, rows), rows);
+    case STAR_PHASE2_DECODE: return star::partial_bytes(s, star::decode_plan(s), 1);
+    default: return 0;
+  }
+}
+
+STAR_ATTN_API star_status_t star_attn_phase1(const star_attn_shape_t* shape, const void* q,
+                                             const void* k, const void* v, void* o, float* lse,
+                                             star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (!q || !k || !v || !o) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned16(q) || !star::aligned16(k) || !star::aligned16(v) || !star::aligned16(o) ||
+      !star::aligned16(lse))
+    return STAR_ERR_INVALID_ARG;
+  return star::cuda_status(
+      star::launch_phase1_sm100(s, q, k, v, o, lse, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+STAR_ATTN_API star_status_t star_attn_phase2_query(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
+    int64_t query_len, const void* k_ctx, const void* v_ctx, void* k_cache, void* v_cache,
+    int64_t cache_capacity, void* o, float* lse, void* workspace, size_t workspace_bytes,
+    star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (query_len < 1 || cache_capacity < 1) return STAR_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, k_ctx, v_ctx, k_cache, v_cache, o};
+  for (const void* p : ptrs)
+    if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned16(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
+  if (query_len > cache_capacity) return STAR_ERR_CACHE_FULL;
+  const star::SplitPlan plan = star::query_plan(s, query_len);
+  const size_t need = star::partial_bytes(s, plan, query_len);
+  if (!workspace || workspace_bytes < need) return STAR_ERR_WORKSPACE;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = star::launch_cache_write(s, k, v, query_len, k_cache, v_cache, cache_capacity, 0, cs);
+  if (e != cudaSuccess) return STAR_ERR_CUDA;
+  float* o_parts = static_cast<float*>(workspace);
+  const size_t per = static_cast<size_t>(plan.n_splits) * s.b * query_len * s.hq;
+  float* lse_parts = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                              ((per * s.d * sizeof(float) + 255) & ~size_t(255)));
+  e = star::launch_query_path(s, plan, q, query_len, k_ctx, v_ctx, k_cache, v_cache,
+                              cache_capacity, o_parts, lse_parts, o, lse, cs);
+  return star::cuda_status(e);
+}
+
+STAR_ATTN_API star_status_t star_attn_phase2_decode(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
+    const void* k_ctx, const void* v_ctx, void* k_cache, void* v_cache, int64_t cache_len,
+    int64_t cache_capacity, void* o, float* lse, void* workspace, size_t workspace_bytes,
+    star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (cache_len < 0 || cache_capacity < 1) return STAR_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, k_ctx, v_ctx, k_cache, v_cache, o};
+  for (const void* p : ptrs)
+    if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned16(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
+  if (cache_len + 1 > cache_capacity) return STAR_ERR_CACHE_FULL;
+  const star::SplitPlan plan = star::decode_plan(s);
+  const size_t need = star::partial_bytes(s, plan, 1);
+  if (!workspace || workspace_bytes < need) return STAR_ERR_WORKSPACE;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  float* o_parts = static_cast<float*>(workspace);
+  const size_t per = static_cast<size_t>(plan.n_splits) * s.b * s.hq;
+  float* lse_parts = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                              ((per * s.d * sizeof(float) + 255) & ~size_t(255)));
+  cudaError_t e = star::launch_decode_partials(s, plan, q, k, v, k_ctx, v_ctx, k_cache, v_cache,
+                                               cache_len, cache_capacity, o_parts, lse_parts, cs);
+  if (e != cudaSuccess) return STAR_ERR_CUDA;
+  e = star::launch_merge(o_parts, lse_parts, plan.n_splits, s.b, 1, s.hq, s.d, o, lse, cs);
+  return star::cuda_status(e);
+}
+
+STAR_ATTN_API star_status_t star_attn_lse_merge(const float* o_parts, const float* lse_parts,
+                                                int32_t num_splits, int32_t batch,
+                                                int64_t tokens, int32_t heads, int32_t head_dim,
+                                                void* o, float* lse, star_stream_t stream) {
+  if (!o_parts || !lse_parts || !o) return STAR_ERR_INVALID_ARG;
+  if (num_splits < 1 || batch < 1 || tokens < 1 || heads < 1) return STAR_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return STAR_ERR_UNSUPPORTED;
+  if (!star::aligned16(o_parts) || !star::aligned16(o)) return STAR_ERR_INVALID_ARG;
+  return star::cuda_status(star::launch_merge(o_parts, lse_parts, num_splits, batch, tokens,
+                                              heads, head_dim, o, lse,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+STAR_ATTN_API star_status_t star_attn_simple_phase1(const star_attn_shape_t* shape,
+                                                    const void* q, const void* k, const void* v,
+                                                    void* o, float* lse, star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (!q || !k || !v || !o) return STAR_ERR_INVALID_ARG;
+  return star::cuda_status(star::launch_simple_phase1(s, q, k, v, o, lse,
+                                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+STAR_ATTN_API star_status_t star_attn_simple_phase2(
+    const star_attn_shape_t* shape, const void* q, int64_t rows, const void* k_ctx,
+    const void* v_ctx, const void* k_cache, const void* v_cache, int64_t cache_capacity,
+    int64_t cache_visible_base, int32_t causal, void* o, float* lse, star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (!q || !k_ctx || !v_ctx || !k_cache || !v_cache || !o || rows < 1 || cache_capacity < 1 ||
+      cache_visible_base < 0)
+    return STAR_ERR_INVALID_ARG;
+  return star::cuda_status(star::launch_simple_phase2(
+      s, q, rows, k_ctx, v_ctx, k_cache, v_cache, cache_capacity, cache_visible_base, causal, o,
+      lse, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+STAR_ATTN_API star_status_t star_attn_get_device_status(star_stream_t stream) {
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return STAR_ERR_CUDA;
+  uint32_t* word = star::device_status_word();
+  if (!word) return STAR_ERR_CUDA;
+  uint32_t flags = 0;
+  if (cudaMemcpy(&flags, word, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return STAR_ERR_CUDA;
+  if (flags) {
+    const uint32_t zero = 0;
+    if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return STAR_ERR_CUDA;
+  }
+  if (flags & star::kTimeoutFlag) return STAR_ERR_TIMEOUT;
+  if (flags) return STAR_ERR_CUDA;
+  return STAR_OK;
+}
+
+STAR_ATTN_API star_status_t star_attn_selftest_wait_timeout(uint64_t wait_ns,
+                                                            star_stream_t stream) {
+  if (wait_ns < 1000000ull) wait_ns = 1000000ull;
+  if (wait_ns > 2000000000ull) wait_ns = 2000000000ull;
+  return star::cuda_status(
+      star::launch_selftest_wait(wait_ns, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

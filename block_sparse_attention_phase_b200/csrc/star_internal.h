@@ -1,0 +1,83 @@
+// Internal interface between the C-ABI layer (star_attn_capi.cpp) and the
+// kernel launchers in the .cu files. Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#if defined(__CUDACC__)
+#define STAR_HD __host__ __device__
+#else
+#define STAR_HD
+#endif
+
+namespace star {
+
+// Flags kernels OR into the device status word (they never trap).
+constexpr uint32_t kTimeoutFlag = 1u;  // a bounded wait ran out
+constexpr uint32_t kBoundsFlag = 2u;   // a bounds check refused an access
+
+struct Shape {
+  int32_t b, hq, hkv, d;
+  int64_t L, B;
+  float scale;  // resolved softmax scale (> 0)
+  STAR_HD int64_t n_blocks() const { return (L + B - 1) / B; }
+  STAR_HD int32_t group() const { return hq / hkv; }
+};
+
+// Split plan of a Phase-2 pass: every context block is cut into `spb` chunks of
+// at most `chunk` keys (a chunk never straddles two blocks); one more split
+// covers the query-local cache.
+struct SplitPlan {
+  int32_t spb = 1;
+  int64_t chunk = 1;
+  int32_t n_ctx = 0;    // n_blocks * spb
+  int32_t n_splits = 0; // n_ctx + 1
+};
+
+SplitPlan decode_plan(const Shape& s);
+SplitPlan query_plan(const Shape& s, int64_t lq);
+size_t partial_bytes(const Shape& s, const SplitPlan& p, int64_t rows);
+
+// Counts kernel launches (host side); every launcher calls it once per launch.
+void count_launch(uint64_t n = 1);
+
+// Device status word of the current device (address valid on that device).
+uint32_t* device_status_word();
+
+// ---- launchers (return the launch's cudaError_t) ----
+cudaError_t launch_simple_phase1(const Shape& s, const void* q, const void* k, const void* v,
+                                 void* o, float* lse, cudaStream_t st);
+cudaError_t launch_simple_phase2(const Shape& s, const void* q, int64_t rows, const void* kc,
+                                 const void* vc, const void* kk, const void* vk, int64_t cap,
+                                 int64_t vis_base, int causal, void* o, float* lse,
+                                 cudaStream_t st);
+cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int32_t n_splits,
+                         int32_t b, int64_t tokens, int32_t heads, int32_t d, void* o,
+                         float* lse, cudaStream_t st);
+cudaError_t launch_cache_write(const Shape& s, const void* k, const void* v, int64_t rows,
+                               void* kc, void* vc, int64_t cap, int64_t row0, cudaStream_t st);
+cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const void* q,
+                                   const void* k_new, const void* v_new, const void* kc,
+                                   const void* vc, void* k_cache, void* v_cache, int64_t cache_len,
+                                   int64_t cap, float* o_parts, float* lse_parts,
+                                   cudaStream_t st);
+cudaError_t launch_phase1_sm100(const Shape& s, const void* q, const void* k, const void* v,
+                                void* o, float* lse, cudaStream_t st);
+// Phase-2 query tokens after their KV is in the cache: partials + merge into o/lse.
+cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q, int64_t lq,
+                              const void* kc, const void* vc, const void* k_cache,
+                              const void* v_cache, int64_t cap, float* o_parts, float* lse_parts,
+                              void* o, float* lse, cudaStream_t st);
+cudaError_t launch_selftest_wait(uint64_t wait_ns, cudaStream_t st);
+
+// TMA descriptor encoding (host). Returns false if the driver entry point is
+// unavailable or the encode call rejects the arguments.
+// 4-D bf16 tensor [outer3][outer2][outer1][inner0] viewed as
+// (inner0 = d, dim1 = heads, dim2 = tokens, dim3 = batch), box (box0, 1, box2, 1).
+bool encode_tma_bf16_4d(void* tmap_out, const void* base, uint64_t d, uint64_t heads,
+                        uint64_t tokens, uint64_t batch, uint32_t box0, uint32_t box2,
+                        bool swizzle128);
+
+}  // namespace star

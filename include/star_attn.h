@@ -1,0 +1,206 @@
+/*
+ * star_attn.h — C ABI of the B200 (sm_100a) Star Attention two-phase attention library.
+ *
+ * The method is Star Attention ("Star Attention: Efficient LLM Inference over
+ * Long Sequences", Acharya, Jia, Ginsburg; ICML 2025). On one GPU the pages'
+ * "hosts" become context blocks resident in HBM:
+ *
+ *   Phase 1 (context prefill): the context of L tokens is cut into blocks
+ *     b_0..b_{n-1} of B tokens (n = ceil(L/B), the last block may be short).
+ *     Block b_0 runs plain causal attention; every block b_i, i > 0, runs causal
+ *     attention over [anchor = b_0 ; b_i] and keeps only its own rows
+ *     (hotaipapers.com page, Phase 1 paragraph; rebuttal to reviewer EMsM,
+ *     "Size of Anchor Block"). The anchor is read in place from b_0's K/V.
+ *   Phase 2 (query and decode): each query or decoded token attends to every
+ *     cached token. Every context block returns a partial output and its
+ *     log-sum-exp; the partials are merged exactly (hotaipapers.com page, Phase 2
+ *     paragraph). The query tokens' K/V and each decoded token's K/V are
+ *     appended to a query-local cache.
+ *
+ * Conventions for every call
+ *   - Q/K/V/O are bf16, contiguous, token-major: [batch, tokens, heads, head_dim].
+ *   - LSE outputs are fp32 [batch, num_q_heads, rows], natural log of the sum of
+ *     exp(softmax_scale * q.k) over the row's visible keys.
+ *   - GQA: q-head h reads kv-head h / (num_q_heads / num_kv_heads).
+ *   - All pointers are device pointers owned by the caller and must be 16-byte
+ *     aligned. The library never allocates device memory and never frees a
+ *     caller's buffer; any scratch it needs is the caller's `workspace`.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *     Arguments are checked on the host before anything is launched; an invalid
+ *     call returns an error and launches nothing. No C++ exception crosses the ABI.
+ *   - Kernels never trap. A device-side wait that runs out (about one second)
+ *     records a flag that star_attn_get_device_status() reports.
+ */
+#ifndef STAR_ATTN_H_
+#define STAR_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define STAR_ATTN_API __attribute__((visibility("default")))
+#else
+#define STAR_ATTN_API
+#endif
+
+/* Same type as cudaStream_t, declared here so that this header needs no CUDA headers. */
+struct CUstream_st;
+typedef struct CUstream_st* star_stream_t;
+
+typedef enum {
+  STAR_OK = 0,
+  STAR_ERR_INVALID_ARG = 1,  /* null or misaligned pointer, inconsistent shape */
+  STAR_ERR_UNSUPPORTED = 2,  /* a shape this build does not implement (head_dim not 64/128) */
+  STAR_ERR_WORKSPACE = 3,    /* workspace missing or smaller than star_attn_workspace_bytes() */
+  STAR_ERR_CACHE_FULL = 4,   /* the query-local cache has no room for the rows to append */
+  STAR_ERR_CUDA = 5,         /* a CUDA runtime call or a kernel launch failed */
+  STAR_ERR_TIMEOUT = 6       /* a bounded device-side wait ran out (see get_device_status) */
+} star_status_t;
+
+/* Problem shape shared by all calls. */
+typedef struct {
+  int32_t batch;          /* sequences, >= 1; every sequence has the same ctx_len */
+  int32_t num_q_heads;    /* Hq >= 1 */
+  int32_t num_kv_heads;   /* Hkv >= 1, Hq % Hkv == 0 */
+  int32_t head_dim;       /* d: 64 or 128 */
+  int64_t ctx_len;        /* L >= 1 context tokens */
+  int64_t block_size;     /* B >= 1; also the anchor size (rebuttal to EMsM) */
+  float softmax_scale;    /* <= 0 selects 1/sqrt(head_dim) */
+} star_attn_shape_t;
+
+/* Phase selectors for star_attn_workspace_bytes(). */
+enum { STAR_PHASE1 = 1, STAR_PHASE2_QUERY = 2, STAR_PHASE2_DECODE = 3 };
+
+/*
+ * Workspace (device scratch) a call needs, in bytes; 0 if none.
+ * phase: STAR_PHASE1, STAR_PHASE2_QUERY (rows = query_len) or STAR_PHASE2_DECODE
+ * (rows ignored). The workspace holds the per-split fp32 partial outputs and
+ * LSEs of Phase 2 before they are merged. Returns 0 for an invalid shape.
+ */
+STAR_ATTN_API size_t star_attn_workspace_bytes(const star_attn_shape_t* shape, int32_t phase,
+                                               int64_t rows);
+
+/*
+ * Phase 1: anchor-prefixed blockwise-local causal attention over the context
+ * (hotaipapers.com page, Phase 1 paragraph; rebuttal to EMsM, "Size of Anchor
+ * Block"; rebuttal to x5MA, "Anchor Block Content and Position").
+ *
+ * For token t of block b_i (i = t / B) the visible keys are b_0 (all of it,
+ * if i > 0) and the tokens of b_i up to t:
+ *   o[t]   = sum_j softmax_j(scale * q_t . k_j) v_j,   lse[t] = ln sum_j exp(scale * q_t . k_j)
+ * q [batch, L, Hq, d]; k, v [batch, L, Hkv, d]  (inputs, read only; k and v of
+ *   every block are kept by the caller as that block's KV cache)
+ * o [batch, L, Hq, d] bf16 (output, round-to-nearest-even from fp32)
+ * lse [batch, Hq, L] fp32 (output) or NULL.
+ * Needs no workspace.
+ */
+STAR_ATTN_API star_status_t star_attn_phase1(const star_attn_shape_t* shape, const void* q,
+                                             const void* k, const void* v, void* o, float* lse,
+                                             star_stream_t stream);
+
+/*
+ * Phase 2, query tokens (abstract: query tokens attend to all prior cached
+ * tokens; hotaipapers.com page, Phase 2 paragraph).
+ *
+ * Writes the query tokens' k, v into cache rows [0, query_len) and computes,
+ * for query token j, attention over all L context keys and cache rows 0..j.
+ * Each context block contributes a partial (o_s, lse_s); the query-local cache
+ * contributes a causal partial; they are merged as in star_attn_lse_merge().
+ *   q [batch, Lq, Hq, d]; k, v [batch, Lq, Hkv, d]   query tokens (inputs)
+ *   k_ctx, v_ctx [batch, L, Hkv, d]                   Phase-1 context KV (inputs)
+ *   k_cache, v_cache [batch, cache_capacity, Hkv, d]  query-local cache (rows 0..Lq-1 written)
+ *   o [batch, Lq, Hq, d] bf16, lse [batch, Hq, Lq] fp32 or NULL (outputs)
+ *   workspace: at least star_attn_workspace_bytes(shape, STAR_PHASE2_QUERY, query_len) bytes.
+ * Errors: STAR_ERR_CACHE_FULL if query_len > cache_capacity.
+ */
+STAR_ATTN_API star_status_t star_attn_phase2_query(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
+    int64_t query_len, const void* k_ctx, const void* v_ctx, void* k_cache, void* v_cache,
+    int64_t cache_capacity, void* o, float* lse, void* workspace, size_t workspace_bytes,
+    star_stream_t stream);
+
+/*
+ * Phase 2, one decode step (hotaipapers.com page, Phase 2 paragraph: the query
+ * host appends the new token's KV to its cache and the token attends globally).
+ *
+ * Appends k, v at cache row cache_len, then computes attention of q over all L
+ * context keys and cache rows 0..cache_len (its own new key included), as a
+ * split-KV pass over every block plus the cache, merged exactly.
+ *   q [batch, 1, Hq, d]; k, v [batch, 1, Hkv, d]      new token (inputs)
+ *   k_ctx, v_ctx [batch, L, Hkv, d]                    context KV (inputs)
+ *   k_cache, v_cache [batch, cache_capacity, Hkv, d]   rows 0..cache_len-1 valid; row cache_len written
+ *   o [batch, 1, Hq, d] bf16, lse [batch, Hq, 1] fp32 or NULL (outputs)
+ *   workspace: at least star_attn_workspace_bytes(shape, STAR_PHASE2_DECODE, 1) bytes.
+ * Errors: STAR_ERR_CACHE_FULL if cache_len + 1 > cache_capacity.
+ */
+STAR_ATTN_API star_status_t star_attn_phase2_decode(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
+    const void* k_ctx, const void* v_ctx, void* k_cache, void* v_cache, int64_t cache_len,
+    int64_t cache_capacity, void* o, float* lse, void* workspace, size_t workspace_bytes,
+    star_stream_t stream);
+
+/*
+ * Exact merge of per-split attention partials (hotaipapers.com page, Phase 2
+ * paragraph: every host sends one vector and one scalar to the query host).
+ *   lse = M + ln sum_s exp(lse_s - M),  M = max_s lse_s
+ *   o   = sum_s exp(lse_s - lse) o_s          (a split with lse_s = -inf weighs 0)
+ * o_parts [num_splits, batch, tokens, heads, head_dim] fp32,
+ * lse_parts [num_splits, batch, heads, tokens] fp32 (inputs);
+ * o [batch, tokens, heads, head_dim] bf16, lse [batch, heads, tokens] fp32 or NULL (outputs).
+ * head_dim: 64 or 128.
+ */
+STAR_ATTN_API star_status_t star_attn_lse_merge(const float* o_parts, const float* lse_parts,
+                                                int32_t num_splits, int32_t batch,
+                                                int64_t tokens, int32_t heads, int32_t head_dim,
+                                                void* o, float* lse, star_stream_t stream);
+
+/*
+ * Straightforward CUDA kernels (one warp per output row, fp32) computing the
+ * same three operations with final outputs directly. They are a second,
+ * independent GPU implementation used to cross-check the fast kernels at sizes
+ * the CPU oracle cannot cover; they are not the fast path.
+ */
+STAR_ATTN_API star_status_t star_attn_simple_phase1(const star_attn_shape_t* shape,
+                                                    const void* q, const void* k, const void* v,
+                                                    void* o, float* lse, star_stream_t stream);
+STAR_ATTN_API star_status_t star_attn_simple_phase2(
+    const star_attn_shape_t* shape, const void* q, int64_t rows, const void* k_ctx,
+    const void* v_ctx, const void* k_cache, const void* v_cache, int64_t cache_capacity,
+    int64_t cache_visible_base, int32_t causal, void* o, float* lse, star_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns STAR_ERR_TIMEOUT if any kernel on the
+ * current device recorded an expired bounded wait since the previous call
+ * (clearing the flag), STAR_ERR_CUDA if the stream reports a CUDA error, else
+ * STAR_OK.
+ */
+STAR_ATTN_API star_status_t star_attn_get_device_status(star_stream_t stream);
+
+/*
+ * Self-test of the bounded-wait path: launches one block that waits on a
+ * shared-memory barrier nobody arrives at, with a limit of `wait_ns`
+ * nanoseconds (clamped to [1 ms, 2 s]); the wait gives up, records the timeout
+ * flag and the block exits normally. The caller then reads the flag with
+ * star_attn_get_device_status(). Faults nothing and leaves the context usable.
+ */
+STAR_ATTN_API star_status_t star_attn_selftest_wait_timeout(uint64_t wait_ns,
+                                                            star_stream_t stream);
+
+/*
+ * Number of kernels this library has launched in this process (all devices).
+ * A host-side counter for accounting, incremented at every successful launch.
+ */
+STAR_ATTN_API uint64_t star_attn_launch_count(void);
+
+STAR_ATTN_API const char* star_attn_status_string(star_status_t status);
+STAR_ATTN_API const char* star_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STAR_ATTN_H_ */

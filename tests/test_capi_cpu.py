@@ -1,0 +1,107 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, exports every
+symbol include/star_attn.h declares, sizes workspaces, and rejects bad arguments
+before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_phase_b200 as sa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    text = open(os.path.join(ROOT, "include", "star_attn.h")).read()
+    return sorted(set(re.findall(r"STAR_ATTN_API\s+[\w\s\*]+?\b(star_attn_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = sa.lib()
+    names = header_symbols()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(sa.EXPORTED) == names
+
+
+def test_version_and_status_strings():
+    assert "sm_100a" in sa.version()
+    L = sa.lib()
+    for code in range(7):
+        assert L.star_attn_status_string(code)
+    assert L.star_attn_status_string(6) == b"device-side wait timed out"
+
+
+def test_workspace_bytes():
+    s = sa.make_shape(1, 32, 8, 128, 32768, 4096)
+    assert sa.workspace_bytes(s, sa.STAR_PHASE1) == 0
+    dec = sa.workspace_bytes(s, sa.STAR_PHASE2_DECODE)
+    q = sa.workspace_bytes(s, sa.STAR_PHASE2_QUERY, 64)
+    # fp32 partial outputs + LSEs: (d + 1) floats per split per (row, head)
+    assert dec >= 32 * 129 * 4 * 9 and dec % 256 == 0
+    assert q >= 64 * dec // 2
+    assert sa.workspace_bytes(s, sa.STAR_PHASE2_QUERY, 0) == 0
+    bad = sa.make_shape(1, 32, 6, 128, 1024, 128)  # Hq % Hkv != 0
+    assert sa.workspace_bytes(bad, sa.STAR_PHASE2_DECODE) == 0
+
+
+def _call_phase1(shape, ptrs):
+    L = sa.lib()
+    p = [ctypes.c_void_p(x) for x in ptrs]
+    return L.star_attn_phase1(ctypes.byref(shape) if shape is not None else None, *p, None)
+
+
+FAKE = 1 << 20  # aligned, never dereferenced: every call below is rejected on the host
+
+
+@pytest.mark.parametrize("shape_args,code", [
+    ((1, 4, 3, 128, 100, 10), 1),    # Hq % Hkv != 0
+    ((1, 4, 2, 96, 100, 10), 2),     # head_dim 96 unsupported
+    ((1, 12, 4, 128, 100, 10), 2),   # GQA group 3 unsupported
+    ((0, 4, 2, 128, 100, 10), 1),    # batch 0
+    ((1, 4, 2, 128, 0, 10), 1),      # empty context
+    ((1, 4, 2, 128, 100, 0), 1),     # block size 0
+])
+def test_phase1_rejects_bad_shapes(shape_args, code):
+    assert _call_phase1(sa.make_shape(*shape_args), [FAKE, FAKE, FAKE, FAKE, FAKE]) == code
+
+
+def test_phase1_rejects_null_and_misaligned():
+    s = sa.make_shape(1, 4, 2, 128, 100, 10)
+    assert _call_phase1(None, [FAKE] * 5) == 1
+    assert _call_phase1(s, [0, FAKE, FAKE, FAKE, FAKE]) == 1
+    assert _call_phase1(s, [FAKE + 2, FAKE, FAKE, FAKE, FAKE]) == 1
+    assert _call_phase1(s, [FAKE, FAKE, FAKE, FAKE, FAKE + 8]) == 1  # misaligned lse
+
+
+def test_phase2_rejects_cache_and_workspace_errors():
+    L = sa.lib()
+    s = sa.make_shape(1, 4, 2, 128, 100, 10)
+    F = ctypes.c_void_p(FAKE)
+    need = sa.workspace_bytes(s, sa.STAR_PHASE2_DECODE)
+    # decode: cache_len + 1 > capacity
+    assert L.star_attn_phase2_decode(ctypes.byref(s), F, F, F, F, F, F, F, 8, 8, F, None, F,
+                                     need, None) == 4
+    # decode: workspace too small
+    assert L.star_attn_phase2_decode(ctypes.byref(s), F, F, F, F, F, F, F, 3, 8, F, None, F,
+                                     need - 1, None) == 3
+    assert L.star_attn_phase2_decode(ctypes.byref(s), F, F, F, F, F, F, F, 3, 8, F, None, None,
+                                     need, None) == 3
+    # query: more query tokens than cache rows
+    needq = sa.workspace_bytes(s, sa.STAR_PHASE2_QUERY, 16)
+    assert L.star_attn_phase2_query(ctypes.byref(s), F, F, F, 16, F, F, F, F, 8, F, None, F,
+                                    needq, None) == 4
+    assert L.star_attn_phase2_query(ctypes.byref(s), F, F, F, 4, F, F, F, F, 8, F, None, F,
+                                    0, None) == 3
+    # merge: bad sizes
+    assert L.star_attn_lse_merge(F, F, 0, 1, 1, 1, 128, F, None, None) == 1
+    assert L.star_attn_lse_merge(F, F, 2, 1, 1, 1, 80, F, None, None) == 2
+
+
+def test_binding_checks_tensors_before_calling():
+    import torch
+    q = torch.zeros(1, 8, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        sa.phase1(q, q, q, 4)  # CPU tensors are refused: there is no CPU path

@@ -1,0 +1,213 @@
+"""GPU parity: the CUDA path (through the C-ABI) against the float64 CPU oracle.
+
+Small shapes are compared row for row; they span several tiles, ragged last
+blocks, one-block and one-token-block contexts, GQA groups 1/2/4/8, head_dim
+64/128 and batch 2. The five named workloads run at full size in the launch
+configuration the benchmark times; there the oracle checks sampled rows (block
+edges, tile edges, planted rows, random rows) for Phase 1 and every row of
+sampled heads for Phase 2.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.parity_util import check_rows, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def sa():
+    import block_sparse_attention_phase_b200 as m
+    return m
+
+
+def make(b, hq, hkv, d, L, B, lq, T, seed=0, plants=0):
+    w = workloads.Workload("case", b, hq, hkv, d, L, B, lq, T, plants, seed)
+    return w, workloads.make_inputs(w, device="cuda")
+
+
+SMALL = [
+    # b, Hq, Hkv, d, L, B, Lq, T
+    (1, 2, 2, 64, 2048, 512, 16, 8),     # the tiny workload
+    (1, 4, 2, 128, 1000, 300, 5, 3),     # ragged last block, B not a tile multiple
+    (2, 8, 1, 64, 700, 256, 3, 2),       # GQA group 8, batch 2
+    (1, 4, 1, 128, 200, 512, 4, 2),      # L < B: one block, plain causal attention
+    (1, 2, 2, 128, 512, 256, 1, 2),      # two blocks, Lq = 1
+    (1, 2, 1, 64, 40, 1, 2, 2),          # B = 1: every block is one token
+    (1, 4, 4, 128, 450, 100, 7, 2),      # B < tile
+    (1, 2, 2, 64, 1, 1, 1, 1),           # L = 1
+    (1, 16, 4, 128, 384, 128, 130, 3),   # Lq > one tile of query rows
+]
+
+
+def _run_small(case):
+    b, hq, hkv, d, L, B, lq, T = case
+    w, x = make(*case)
+    m = sa()
+    # ---------------- Phase 1
+    o, lse = m.phase1(x["q_ctx"], x["k_ctx"], x["v_ctx"], B)
+    ro, rl = oracle.phase1(to_np(x["q_ctx"]), to_np(x["k_ctx"]), to_np(x["v_ctx"]), B)
+    check_rows(to_np(o), ro, to_np(lse), rl, f"phase1 {case}")
+    # ---------------- Phase 2: query
+    cap = lq + T
+    kc = torch.full((b, cap, hkv, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vc = torch.full_like(kc, float("nan"))  # rows not yet written hold NaN on purpose
+    oq, lq_lse = m.phase2_query(x["q_qry"], x["k_qry"], x["v_qry"], x["k_ctx"], x["v_ctx"],
+                                kc, vc, B)
+    rq, rql = oracle.phase2_query(to_np(x["q_qry"]), to_np(x["k_qry"]), to_np(x["v_qry"]),
+                                  to_np(x["k_ctx"]), to_np(x["v_ctx"]))
+    check_rows(to_np(oq), rq, to_np(lq_lse), rql, f"query {case}")
+    assert torch.equal(kc[:, :lq], x["k_qry"]) and torch.equal(vc[:, :lq], x["v_qry"])
+    # ---------------- Phase 2: decode steps
+    k_cache = np.zeros((b, cap, hkv, d))
+    v_cache = np.zeros((b, cap, hkv, d))
+    k_cache[:, :lq] = to_np(x["k_qry"])
+    v_cache[:, :lq] = to_np(x["v_qry"])
+    for t in range(T):
+        od, ld = m.phase2_decode(x["q_dec"][t], x["k_dec"][t], x["v_dec"][t], x["k_ctx"],
+                                 x["v_ctx"], kc, vc, lq + t, B)
+        ro_d, rl_d, k_cache, v_cache = oracle.phase2_decode(
+            to_np(x["q_dec"][t]), to_np(x["k_dec"][t]), to_np(x["v_dec"][t]), to_np(x["k_ctx"]),
+            to_np(x["v_ctx"]), k_cache, v_cache, lq + t)
+        check_rows(to_np(od), ro_d, to_np(ld), rl_d, f"decode {case} t={t}")
+        assert torch.equal(kc[:, lq + t], x["k_dec"][t][:, 0])
+    assert m.device_status() == 0
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "x".join(map(str, c)))
+def test_small_shapes_all_rows(case):
+    _run_small(case)
+
+
+def test_phase1_deterministic():
+    w, x = make(1, 4, 2, 128, 1500, 512, 1, 1, seed=3)
+    m = sa()
+    o1, l1 = m.phase1(x["q_ctx"], x["k_ctx"], x["v_ctx"], 512)
+    o2, l2 = m.phase1(x["q_ctx"], x["k_ctx"], x["v_ctx"], 512)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_lse_merge_kernel_against_oracle():
+    g = torch.Generator(device="cpu").manual_seed(5)
+    S, b, T, H, d = 7, 2, 3, 4, 128
+    o_parts = torch.randn(S, b, T, H, d, generator=g)
+    lse_parts = torch.randn(S, b, H, T, generator=g) * 3
+    lse_parts[2] = float("-inf")  # an empty split
+    o, lse = sa().lse_merge(o_parts.cuda(), lse_parts.cuda())
+    ro, rl = oracle.lse_merge(o_parts.numpy().transpose(0, 1, 3, 2, 4),
+                              lse_parts.numpy())  # oracle wants [S, b, H, T, d]
+    check_rows(to_np(o).transpose(0, 2, 1, 3), ro, to_np(lse), rl, "merge")
+
+
+def test_simple_kernels_agree_with_oracle():
+    w, x = make(1, 4, 2, 64, 600, 200, 4, 1, seed=7)
+    m = sa()
+    o, l = m.simple_phase1(x["q_ctx"], x["k_ctx"], x["v_ctx"], 200)
+    ro, rl = oracle.phase1(to_np(x["q_ctx"]), to_np(x["k_ctx"]), to_np(x["v_ctx"]), 200)
+    check_rows(to_np(o), ro, to_np(l), rl, "simple phase1")
+    cap = 8
+    kc = torch.zeros((1, cap, 2, 64), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    kc[:, :4], vc[:, :4] = x["k_qry"], x["v_qry"]
+    o, l = m.simple_phase2(x["q_qry"], x["k_ctx"], x["v_ctx"], kc, vc, 200, 0, True)
+    rq, rql = oracle.phase2_query(to_np(x["q_qry"]), to_np(x["k_qry"]), to_np(x["v_qry"]),
+                                  to_np(x["k_ctx"]), to_np(x["v_ctx"]))
+    check_rows(to_np(o), rq, to_np(l), rql, "simple phase2")
+
+
+def test_wait_timeout_is_reported_not_trapped():
+    m = sa()
+    assert m.device_status() == 0
+    m.selftest_wait_timeout(20_000_000)  # 20 ms
+    assert m.device_status() == 6        # STAR_ERR_TIMEOUT, then cleared
+    assert m.device_status() == 0
+    # the context is still usable
+    t = torch.ones(4, device="cuda")
+    assert float(t.sum()) == 4.0
+
+
+# ------------------------------------------------------------------ full-size workloads
+def _sample_rows(w, rng, extra=()):
+    L, B = w.ctx_len, w.block_size
+    rows = set(extra)
+    for start, end in oracle.block_plan(L, B):
+        for t in (start, start + 1, start + 127, start + 128, end - 129, end - 128, end - 1):
+            if start <= t < end:
+                rows.add(t)
+    rows.update(int(t) for t in rng.integers(0, L, size=96))
+    return np.array(sorted(rows))
+
+
+def _phase1_sampled(w, x, o, lse, heads):
+    rng = np.random.default_rng(11)
+    plants = [p for p in workloads.plan_plants(w) if p.q_where == "ctx"]
+    for bb in range(w.batch):
+        for h in heads:
+            g = oracle.kv_head_of(h, w.num_q_heads, w.num_kv_heads)
+            extra = [p.q_token for p in plants if p.batch == bb and p.q_head == h]
+            rows = _sample_rows(w, rng, extra)
+            q = x["q_ctx"][bb, :, h].float().cpu().numpy()
+            k = x["k_ctx"][bb, :, g].float().cpu().numpy()
+            v = x["v_ctx"][bb, :, g].float().cpu().numpy()
+            ro, rl = oracle.phase1_head(q, k, v, w.block_size, w.softmax_scale, rows)
+            rows_t = torch.as_tensor(rows, device="cuda")
+            check_rows(to_np(o[bb, rows_t, h]), ro, to_np(lse[bb, h, rows_t]), rl,
+                       f"{w.name} phase1 b={bb} h={h}")
+
+
+def _phase2_sampled(w, x, heads, steps):
+    m = sa()
+    b, hkv, d, lq = w.batch, w.num_kv_heads, w.head_dim, w.query_len
+    kc = torch.zeros((b, w.cache_capacity, hkv, d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    oq, lql = m.phase2_query(x["q_qry"], x["k_qry"], x["v_qry"], x["k_ctx"], x["v_ctx"], kc, vc,
+                             w.block_size)
+    outs = {}
+    for t in range(max(steps) + 1):
+        outs[t] = m.phase2_decode(x["q_dec"][t], x["k_dec"][t], x["v_dec"][t], x["k_ctx"],
+                                  x["v_ctx"], kc, vc, lq + t, w.block_size)
+    torch.cuda.synchronize()
+    for bb in range(b):
+        for h in heads:
+            g = oracle.kv_head_of(h, w.num_q_heads, hkv)
+            kctx = x["k_ctx"][bb, :, g].float().cpu().numpy()
+            vctx = x["v_ctx"][bb, :, g].float().cpu().numpy()
+            kq = x["k_qry"][bb, :, g].float().cpu().numpy()
+            vq = x["v_qry"][bb, :, g].float().cpu().numpy()
+            ro, rl = oracle.phase2_query_head(x["q_qry"][bb, :, h].float().cpu().numpy(), kctx,
+                                              vctx, kq, vq, w.softmax_scale)
+            check_rows(to_np(oq[bb, :, h]), ro, to_np(lql[bb, h]), rl,
+                       f"{w.name} query b={bb} h={h}")
+            kd = x["k_dec"][:, bb, 0, g].float().cpu().numpy()
+            vd = x["v_dec"][:, bb, 0, g].float().cpu().numpy()
+            for t in steps:
+                ro, rl = oracle.phase2_decode_head(
+                    x["q_dec"][t, bb, 0, h].float().cpu().numpy(), kctx, vctx,
+                    np.concatenate([kq, kd[:t]]), np.concatenate([vq, vd[:t]]), kd[t], vd[t],
+                    w.softmax_scale)
+                od, ld = outs[t]
+                check_rows(to_np(od[bb, 0, h])[None], ro[None], to_np(ld[bb, h, 0:1]),
+                           np.array([rl]), f"{w.name} decode t={t} b={bb} h={h}")
+
+
+FULL = ["llama8b-32k", "llama8b-128k", "70b-128k", "1m"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workload(name):
+    w = workloads.get(name)
+    x = workloads.make_inputs(w, device="cuda")
+    m = sa()
+    o, lse = m.phase1(x["q_ctx"], x["k_ctx"], x["v_ctx"], w.block_size)
+    torch.cuda.synchronize()
+    G = w.group
+    plant_heads = sorted({p.q_head for p in workloads.plan_plants(w)})
+    heads = sorted({0, w.num_q_heads - 1, G} | set(plant_heads[:2]))
+    _phase1_sampled(w, x, o, lse, heads[:3] if name == "1m" else heads)
+    del o, lse
+    _phase2_sampled(w, x, heads, steps=[0, 1, w.decode_steps - 1])
+    assert m.device_status() == 0
