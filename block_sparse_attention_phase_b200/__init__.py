@@ -33,7 +33,7 @@ STATUS_NAMES = {0: "STAR_OK", 1: "STAR_ERR_INVALID_ARG", 2: "STAR_ERR_UNSUPPORTE
 
 # Every symbol the header declares; tests check that the library exports them all.
 EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase2_query",
-            "star_attn_phase2_decode", "star_attn_lse_merge", "star_attn_simple_phase1",
+            "star_attn_phase2_decode", "star_attn_phase2_decode_noalloc", "star_attn_lse_merge", "star_attn_simple_phase1",
             "star_attn_simple_phase2", "star_attn_get_device_status",
             "star_attn_selftest_wait_timeout", "star_attn_launch_count", "star_attn_status_string",
             "star_attn_version"]
@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
         "star_attn_phase1": (I32, [SP, P, P, P, P, P, P]),
         "star_attn_phase2_query": (I32, [SP, P, P, P, I64, P, P, P, P, I64, P, P, P, SZ, P]),
         "star_attn_phase2_decode": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P, SZ, P]),
+        "star_attn_phase2_decode_noalloc": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P]),
         "star_attn_lse_merge": (I32, [P, P, I32, I32, I64, I32, I32, P, P, P]),
         "star_attn_simple_phase1": (I32, [SP, P, P, P, P, P, P]),
         "star_attn_simple_phase2": (I32, [SP, P, I64, P, P, P, P, I64, I64, I32, P, P, P]),

@@ -144,6 +144,29 @@ STAR_ATTN_API star_status_t star_attn_phase2_decode(
     star_stream_t stream);
 
 /*
+ * The decode step of star_attn_phase2_decode() for callers that cannot allocate
+ * device memory where they decode (a serving runtime whose pooled allocator owns
+ * all of the GPU's memory, code that must avoid the implicit synchronisation of
+ * cudaMalloc/cudaFree, C callers with no allocator at hand). No counterpart on
+ * the Star Attention pages: this is a deployment variant of the same step.
+ *
+ * Same arguments and results as star_attn_phase2_decode() minus the workspace:
+ * the per-split partials go to a 4 MiB array compiled into the library (one per
+ * GPU, held until the process exits). The call allocates nothing.
+ *   - The first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress) with that device current; make it before any
+ *     stream capture.
+ *   - Every call shares the array: calls that may overlap on one GPU (e.g. on
+ *     two streams) race and must be ordered by the caller.
+ *   - Returns STAR_ERR_WORKSPACE, launching nothing, when the shape's partials
+ *     (star_attn_workspace_bytes(shape, STAR_PHASE2_DECODE, 1)) exceed 4 MiB.
+ */
+STAR_ATTN_API star_status_t star_attn_phase2_decode_noalloc(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
+    const void* k_ctx, const void* v_ctx, void* k_cache, void* v_cache, int64_t cache_len,
+    int64_t cache_capacity, void* o, float* lse, star_stream_t stream);
+
+/*
  * Exact merge of per-split attention partials (hotaipapers.com page, Phase 2
  * paragraph: every host sends one vector and one scalar to the query host).
  *   lse = M + ln sum_s exp(lse_s - M),  M = max_s lse_s
