@@ -363,10 +363,10 @@ cudaError_t launch_decode_t(const Shape& s, const SplitPlan& p, const DecodeArgs
   constexpr int W = 8;
   constexpr int NST = 3;
   alignas(64) CUtensorMap m[4];
-  const bool ok = encode_tma_bf16_4d(&m[0], kc, D, s.hkv, s.L, s.b, D, kTile, false) &&
-                  encode_tma_bf16_4d(&m[1], vc, D, s.hkv, s.L, s.b, D, kTile, false) &&
-                  encode_tma_bf16_4d(&m[2], a.k_cache, D, s.hkv, a.cap, s.b, D, kTile, false) &&
-                  encode_tma_bf16_4d(&m[3], a.v_cache, D, s.hkv, a.cap, s.b, D, kTile, false);
+  const bool ok = encode_tma_bf16_4d(&m[0], kc, D, s.hkv, s.L, s.L, s.b, D, 1, kTile, false) &&
+                  encode_tma_bf16_4d(&m[1], vc, D, s.hkv, s.L, s.L, s.b, D, 1, kTile, false) &&
+                  encode_tma_bf16_4d(&m[2], a.k_cache, D, s.hkv, a.cap, a.cap, s.b, D, 1, kTile, false) &&
+                  encode_tma_bf16_4d(&m[3], a.v_cache, D, s.hkv, a.cap, a.cap, s.b, D, 1, kTile, false);
   if (!ok) return cudaErrorInvalidValue;
   const size_t smem = 2 * NST * kTile * D * 2 + 2 * NST * sizeof(uint64_t);
   auto kern = decode_partials_kernel<D, G, W, NST>;

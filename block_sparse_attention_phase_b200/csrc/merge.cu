@@ -6,10 +6,13 @@
 //   M = max_s lse_s,  W = sum_s exp(lse_s - M),  lse = M + ln W,
 //   o = sum_s exp(lse_s - M) o_s / W
 // A split whose lse_s is -inf (it saw no key) contributes nothing.
-// One warp per (batch, token, head); lanes own D/32 consecutive elements, so
-// every partial row is read with one coalesced 128-/256-byte access.
+//
+// One CTA of 8 warps per (batch, token, head). The warps take the splits in
+// turn (warp w: splits w, w+8, ...), each lane owning d/32 contiguous elements of
+// every partial row (coalesced 128-/256-byte reads), so the S partial rows are
+// read with 8-way parallelism instead of one after another; the warps' sums meet
+// in shared memory.
 #include <cuda_bf16.h>
-#include <math_constants.h>
 
 #include "common.cuh"
 #include "star_internal.h"
@@ -24,10 +27,12 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(
     const float* __restrict__ o_parts, const float* __restrict__ lse_parts, int32_t S, int32_t b,
     int64_t T, int32_t H, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
   constexpr int E = D / 32;
+  __shared__ float red[kWarps];
+  __shared__ float acc_s[kWarps][D];
+  __shared__ float wsum_s[kWarps];
   const int lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-  const int64_t rows = static_cast<int64_t>(b) * T * H;
-  if (row >= rows) return;
+  const int warp = threadIdx.x >> 5;
+  const int64_t row = blockIdx.x;  // (bb, t, h) with h fastest
   const int h = static_cast<int>(row % H);
   const int64_t t = (row / H) % T;
   const int bb = static_cast<int>(row / (static_cast<int64_t>(H) * T));
@@ -37,21 +42,27 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(
   const int64_t o_stride = static_cast<int64_t>(b) * T * H * D;
   const int64_t o_off = ((static_cast<int64_t>(bb) * T + t) * H + h) * D + lane * E;
 
+  // M = max over splits
   float M = -INFINITY;
-  for (int sidx = lane; sidx < S; sidx += 32) M = fmaxf(M, lse_parts[sidx * lse_stride + lse_off]);
+  for (int s = threadIdx.x; s < S; s += kWarps * 32) M = fmaxf(M, lse_parts[s * lse_stride + lse_off]);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = red[0];
+#pragma unroll
+  for (int w = 1; w < kWarps; ++w) M = fmaxf(M, red[w]);
 
   float W = 0.f;
   float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
   if (M != -INFINITY) {
-    for (int sidx = 0; sidx < S; ++sidx) {
-      const float ls = lse_parts[sidx * lse_stride + lse_off];
-      const float w = expf(ls - M);  // exp(-inf) = 0 for an empty split
+#pragma unroll 2
+    for (int s = warp; s < S; s += kWarps) {
+      const float w = expf(lse_parts[s * lse_stride + lse_off] - M);  // 0 for an empty split
       W += w;
-      const float* src = o_parts + sidx * o_stride + o_off;
+      const float* src = o_parts + s * o_stride + o_off;
       if constexpr (E == 4) {
         const float4 x = *reinterpret_cast<const float4*>(src);
         acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
@@ -61,11 +72,25 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(
       }
     }
   }
-  const float inv = W > 0.f ? 1.f / W : 0.f;
-  __nv_bfloat16* dst = o + ((static_cast<int64_t>(bb) * T + t) * H + h) * D + lane * E;
 #pragma unroll
-  for (int e = 0; e < E; ++e) dst[e] = __float2bfloat16_rn(acc[e] * inv);
-  if (lse && lane == 0) lse[lse_off] = W > 0.f ? M + logf(W) : -INFINITY;
+  for (int e = 0; e < E; ++e) acc_s[warp][lane * E + e] = acc[e];
+  if (lane == 0) wsum_s[warp] = W;
+  __syncthreads();
+  if (warp == 0) {
+    float Wt = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) Wt += wsum_s[w];
+    const float inv = Wt > 0.f ? 1.f / Wt : 0.f;
+    __nv_bfloat16* dst = o + ((static_cast<int64_t>(bb) * T + t) * H + h) * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      float x = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) x += acc_s[w][lane * E + e];
+      dst[e] = __float2bfloat16_rn(x * inv);
+    }
+    if (lse && lane == 0) lse[lse_off] = Wt > 0.f ? M + logf(Wt) : -INFINITY;
+  }
 }
 
 }  // namespace
@@ -75,7 +100,8 @@ cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int32_t n
                          float* lse, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(b) * tokens * heads;
   if (rows == 0) return cudaSuccess;
-  const dim3 grid(static_cast<unsigned>((rows + kWarps - 1) / kWarps));
+  if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(rows));
   auto* oo = static_cast<__nv_bfloat16*>(o);
   if (d == 128)
     merge_kernel<128><<<grid, kWarps * 32, 0, st>>>(o_parts, lse_parts, n_splits, b, tokens,

@@ -74,10 +74,15 @@ cudaError_t launch_selftest_wait(uint64_t wait_ns, cudaStream_t st);
 
 // TMA descriptor encoding (host). Returns false if the driver entry point is
 // unavailable or the encode call rejects the arguments.
-// 4-D bf16 tensor [outer3][outer2][outer1][inner0] viewed as
-// (inner0 = d, dim1 = heads, dim2 = tokens, dim3 = batch), box (box0, 1, box2, 1).
+// 4-D bf16 tensor [batch][token_rows][heads][d] viewed as (inner0 = d, dim1 =
+// heads, dim2 = tokens, dim3 = batch), box (box0, box1, box2, 1). Only the first
+// `tokens` of the `token_rows` rows per sequence are in bounds: a box reaching
+// past them reads zeros.
 bool encode_tma_bf16_4d(void* tmap_out, const void* base, uint64_t d, uint64_t heads,
-                        uint64_t tokens, uint64_t batch, uint32_t box0, uint32_t box2,
-                        bool swizzle128);
+                        uint64_t tokens, uint64_t token_rows, uint64_t batch, uint32_t box0,
+                        uint32_t box1, uint32_t box2, bool swizzle128);
+
+// 128-row query tiles of the Phase-2 query pass (rows = query tokens x GQA heads).
+int64_t query_tiles(const Shape& s, int64_t lq);
 
 }  // namespace star

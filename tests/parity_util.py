@@ -7,8 +7,11 @@ MAX_ABS = 2e-2
 MEAN_ABS = 2e-3
 LSE_ABS = 1e-3
 # A tighter check on top: the error of each output row relative to the row's
-# largest magnitude. bf16 rounding alone is below 2^-8 of it.
+# largest magnitude. bf16 rounding alone is below 2^-8 of it. The small absolute
+# floor covers rows that average ~1e6 random values (|o| ~ 1e-4), where fp32
+# summation error, not rounding of the output, sets the error.
 ROW_REL = 1e-2
+ROW_FLOOR = 2e-5
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:
@@ -25,7 +28,7 @@ def check_rows(o_gpu: np.ndarray, o_ref: np.ndarray, lse_gpu=None, lse_ref=None,
     max_abs, mean_abs = float(err.max()), float(err.mean())
     assert max_abs <= MAX_ABS, f"{what}: max-abs {max_abs:.3e}"
     assert mean_abs <= MEAN_ABS, f"{what}: mean-abs {mean_abs:.3e}"
-    scale = np.abs(o_ref).max(axis=-1, keepdims=True) + 1e-6
+    scale = np.abs(o_ref).max(axis=-1, keepdims=True) + ROW_FLOOR / ROW_REL
     rel = float((err / scale).max())
     assert rel <= ROW_REL, f"{what}: row-relative error {rel:.3e}"
     if lse_gpu is not None:
