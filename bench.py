@@ -121,9 +121,39 @@ class Step:
         self.lse_dec = torch.empty((w.decode_steps, b, hq, 1), dtype=torch.float32, device=device)
         self.flush = torch.empty(workloads.l2_flush_bytes(), dtype=torch.uint8, device=device)
         self.events = None
+        self.graphs = None
+        self.launches_per_step = None
+
+    # The three phases, issued through the public API on the current stream.
+    def prefill(self):
+        x = self.x
+        self.layer.prefill(x["q_ctx"], x["k_ctx"], x["v_ctx"], o=self.o_ctx, lse=self.lse_ctx)
+
+    def query(self):
+        x = self.x
+        self.layer.query(x["q_qry"], x["k_qry"], x["v_qry"], o=self.o_q, lse=self.lse_q)
+
+    def decode_all(self):
+        x = self.x
+        for t in range(self.w.decode_steps):
+            self.layer.decode(x["q_dec"][t], x["k_dec"][t], x["v_dec"][t], o=self.o_dec[t],
+                              lse=self.lse_dec[t])
+
+    def capture(self):
+        """Record each phase once into a CUDA graph (the decode graph holds all T steps),
+        so that replays launch the same kernels without per-call host overhead."""
+        torch.cuda.synchronize()
+        n0 = self.sa.launch_count()
+        self.graphs = []
+        for fn in (self.prefill, self.query, self.decode_all):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            self.graphs.append(g)
+        torch.cuda.synchronize()
+        self.launches_per_step = self.sa.launch_count() - n0
 
     def run(self, record: bool = False):
-        w, x, layer = self.w, self.x, self.layer
         ev = []
         self.flush.fill_(1)  # evict L2 between steps (buffer > 126 MB L2)
 
@@ -134,23 +164,20 @@ class Step:
                 ev.append(e)
 
         mark()
-        layer.prefill(x["q_ctx"], x["k_ctx"], x["v_ctx"], o=self.o_ctx, lse=self.lse_ctx)
-        mark()
-        layer.query(x["q_qry"], x["k_qry"], x["v_qry"], o=self.o_q, lse=self.lse_q)
-        mark()
-        for t in range(w.decode_steps):
-            layer.decode(x["q_dec"][t], x["k_dec"][t], x["v_dec"][t], o=self.o_dec[t],
-                         lse=self.lse_dec[t])
+        for i, fn in enumerate((self.prefill, self.query, self.decode_all)):
+            if self.graphs is not None:
+                self.graphs[i].replay()
+            else:
+                fn()
             mark()
         if record:
             self.events = ev
 
     def phase_times_ms(self):
+        """(Phase 1, query, average decode step) in ms from the last recorded run."""
         ev = self.events
-        p1 = ev[0].elapsed_time(ev[1])
-        q = ev[1].elapsed_time(ev[2])
-        dec = [ev[2 + t].elapsed_time(ev[3 + t]) for t in range(self.w.decode_steps)]
-        return p1, q, dec
+        return (ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]),
+                ev[2].elapsed_time(ev[3]) / self.w.decode_steps)
 
 
 def decode_cold_ms(step: Step, reps: int = 1):
@@ -182,6 +209,7 @@ def e2e_run(step: Step, steps: int):
     host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in outs)
+    graphs, step.graphs = step.graphs, None  # every call issued through the API, no replay
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
@@ -194,6 +222,7 @@ def e2e_run(step: Step, steps: int):
             h.copy_(o, non_blocking=True)
     t1.record()
     t1.synchronize()
+    step.graphs = graphs
     return t0.elapsed_time(t1) / steps, h2d, d2h
 
 
@@ -318,6 +347,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=10.0)
+    ap.add_argument("--eager", action="store_true",
+                    help="issue every call from Python instead of replaying CUDA graphs")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -336,12 +367,18 @@ def main(argv=None):
 
     for _ in range(args.warmup):
         step.run()
+    if not args.eager:
+        step.capture()
+        step.run()
+    else:
+        n0 = sa.launch_count()
+        step.run()
+        step.launches_per_step = sa.launch_count() - n0
     torch.cuda.synchronize()
 
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
-    launches0 = sa.launch_count()
-    p1_ms, q_ms, dec_ms = [], [], []
+    recorded = []
     barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
@@ -349,21 +386,23 @@ def main(argv=None):
     t0.record()
     for _ in range(args.steps):
         step.run(record=True)
-        p1_ms.append(step.events)  # read after the timed region
+        recorded.append(step.events)  # read after the timed region
     t1.record()
     torch.cuda.synchronize()
     barrier(world)
-    launches = sa.launch_count() - launches0
+    # Kernels launched in the timed region: each step replays (or re-issues) the
+    # same launches the library counted when the step was first issued.
+    launches = step.launches_per_step * args.steps
     clk = clocks.stop()
     elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world, device)
 
     phases = []
-    for evs in p1_ms:
+    for evs in recorded:
         step.events = evs
         phases.append(step.phase_times_ms())
     p1_list = [p[0] for p in phases]
     q_list = [p[1] for p in phases]
-    dec_all = [t for p in phases for t in p[2]]
+    dec_all = [p[2] for p in phases]
 
     ms_per_step = elapsed_ms / args.steps
     tokens = w.batch * w.ctx_len
@@ -385,12 +424,16 @@ def main(argv=None):
              "frac_of_burst": p1_tflops / peaks["bf16_tflops"],
              "peak_kind": f"bf16 sustained ({peaks['source']})", "traffic": None,
              "algorithmic_per_launch": flops, "avg_launch_ms": p1_avg}
-    rl_dec = {"bound": "hbm", "kernel": "phase2_decode (partials + merge)", "achieved": dec_cold_gbs,
-              "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dec_cold_gbs / peaks["hbm_gbs"],
+    # Decode: per-step duration inside the timed region (partials + merge, consecutive
+    # steps overlapping through programmatic launch); "cold" = one step timed alone
+    # right after an L2 flush, launch latency included.
+    rl_dec = {"bound": "hbm", "kernel": "phase2_decode (partials + merge)", "achieved": dec_gbs,
+              "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
               "peak_kind": f"HBM copy ({peaks['source']})", "traffic": None,
-              "algorithmic_per_launch": statistics.mean(kv_bytes), "avg_launch_ms": dec_cold_avg,
-              "in_step_gbs": dec_gbs, "in_step_avg_launch_ms": dec_avg}
-    dominant = rl_p1 if p1_avg >= sum(dec_all) / args.steps else rl_dec
+              "algorithmic_per_launch": statistics.mean(kv_bytes), "avg_launch_ms": dec_avg,
+              "cold_gbs": dec_cold_gbs, "cold_avg_launch_ms": dec_cold_avg,
+              "cold_frac": dec_cold_gbs / peaks["hbm_gbs"]}
+    dominant = rl_p1 if p1_avg >= statistics.mean(dec_all) * w.decode_steps else rl_dec
 
     e2e = None
     if not args.no_e2e:
@@ -416,12 +459,14 @@ def main(argv=None):
                        "ctx_len": w.ctx_len, "block_size": w.block_size,
                        "query_len": w.query_len, "decode_steps": w.decode_steps,
                        "planted_pairs": w.planted_pairs, "parallelism": f"replicas{world}",
+                       "launch": "eager" if args.eager else "cuda-graph replay per phase",
                        "l2": "256 MiB write before every step; every decode step reads "
                              f"{w.decode_kv_bytes(0) / 1e6:.1f} MB of KV"},
             "phase1": {"ms": p1_avg, "tok_s": tokens / (p1_avg / 1e3), "tflops": p1_tflops,
                        "frac_sustained": rl_p1["frac"], "frac_burst": rl_p1["frac_of_burst"]},
             "query": {"ms": statistics.mean(q_list)},
             "decode": {"ms_per_token_in_step": dec_avg, "gbs_in_step": dec_gbs,
+                       "frac_hbm_in_step": dec_gbs / peaks["hbm_gbs"],
                        "ms_per_token_cold": dec_cold_avg, "gbs_cold": dec_cold_gbs,
                        "frac_hbm_cold": dec_cold_gbs / peaks["hbm_gbs"]},
             "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac",

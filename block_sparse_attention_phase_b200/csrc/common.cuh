@@ -173,6 +173,16 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// ------------------------------------------------------------------ programmatic launch
+// With programmatic stream serialisation, a kernel may start before the previous
+// kernel in the stream has finished. pdl_wait() blocks until that kernel has
+// completed and its memory is visible (a no-op without such a dependency);
+// pdl_launch_dependents() lets the next kernel start being scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ warp-level MMA
 // Four 8x8 b16 matrices from shared memory; lane l supplies the address of row
 // l % 8 of matrix l / 8.

@@ -4,22 +4,23 @@
 // appends the token's KV to its cache).
 //
 // One CTA = (split, batch, kv-head). A split is a chunk of one context block, or
-// the query-local cache plus the new token. The CTA streams its chunk's K and V
-// rows for that kv-head once (TMA tiles of 64 tokens into a shared-memory ring)
-// and serves all G = Hq/Hkv q-heads of the group from each row, so every KV byte
-// is read from HBM exactly once per step. The work is HBM-bound: per key the
-// CTA does 2*G*d multiply-adds against 4*d bytes.
+// the query-local cache (which, after the append this kernel does, ends with the
+// new token). The CTA streams its chunk's K and V rows for that kv-head once and
+// serves all G = Hq/Hkv q-heads from them, so every KV byte is read from HBM
+// exactly once per step. That makes the step HBM-bound; to keep the SMs from
+// becoming the limit, the G x d x tokens contractions run as warp-level bf16
+// MMAs (m16n8k16, fp32 accumulate) with the G heads as the MMA rows, about five
+// instructions per key instead of ~80 on the FMA pipes.
 //
-// Consumer lanes own one 16-byte slice (8 elements) of a token row: a row is
-// LPT = d/8 lanes, a warp covers 32/LPT rows per step. The G partial dot
-// products of a lane are folded into full dot products with a transpose-reduce
-// (each xor-shuffle level also halves the number of heads a lane carries), so a
-// lane ends with the logit of one (token, head) pair. A running max / sum per
-// head gives each warp a partial softmax state; warps are combined through
-// shared memory at the end, and the CTA writes (o_s, lse_s) in fp32.
+// Data movement: a producer warp streams 64-token K and V tiles of one kv-head
+// into a 3-stage ring with TMA (64-column boxes, 128-byte swizzle, so that the
+// ldmatrix reads below hit 8 different bank groups). Each of the 4 consumer warps
+// takes 16 tokens of every tile: S = Q K^T (2 n-tiles x d/16 k-steps), an online
+// softmax per head (running max shared by the 4 lanes of a row), then O += P V
+// with P reused straight from the S accumulators as the A operand. The warps'
+// (m, l, O) meet in shared memory and the CTA writes one fp32 partial per head.
 #include <cuda.h>
 #include <cuda_bf16.h>
-#include <math_constants.h>
 
 #include "common.cuh"
 #include "star_internal.h"
@@ -42,165 +43,28 @@ struct DecodeArgs {
   uint32_t* status;
 };
 
-constexpr int kTile = 64;
+constexpr int kTile = 64;      // tokens per TMA tile
+constexpr int kWarps = 4;      // consumer warps (16 tokens of each tile apiece)
+constexpr int kStages = 3;
+constexpr float kRescaleLog2 = 8.f;
 
 template <int D, int G>
-struct Lanes {
-  static constexpr int LPT = D / 8;     // lanes per token row
-  static constexpr int TPW = 32 / LPT;  // token rows per warp step
-  // Head a lane carries after the transpose-reduce.
-  __device__ static int head_of(int lane) {
-    int h = 0, nh = G;
-#pragma unroll
-    for (int o = LPT / 2; o >= 1; o >>= 1) {
-      if (nh > 1) {
-        nh >>= 1;
-        if (lane & o) h += nh;
-      }
-    }
-    return h;
-  }
-  // A lane of token group g that carries head h.
-  __device__ static int src_of(int h, int g) {
-    int src = g * LPT, nh = G;
-#pragma unroll
-    for (int o = LPT / 2; o >= 1; o >>= 1) {
-      if (nh > 1) {
-        nh >>= 1;
-        if (h >= nh) {
-          src |= o;
-          h -= nh;
-        }
-      }
-    }
-    return src;
-  }
-};
-
-template <int D, int G>
-struct WarpState {
-  float q[G][8];
-  float acc[G][8];
-  float m = -INFINITY;  // running max (log2 units) of the head this lane carries
-  float l = 0.f;            // running sum over this lane's token group
-};
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& r, float (&f)[8]) {
-  f[0] = bf16_lo(r.x); f[1] = bf16_hi(r.x); f[2] = bf16_lo(r.y); f[3] = bf16_hi(r.y);
-  f[4] = bf16_lo(r.z); f[5] = bf16_hi(r.z); f[6] = bf16_lo(r.w); f[7] = bf16_hi(r.w);
-}
-
-// Fold G partial dots across the LPT lanes of a token row into one full dot
-// for the head `head_of(lane)`.
-template <int D, int G>
-__device__ __forceinline__ float transpose_reduce(float (&v)[G], int lane) {
-  constexpr int LPT = D / 8;
-  int nh = G;
-#pragma unroll
-  for (int o = LPT / 2; o >= 1; o >>= 1) {
-    if (nh > 1) {
-      const int half = nh >> 1;
-      const bool upper = (lane & o) != 0;
-#pragma unroll
-      for (int j = 0; j < G / 2; ++j) {
-        if (j < half) {
-          const float send = upper ? v[j] : v[j + half];
-          const float keep = upper ? v[j + half] : v[j];
-          v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-      }
-      nh = half;
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
-    }
-  }
-  return v[0];
-}
-
-// Consume U warp-steps of token rows. krow[u] / vrow[u] point at this lane's
-// 16-byte slice of step u's K and V rows (shared or global memory); valid[u]
-// says whether that row is a key of this split. Rows are loaded lazily to keep
-// register pressure low.
-template <int D, int G, int U>
-__device__ __forceinline__ void consume(WarpState<D, G>& st, const uint8_t* const (&krow)[U],
-                                        const uint8_t* const (&vrow)[U], const bool (&valid)[U],
-                                        int lane) {
-  using LN = Lanes<D, G>;
-  const int g = lane / LN::LPT;
-  float s[U];
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    float kf[8];
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(krow[u]), kf);
-    float part[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float a = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) a = fmaf(st.q[h][e], kf[e], a);
-      part[h] = a;
-    }
-    const float dot = transpose_reduce<D, G>(part, lane);
-    s[u] = valid[u] ? dot : -INFINITY;
-  }
-  float mt = s[0];
-#pragma unroll
-  for (int u = 1; u < U; ++u) mt = fmaxf(mt, s[u]);
-#pragma unroll
-  for (int o = LN::LPT; o < 32; o <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
-  const float m_new = fmaxf(st.m, mt);
-  const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-  const float alpha = exp2f(st.m - m_use);
-  float p[U];
-  float psum = 0.f;
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    p[u] = exp2f(s[u] - m_use);
-    psum += p[u];
-  }
-  st.l = st.l * alpha + psum;
-  st.m = m_new;
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const float ah = __shfl_sync(0xffffffffu, alpha, LN::src_of(h, 0));
-#pragma unroll
-    for (int e = 0; e < 8; ++e) st.acc[h][e] *= ah;
-  }
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    // Rows past the split end may hold stale cache bytes (even NaN patterns);
-    // use zeros there so that p = 0 never meets a NaN.
-    uint4 raw = *reinterpret_cast<const uint4*>(vrow[u]);
-    if (!valid[u]) raw = make_uint4(0u, 0u, 0u, 0u);
-    float vf[8];
-    bf16x8_to_f32(raw, vf);
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float ph = __shfl_sync(0xffffffffu, p[u], LN::src_of(h, g));
-#pragma unroll
-      for (int e = 0; e < 8; ++e) st.acc[h][e] = fmaf(ph, vf[e], st.acc[h][e]);
-    }
-  }
-}
-
-template <int D, int G, int W, int NST>
-__global__ void __launch_bounds__((W + 1) * 32, (G <= 4 ? 2 : 1)) decode_partials_kernel(
+__global__ void __launch_bounds__((kWarps + 1) * 32) decode_partials_kernel(
     const __grid_constant__ CUtensorMap mk_ctx, const __grid_constant__ CUtensorMap mv_ctx,
     const __grid_constant__ CUtensorMap mk_cache, const __grid_constant__ CUtensorMap mv_cache,
     const DecodeArgs a) {
-  using LN = Lanes<D, G>;
-  constexpr int LPT = LN::LPT;
-  constexpr int TPW = LN::TPW;
-  constexpr int TOK_PER_WARP = kTile / W;
-  constexpr int U = TOK_PER_WARP / TPW;
-  static_assert(U >= 1 && TOK_PER_WARP % TPW == 0, "tile must split evenly over warps");
-  constexpr uint32_t kTileBytes = kTile * D * 2;
+  constexpr int CH = D / 64;                        // 64-column chunks of a row
+  constexpr uint32_t kChunk = kTile * 128;          // one chunk of a tile: 64 rows x 128 B
+  constexpr uint32_t kTileBytes = CH * kChunk;
+  static_assert(G == 1 || G == 2 || G == 4 || G == 8, "GQA group must be 1, 2, 4 or 8");
 
-  extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* kbuf = smem;
-  uint8_t* vbuf = smem + NST * kTileBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + 2 * NST * kTileBytes);
-  uint64_t* empty = full + NST;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* kbuf = base;                          // [kStages][kTileBytes]
+  uint8_t* vbuf = base + kStages * kTileBytes;   // [kStages][kTileBytes]
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + 2 * kStages * kTileBytes);
+  uint64_t* empty = full + kStages;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -219,139 +83,204 @@ __global__ void __launch_bounds__((W + 1) * 32, (G <= 4 ? 2 : 1)) decode_partial
     k1 = min(bend, k0 + a.chunk);
   } else {
     k0 = 0;
-    k1 = a.cache_len;
+    k1 = a.cache_len + 1;  // the cached rows and the new token, appended below
   }
   const int ntiles = static_cast<int>((k1 - k0 + kTile - 1) / kTile);
 
   if (threadIdx.x == 0) {
 #pragma unroll
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], W);
+      mbar_init(&empty[s], kWarps);
     }
     fence_barrier_init();
   }
   __syncthreads();
+  // The merge that reads this launch's partials may be scheduled now; it waits for
+  // this grid to finish before reading anything. (This kernel itself may have
+  // started while the previous step's merge was still reading the workspace: the
+  // partials are written only after pdl_wait() below. Everything it reads — the
+  // context, the cache rows and this step's inputs — was complete before that
+  // merge could start.)
+  pdl_launch_dependents();
 
-  if (warp == W) {
-    // ---------------- producer warp: TMA loads, and the cache append ----------------
-    if (lane == 0 && ntiles > 0) {
-      const CUtensorMap* mk = is_cache ? &mk_cache : &mk_ctx;
-      const CUtensorMap* mv = is_cache ? &mv_cache : &mv_ctx;
-      for (int i = 0; i < ntiles; ++i) {
-        const int stg = i % NST;
-        const uint32_t ph = (i / NST) & 1;
-        if (i >= NST && !mbar_wait(&empty[stg], ph ^ 1, a.status)) break;
-        mbar_arrive_expect_tx(&full[stg], 2 * kTileBytes);
-        const int32_t t0 = static_cast<int32_t>(k0 + static_cast<int64_t>(i) * kTile);
-        tma_load_4d(kbuf + stg * kTileBytes, mk, &full[stg], 0, kvh, t0, bb);
-        tma_load_4d(vbuf + stg * kTileBytes, mv, &full[stg], 0, kvh, t0, bb);
-      }
-    }
-    if (is_cache && lane < LPT) {
-      // Append the new token's K/V at cache row cache_len. No CTA of this launch
-      // reads that row as a cache key (the token is taken from k_new / v_new).
+  if (warp == kWarps) {
+    // ---------------- producer warp: the cache append, then TMA loads ----------------
+    if (is_cache && lane < D / 8) {
       const int64_t src = (static_cast<int64_t>(bb) * a.hkv + kvh) * D + lane * 8;
       const int64_t dst = ((static_cast<int64_t>(bb) * a.cap + a.cache_len) * a.hkv + kvh) * D + lane * 8;
       *reinterpret_cast<uint4*>(a.k_cache + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
       *reinterpret_cast<uint4*>(a.v_cache + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
+      fence_proxy_async_global();  // the TMA loads below read this row
+    }
+    __syncwarp();
+    if (lane == 0 && ntiles > 0) {
+      const CUtensorMap* mk = is_cache ? &mk_cache : &mk_ctx;
+      const CUtensorMap* mv = is_cache ? &mv_cache : &mv_ctx;
+      for (int i = 0; i < ntiles; ++i) {
+        const int stg = i % kStages;
+        const uint32_t ph = (i / kStages) & 1;
+        if (i >= kStages && !mbar_wait(&empty[stg], ph ^ 1, a.status)) break;
+        mbar_arrive_expect_tx(&full[stg], 2 * kTileBytes);
+        const int32_t t0 = static_cast<int32_t>(k0 + static_cast<int64_t>(i) * kTile);
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          tma_load_4d(kbuf + stg * kTileBytes + c * kChunk, mk, &full[stg], c * 64, kvh, t0, bb);
+          tma_load_4d(vbuf + stg * kTileBytes + c * kChunk, mv, &full[stg], c * 64, kvh, t0, bb);
+        }
+      }
     }
   } else {
     // ---------------- consumer warps ----------------
-    const int g = lane / LPT;
-    const int c = lane % LPT;
-    WarpState<D, G> st;
+    const int g = lane >> 2;        // MMA row: the q-head within the group (rows >= G are zero)
+    const int q2 = (lane & 3) * 2;  // MMA column pair
+    // Q as the A operand (rows = heads, k = d): a0 = row g, cols q2..q2+1; a2 = cols +8.
+    uint32_t qa[D / 16][2];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const int hq = kvh * G + h;
-      const uint4 r = *reinterpret_cast<const uint4*>(
-          a.q + (static_cast<int64_t>(bb) * a.hq + hq) * D + c * 8);
-      float f[8];
-      bf16x8_to_f32(r, f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        st.q[h][e] = f[e] * a.scale_log2;
-        st.acc[h][e] = 0.f;
+    for (int ks = 0; ks < D / 16; ++ks) {
+      if (g < G) {
+        const __nv_bfloat16* qrow = a.q + (static_cast<int64_t>(bb) * a.hq + kvh * G + g) * D + ks * 16;
+        qa[ks][0] = *reinterpret_cast<const uint32_t*>(qrow + q2);
+        qa[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + q2 + 8);
+      } else {
+        qa[ks][0] = 0u;
+        qa[ks][1] = 0u;
       }
     }
-    for (int i = 0; i < ntiles; ++i) {
-      const int stg = i % NST;
-      const uint32_t ph = (i / NST) & 1;
-      const bool ok = mbar_wait(&full[stg], ph, a.status);
-      if (ok) {
-        const uint8_t* kt = kbuf + stg * kTileBytes;
-        const uint8_t* vt = vbuf + stg * kTileBytes;
-        const uint8_t* krow[U];
-        const uint8_t* vrow[U];
-        bool valid[U];
+    float o[D / 8][4];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int tok = warp * TOK_PER_WARP + u * TPW + g;
-          valid[u] = k0 + static_cast<int64_t>(i) * kTile + tok < k1;
-          krow[u] = kt + tok * (D * 2) + c * 16;
-          vrow[u] = vt + tok * (D * 2) + c * 16;
+    for (int nt = 0; nt < D / 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+    float m_run = -INFINITY;  // running max of row g (raw score units); equal on its 4 lanes
+    float l_run = 0.f;        // this lane's share of row g's running sum
+    const float sl2 = a.scale_log2;
+
+    // ldmatrix row addresses inside one stage tile, swizzled the way the TMA wrote them.
+    // QK (B = K rows): lane -> matrix mi = lane/8 (d offset 8*mi), row ri = lane%8 (token).
+    // PV (B = V rows, transposed): matrix mi -> tokens +8*(mi&1), d offset 8*(mi>>1).
+    const int mi = lane >> 3, ri = lane & 7;
+    const int tw0 = warp * 16;
+
+    for (int i = 0; i < ntiles; ++i) {
+      const int stg = i % kStages;
+      const bool ok = mbar_wait(&full[stg], (i / kStages) & 1, a.status);
+      if (ok) {
+        const uint32_t kt = smem_u32(kbuf + stg * kTileBytes);
+        const uint32_t vt = smem_u32(vbuf + stg * kTileBytes);
+        // ---- S = Q K^T for this warp's 16 tokens (two n-tiles of 8)
+        float s[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+          const int tok = tw0 + nt * 8 + ri;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ks += 2) {
+            const int d0 = ks * 16 + mi * 8;  // this lane's matrix covers d0..d0+7
+            const uint32_t addr = kt + (d0 >> 6) * kChunk + tok * 128 +
+                                  ((((d0 & 63) >> 3) ^ (tok & 7)) << 4);
+            uint32_t b[4];
+            ldsm_x4(addr, b);
+            mma_16816(s[nt], qa[ks][0], 0u, qa[ks][1], 0u, b[0], b[1]);
+            mma_16816(s[nt], qa[ks + 1][0], 0u, qa[ks + 1][1], 0u, b[2], b[3]);
+          }
         }
-        consume<D, G, U>(st, krow, vrow, valid, lane);
+        // ---- mask keys past the end of the split
+        const int64_t tbase = k0 + static_cast<int64_t>(i) * kTile + tw0;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            if (tbase + nt * 8 + q2 + e >= k1) s[nt][e] = -INFINITY;
+        // ---- online softmax for row g (values s[nt][0..1]; rows g+8 are padding)
+        float mt = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+        const bool need = (m_run == -INFINITY) || ((mt - m_run) * sl2 > kRescaleLog2);
+        const float m_new = need ? mt : m_run;
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        if (need) {
+          const float alpha = ex2_approx((m_run - m_use) * sl2);
+          l_run *= alpha;
+#pragma unroll
+          for (int nt = 0; nt < D / 8; ++nt) {
+            o[nt][0] *= alpha;
+            o[nt][1] *= alpha;
+          }
+        }
+        m_run = m_new;
+        const float ms = m_use * sl2;
+        float p[2][2];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            p[nt][e] = ex2_approx(fmaf(s[nt][e], sl2, -ms));
+            l_run += p[nt][e];
+          }
+        // P as the A operand (16 tokens): a0 = tokens q2.. of n-tile 0, a2 = of n-tile 1.
+        const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]);
+        const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]);
+        // ---- O += P V
+        const int vtok = tw0 + ri + 8 * (mi & 1);
+#pragma unroll
+        for (int dt = 0; dt < D / 16; ++dt) {
+          const int d0 = dt * 16 + 8 * (mi >> 1);
+          const uint32_t addr = vt + (d0 >> 6) * kChunk + vtok * 128 +
+                                ((((d0 & 63) >> 3) ^ (vtok & 7)) << 4);
+          uint32_t b[4];
+          ldsm_x4_trans(addr, b);
+          mma_16816(o[2 * dt], pa0, 0u, pa2, 0u, b[0], b[1]);
+          mma_16816(o[2 * dt + 1], pa0, 0u, pa2, 0u, b[2], b[3]);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[stg]);
     }
-    if (is_cache && warp == 0) {
-      // The new token: one more row, read straight from the input.
-      const int64_t off = (static_cast<int64_t>(bb) * a.hkv + kvh) * D + c * 8;
-      const uint8_t* krow[1] = {reinterpret_cast<const uint8_t*>(a.k_new + off)};
-      const uint8_t* vrow[1] = {reinterpret_cast<const uint8_t*>(a.v_new + off)};
-      const bool valid[1] = {g == 0};
-      consume<D, G, 1>(st, krow, vrow, valid, lane);
-    }
 
-    // Fold the token groups of the warp together.
-#pragma unroll
-    for (int o = LPT; o < 32; o <<= 1) {
-      st.l += __shfl_xor_sync(0xffffffffu, st.l, o);
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) st.acc[h][e] += __shfl_xor_sync(0xffffffffu, st.acc[h][e], o);
-    }
+    // ---- combine the 4 lanes of each row, then the warps
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     // Every stage has been consumed and no copy is in flight: reuse the ring.
-    asm volatile("bar.sync 1, %0;" ::"r"(W * 32) : "memory");
-    float* cm = reinterpret_cast<float*>(smem);  // [W][G]
-    float* cl = cm + W * G;                      // [W][G]
-    float* cacc = cl + W * G;                    // [W][G][D]
-    if (g == 0) {
+    asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
+    float* cm = reinterpret_cast<float*>(base);  // [kWarps][G]
+    float* cl = cm + kWarps * G;                 // [kWarps][G]
+    float* cacc = cl + kWarps * G;               // [kWarps][G][D]
+    if (g < G) {
 #pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) cacc[(warp * G + h) * D + c * 8 + e] = st.acc[h][e];
-      const int h = LN::head_of(lane);
-      if (LN::src_of(h, 0) == lane) {
-        cm[warp * G + h] = st.m;
-        cl[warp * G + h] = st.l;
+      for (int nt = 0; nt < D / 8; ++nt) {
+        cacc[(warp * G + g) * D + nt * 8 + q2] = o[nt][0];
+        cacc[(warp * G + g) * D + nt * 8 + q2 + 1] = o[nt][1];
+      }
+      if (q2 == 0) {
+        cm[warp * G + g] = m_run;
+        cl[warp * G + g] = l_run;
       }
     }
-    asm volatile("bar.sync 1, %0;" ::"r"(W * 32) : "memory");
-    for (int idx = threadIdx.x; idx < G * D; idx += W * 32) {
+    asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
+    pdl_wait();  // the previous kernel (which may still read the workspace) has finished
+    for (int idx = threadIdx.x; idx < G * D; idx += kWarps * 32) {
       const int h = idx / D;
       const int e = idx % D;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < W; ++w) M = fmaxf(M, cm[w * G + h]);
-      float lsum = 0.f, o = 0.f;
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, cm[w * G + h]);
+      float lsum = 0.f, acc = 0.f;
       if (M != -INFINITY) {
 #pragma unroll
-        for (int w = 0; w < W; ++w) {
-          const float sc = exp2f(cm[w * G + h] - M);
+        for (int w = 0; w < kWarps; ++w) {
+          const float sc = ex2_approx((cm[w * G + h] - M) * sl2);
           lsum += cl[w * G + h] * sc;
-          o += cacc[(w * G + h) * D + e] * sc;
+          acc += cacc[(w * G + h) * D + e] * sc;
         }
       }
       const int hq = kvh * G + h;
       const int64_t row = static_cast<int64_t>(split) * a.b + bb;
-      a.o_parts[(row * a.hq + hq) * D + e] = lsum > 0.f ? o / lsum : 0.f;
+      a.o_parts[(row * a.hq + hq) * D + e] = lsum > 0.f ? acc / lsum : 0.f;
       if (e == 0) {
         a.lse_parts[row * a.hq + hq] =
-            lsum > 0.f ? (M + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+            lsum > 0.f ? (M * sl2 + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
       }
     }
   }
@@ -360,21 +289,23 @@ __global__ void __launch_bounds__((W + 1) * 32, (G <= 4 ? 2 : 1)) decode_partial
 template <int D, int G>
 cudaError_t launch_decode_t(const Shape& s, const SplitPlan& p, const DecodeArgs& a,
                             const void* kc, const void* vc, cudaStream_t st) {
-  constexpr int W = 8;
-  constexpr int NST = 3;
   alignas(64) CUtensorMap m[4];
-  const bool ok = encode_tma_bf16_4d(&m[0], kc, D, s.hkv, s.L, s.L, s.b, D, 1, kTile, false) &&
-                  encode_tma_bf16_4d(&m[1], vc, D, s.hkv, s.L, s.L, s.b, D, 1, kTile, false) &&
-                  encode_tma_bf16_4d(&m[2], a.k_cache, D, s.hkv, a.cap, a.cap, s.b, D, 1, kTile, false) &&
-                  encode_tma_bf16_4d(&m[3], a.v_cache, D, s.hkv, a.cap, a.cap, s.b, D, 1, kTile, false);
+  // The cache map covers the cached rows and the new one; rows past them read as zeros.
+  const uint64_t cache_rows = static_cast<uint64_t>(a.cache_len + 1);
+  const bool ok =
+      encode_tma_bf16_4d(&m[0], kc, D, s.hkv, s.L, s.L, s.b, 64, 1, kTile, true) &&
+      encode_tma_bf16_4d(&m[1], vc, D, s.hkv, s.L, s.L, s.b, 64, 1, kTile, true) &&
+      encode_tma_bf16_4d(&m[2], a.k_cache, D, s.hkv, cache_rows, a.cap, s.b, 64, 1, kTile, true) &&
+      encode_tma_bf16_4d(&m[3], a.v_cache, D, s.hkv, cache_rows, a.cap, s.b, 64, 1, kTile, true);
   if (!ok) return cudaErrorInvalidValue;
-  const size_t smem = 2 * NST * kTile * D * 2 + 2 * NST * sizeof(uint64_t);
-  auto kern = decode_partials_kernel<D, G, W, NST>;
+  const size_t smem = 2 * kStages * (D / 64) * kTile * 128 + 2 * kStages * sizeof(uint64_t) + 1024;
+  auto kern = decode_partials_kernel<D, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const dim3 grid(p.n_splits, s.b * s.hkv);
-  kern<<<grid, (W + 1) * 32, smem, st>>>(m[0], m[1], m[2], m[3], a);
+  e = launch_programmatic(kern, grid, dim3((kWarps + 1) * 32), smem, st, m[0], m[1], m[2], m[3], a);
+  if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();
 }

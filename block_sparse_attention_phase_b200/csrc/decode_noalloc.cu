@@ -70,7 +70,7 @@ extern "C" STAR_ATTN_API star_status_t star_attn_phase2_decode_noalloc(
   const void* ptrs[] = {q, k, v, k_ctx, v_ctx, k_cache, v_cache, o};
   for (const void* p : ptrs)
     if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
-  if (!star::aligned16(lse)) return STAR_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return STAR_ERR_INVALID_ARG;  // one float each
   if (cache_len + 1 > cache_capacity) return STAR_ERR_CACHE_FULL;
   void* scratch = star::scratch_address();
   if (!scratch) return STAR_ERR_CUDA;

@@ -42,6 +42,12 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(
   const int64_t o_stride = static_cast<int64_t>(b) * T * H * D;
   const int64_t o_off = ((static_cast<int64_t>(bb) * T + t) * H + h) * D + lane * E;
 
+  // Launched programmatically: wait until the kernel that wrote the partials has
+  // finished, then let the next kernel in the stream start being scheduled (the
+  // next decode step writes this workspace only after its own pdl_wait()).
+  pdl_wait();
+  pdl_launch_dependents();
+
   // M = max over splits
   float M = -INFINITY;
   for (int s = threadIdx.x; s < S; s += kWarps * 32) M = fmaxf(M, lse_parts[s * lse_stride + lse_off]);
@@ -103,12 +109,12 @@ cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int32_t n
   if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(rows));
   auto* oo = static_cast<__nv_bfloat16*>(o);
-  if (d == 128)
-    merge_kernel<128><<<grid, kWarps * 32, 0, st>>>(o_parts, lse_parts, n_splits, b, tokens,
-                                                    heads, oo, lse);
-  else
-    merge_kernel<64><<<grid, kWarps * 32, 0, st>>>(o_parts, lse_parts, n_splits, b, tokens,
-                                                   heads, oo, lse);
+  const cudaError_t e =
+      d == 128 ? launch_programmatic(merge_kernel<128>, grid, dim3(kWarps * 32), 0, st, o_parts,
+                                     lse_parts, n_splits, b, tokens, heads, oo, lse)
+               : launch_programmatic(merge_kernel<64>, grid, dim3(kWarps * 32), 0, st, o_parts,
+                                     lse_parts, n_splits, b, tokens, heads, oo, lse);
+  if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();
 }

@@ -18,6 +18,8 @@ constexpr int kDecodeCtasPerSM = 2;
 constexpr int64_t kMinChunk = 64;      // one TMA tile of keys
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// LSE outputs are written one float at a time: 4-byte alignment is enough.
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 star_status_t resolve(const star_attn_shape_t* in, Shape* out) {
   if (!in) return STAR_ERR_INVALID_ARG;
@@ -130,7 +132,7 @@ STAR_ATTN_API star_status_t star_attn_phase1(const star_attn_shape_t* shape, con
   if (st != STAR_OK) return st;
   if (!q || !k || !v || !o) return STAR_ERR_INVALID_ARG;
   if (!star::aligned16(q) || !star::aligned16(k) || !star::aligned16(v) || !star::aligned16(o) ||
-      !star::aligned16(lse))
+      !star::aligned4(lse))
     return STAR_ERR_INVALID_ARG;
   return star::cuda_status(
       star::launch_phase1_sm100(s, q, k, v, o, lse, reinterpret_cast<cudaStream_t>(stream)));
@@ -148,7 +150,7 @@ STAR_ATTN_API star_status_t star_attn_phase2_query(
   const void* ptrs[] = {q, k, v, k_ctx, v_ctx, k_cache, v_cache, o};
   for (const void* p : ptrs)
     if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
-  if (!star::aligned16(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned4(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
   if (query_len > cache_capacity) return STAR_ERR_CACHE_FULL;
   const star::SplitPlan plan = star::query_plan(s, query_len);
   const size_t need = star::partial_bytes(s, plan, query_len);
@@ -177,7 +179,7 @@ STAR_ATTN_API star_status_t star_attn_phase2_decode(
   const void* ptrs[] = {q, k, v, k_ctx, v_ctx, k_cache, v_cache, o};
   for (const void* p : ptrs)
     if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
-  if (!star::aligned16(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned4(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
   if (cache_len + 1 > cache_capacity) return STAR_ERR_CACHE_FULL;
   const star::SplitPlan plan = star::decode_plan(s);
   const size_t need = star::partial_bytes(s, plan, 1);

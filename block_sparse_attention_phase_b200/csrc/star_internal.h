@@ -43,6 +43,27 @@ size_t partial_bytes(const Shape& s, const SplitPlan& p, int64_t rows);
 // Counts kernel launches (host side); every launcher calls it once per launch.
 void count_launch(uint64_t n = 1);
 
+#if defined(__CUDACC__)
+// Launch with programmatic stream serialisation: the kernel may begin while the
+// previous kernel in the stream is still running; it must call pdl_wait() before
+// touching anything that kernel writes or reads.
+template <typename... Params, typename... Args>
+cudaError_t launch_programmatic(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                                cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+#endif
+
 // Device status word of the current device (address valid on that device).
 uint32_t* device_status_word();
 

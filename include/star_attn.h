@@ -23,8 +23,9 @@
  *     exp(softmax_scale * q.k) over the row's visible keys.
  *   - GQA: q-head h reads kv-head h / (num_q_heads / num_kv_heads).
  *   - All pointers are device pointers owned by the caller and must be 16-byte
- *     aligned. The library never allocates device memory and never frees a
- *     caller's buffer; any scratch it needs is the caller's `workspace`.
+ *     aligned, except LSE outputs, which need 4-byte alignment. The library
+ *     never allocates device memory and never frees a caller's buffer; any
+ *     scratch it needs is the caller's `workspace`.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
  *     Arguments are checked on the host before anything is launched; an invalid
  *     call returns an error and launches nothing. No C++ exception crosses the ABI.

@@ -73,7 +73,8 @@ def test_phase1_rejects_null_and_misaligned():
     assert _call_phase1(None, [FAKE] * 5) == 1
     assert _call_phase1(s, [0, FAKE, FAKE, FAKE, FAKE]) == 1
     assert _call_phase1(s, [FAKE + 2, FAKE, FAKE, FAKE, FAKE]) == 1
-    assert _call_phase1(s, [FAKE, FAKE, FAKE, FAKE, FAKE + 8]) == 1  # misaligned lse
+    assert _call_phase1(s, [FAKE, FAKE, FAKE, FAKE + 8, FAKE]) == 1  # misaligned o
+    assert _call_phase1(s, [FAKE, FAKE, FAKE, FAKE, FAKE + 2]) == 1  # lse not 4-byte aligned
 
 
 def test_phase2_rejects_cache_and_workspace_errors():
