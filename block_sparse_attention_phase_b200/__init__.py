@@ -35,8 +35,8 @@ STATUS_NAMES = {0: "STAR_OK", 1: "STAR_ERR_INVALID_ARG", 2: "STAR_ERR_UNSUPPORTE
 EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase2_query",
             "star_attn_phase2_decode", "star_attn_phase2_decode_noalloc", "star_attn_lse_merge", "star_attn_simple_phase1",
             "star_attn_simple_phase2", "star_attn_get_device_status",
-            "star_attn_selftest_wait_timeout", "star_attn_launch_count", "star_attn_status_string",
-            "star_attn_version"]
+            "star_attn_selftest_wait_timeout", "star_attn_selftest_exp2", "star_attn_launch_count",
+            "star_attn_status_string", "star_attn_version"]
 
 
 class StarAttnError(RuntimeError):
@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
         "star_attn_simple_phase2": (I32, [SP, P, I64, P, P, P, P, I64, I64, I32, P, P, P]),
         "star_attn_get_device_status": (I32, [P]),
         "star_attn_selftest_wait_timeout": (I32, [ctypes.c_uint64, P]),
+        "star_attn_selftest_exp2": (I32, [P, P, I64, P]),
         "star_attn_launch_count": (ctypes.c_uint64, []),
         "star_attn_status_string": (ctypes.c_char_p, [I32]),
         "star_attn_version": (ctypes.c_char_p, []),
@@ -240,6 +241,17 @@ def device_status() -> int:
 def selftest_wait_timeout(wait_ns: int = 20_000_000) -> None:
     _check(lib().star_attn_selftest_wait_timeout(int(wait_ns), _stream()),
            "star_attn_selftest_wait_timeout")
+
+
+def selftest_exp2(x: torch.Tensor) -> torch.Tensor:
+    """The FMA-pipe 2^x of the softmax, applied to a float32 CUDA tensor."""
+    if not x.is_cuda or x.dtype != torch.float32:
+        raise TypeError("x must be a float32 CUDA tensor")
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    _check(lib().star_attn_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream()),
+           "star_attn_selftest_exp2")
+    return y
 
 
 def launch_count() -> int:

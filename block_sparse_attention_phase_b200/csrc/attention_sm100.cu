@@ -44,6 +44,13 @@ constexpr int kThreads = 192;
 constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle row each)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;          // lazy-rescale threshold (log2 units)
+// Of every 8 pairs of scores, this many take the FMA-pipe exponential; the MUFU
+// (16 results per clock per SM) would otherwise pace the softmax at the same
+// rate as the tensor core's MMAs.
+#ifndef STAR_POLY_PAIRS
+#define STAR_POLY_PAIRS 2
+#endif
+constexpr int kPolyPairs = STAR_POLY_PAIRS;
 
 enum class Mode { kPhase1, kQuery };
 
@@ -389,8 +396,16 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         for (int e = 0; e < 32; e += 2) {
           const float2 x = ffma2(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])),
                                  sl2v, nms);
-          const float p0 = ex2_approx(x.x);
-          const float p1 = ex2_approx(x.y);
+          float p0, p1;
+          if (((e >> 1) & 7) < kPolyPairs) {
+            // a share of the exponentials on the FMA pipe, the rest on the MUFU
+            const float2 pp = exp2_poly2(x);
+            p0 = pp.x;
+            p1 = pp.y;
+          } else {
+            p0 = ex2_approx(x.x);
+            p1 = ex2_approx(x.y);
+          }
           ps[(e >> 1) & 1] = fadd2(ps[(e >> 1) & 1], make_float2(p0, p1));
           pk[c >> 1][(c & 1) * 16 + e / 2] = pack_bf16x2(p0, p1);
         }

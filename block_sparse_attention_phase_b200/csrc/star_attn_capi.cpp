@@ -253,6 +253,13 @@ STAR_ATTN_API star_status_t star_attn_get_device_status(star_stream_t stream) {
   return STAR_OK;
 }
 
+STAR_ATTN_API star_status_t star_attn_selftest_exp2(const float* x, float* y, int64_t n,
+                                                    star_stream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return STAR_ERR_INVALID_ARG;
+  return star::cuda_status(
+      star::launch_selftest_exp2(x, y, n, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 STAR_ATTN_API star_status_t star_attn_selftest_wait_timeout(uint64_t wait_ns,
                                                             star_stream_t stream) {
   if (wait_ns < 1000000ull) wait_ns = 1000000ull;

@@ -92,6 +92,7 @@ cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q,
                               const void* v_cache, int64_t cap, float* o_parts, float* lse_parts,
                               void* o, float* lse, cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t wait_ns, cudaStream_t st);
+cudaError_t launch_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t st);
 
 // TMA descriptor encoding (host). Returns false if the driver entry point is
 // unavailable or the encode call rejects the arguments.

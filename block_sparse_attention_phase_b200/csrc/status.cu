@@ -38,7 +38,28 @@ __global__ void selftest_wait_kernel(uint64_t wait_ns, uint32_t* status) {
   __syncthreads();
 }
 
+// y[i] = the FMA-pipe 2^x the attention softmax uses for part of its scores.
+__global__ void selftest_exp2_kernel(const float* x, float* y, int64_t n) {
+  const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_poly2(make_float2(x[i], x[i])).x;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t pairs = (n + 1) / 2;
+  const unsigned blocks = static_cast<unsigned>((pairs + 255) / 256);
+  selftest_exp2_kernel<<<blocks, 256, 0, st>>>(x, y, n);
+  count_launch();
+  return cudaGetLastError();
+}
 
 uint32_t* device_status_word() {
   int dev = 0;

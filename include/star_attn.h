@@ -215,6 +215,17 @@ STAR_ATTN_API star_status_t star_attn_selftest_wait_timeout(uint64_t wait_ns,
                                                             star_stream_t stream);
 
 /*
+ * Self-test of the base-2 exponential the attention softmax evaluates on the FMA
+ * pipe for part of its scores (range reduction to n + f, f in [-1/2, 1/2], and a
+ * degree-3 polynomial for 2^f; relative error about 7.5e-5 where the result is a
+ * normal float, x in (-125, 8]; below that the result is below 2^-124 and
+ * inputs under -126 give a subnormal near 2^-126 rather than 0).
+ * x, y: device arrays of n floats. No counterpart on the Star Attention pages.
+ */
+STAR_ATTN_API star_status_t star_attn_selftest_exp2(const float* x, float* y, int64_t n,
+                                                    star_stream_t stream);
+
+/*
  * Number of kernels this library has launched in this process (all devices).
  * A host-side counter for accounting, incremented at every successful launch.
  */

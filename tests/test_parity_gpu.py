@@ -119,6 +119,24 @@ def test_simple_kernels_agree_with_oracle():
     check_rows(to_np(o), rq, to_np(l), rql, "simple phase2")
 
 
+def test_fma_pipe_exp2_accuracy():
+    """The softmax's FMA-pipe 2^x against float64 2^x (and CUDA's own exp2f for
+    reference): relative error within the fitted 7.5e-5 bound where the result
+    is a normal float (x > -125); near 2^-126 it is only absolutely tiny."""
+    x = torch.cat([torch.linspace(-126.0, 8.0, 1_000_001), torch.tensor([0.0, -0.5, 0.5, 7.999])])
+    y = sa().selftest_exp2(x.cuda()).cpu().double()
+    ref = torch.exp2(x.double())
+    normal = x > -125.0
+    rel = ((y - ref).abs() / ref)[normal].max().item()
+    assert rel < 7.6e-5, rel
+    ref32 = torch.exp2(x.cuda()).cpu().double()
+    assert ((y - ref32).abs() / ref32)[normal].max().item() < 7.7e-5
+    assert (y - ref)[~normal].abs().max().item() < 2.0 ** -135
+    # below the range the result is a tiny non-negative float, never NaN
+    lo = sa().selftest_exp2(torch.tensor([-127.0, -1e4, float("-inf")], device="cuda")).cpu()
+    assert torch.isfinite(lo).all() and (lo >= 0).all() and (lo < 1.2e-38).all()
+
+
 def test_wait_timeout_is_reported_not_trapped():
     m = sa()
     assert m.device_status() == 0
