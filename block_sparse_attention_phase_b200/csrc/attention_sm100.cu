@@ -5,32 +5,39 @@
 // "Size of Anchor Block"): block b_0 runs plain causal attention, every block
 // b_i (i > 0) runs causal attention over [anchor = b_0 ; b_i] and keeps only its
 // own rows. The anchor is never copied: a work item of block i first streams
-// b_0's K/V tiles (all visible), then its own block's tiles up to the diagonal
-// (the diagonal tile causally masked).
-//   Work item = (batch, kv-head, block i, 128-row q-tile m, head in the GQA
-//   group). Items are ordered so that the q-tiles and the G heads of one block
-//   run together (their K/V and the anchor's stay in L2), blocks i > 0 before
-//   b_0, larger m (longer rows) first.
+// b_0's K/V tiles (all visible), then its own block's tiles up to the diagonal.
 //
 // Phase-2 query tokens (hotaipapers.com page, Phase 2 paragraph): every split
 // (a chunk of one context block, or the query-local cache) returns a partial
 // output and its LSE for all query rows; the merge kernel combines them.
-//   Work item = (batch, kv-head, split, q-tile). A q-tile packs 128/G query
-//   tokens x the G heads of one kv-head into 128 rows, so each K/V tile feeds
-//   all G heads. Context splits see every key of their chunk; the cache split is
-//   causal: query token j sees cache rows 0..j.
 //
-// CTA = 6 warps:
-//   warp 0     TMA producer: Q once, then K and V tiles into 2-stage rings
-//   warp 1     TMEM allocator and MMA issuer (one thread):
-//                S_j = Q K_j^T  (SS MMA, fp32 into TMEM, double-buffered)
-//                O  += P_j V_j  (TS MMA: P read from TMEM, V from smem)
-//   warps 2-5  softmax, one thread per row (TMEM lane = row): read S_j, mask,
-//              running max with lazy rescaling (O is rescaled only when the max
-//              grows by more than 2^8), P_j = exp2(...) written back to TMEM as
-//              bf16 over S_j's columns; epilogue O / l and LSE.
-// TMEM columns: S_0 [0,128), S_1 [128,256), O [256, 256+d).
-// The QK^T MMA of tile j+1 overlaps the softmax of tile j.
+// One CTA computes two 128-row Q tiles against the same sequence of 128-key K/V
+// tiles, so every K/V tile loaded serves 256 rows:
+//   Phase 1: the two tiles are two heads of one GQA group at the same block
+//            rows (G >= 2), or two consecutive 128-row tiles of one head (G = 1;
+//            the first tile then sees one fully masked extra K/V tile).
+//   Query:   two consecutive tiles of packed rows, each 128/G query tokens x the
+//            G heads of one kv-head; context splits see every key of their
+//            chunk, the cache split is causal (query token j sees cache rows <= j).
+// Work items are ordered so that the tiles of one block run together (their
+// K/V and the anchor's stay in L2), blocks i > 0 before b_0, longer rows first.
+//
+// CTA = 3 warpgroups (12 warps):
+//   warpgroup 0  warp 0: TMA producer (both Q tiles once, then K and V tiles
+//                into 2-stage rings); warp 1: TMEM allocator and MMA issuer
+//                (one thread); warps 2-3 idle. Registers trimmed to 40.
+//   warpgroups 1, 2  the softmax of Q tile 0 and of Q tile 1, one thread per row
+//                (TMEM lane = row), registers raised to 232.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256, 256+d), O_1 [256+d, 256+2d).
+// MMA order (one thread): S_0(0), S_1(0), then for every K/V tile j
+//   O_0 += P_0(j) V_j, S_0(j+1), O_1 += P_1(j) V_j, S_1(j+1),
+// so the tensor core computes one tile's scores while the other tile's softmax
+// runs. P_q(j) is written over S_q(j)'s columns as bf16 pairs and read by the
+// MMA from TMEM. A commit after S_q(j+1) also covers O_q += P_q(j) V_j (a commit
+// tracks every earlier MMA of the thread), so a softmax warp may rescale O_q as
+// soon as it sees S_q(j+1). The running max is lazy: O is rescaled only when a
+// row's max grows by more than 2^8; the final normalisation uses the same stale
+// max, so the result is exact.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -40,10 +47,16 @@
 namespace star {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
 constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle row each)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;          // lazy-rescale threshold (log2 units)
+// Register split: 384 threads launch with 168 registers each (64512); warpgroup 0
+// gives back down to 56, the two softmax warpgroups take 224: 128*56 + 256*224 = 64512.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsLow = 56;
+constexpr int kRegsHigh = 224;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
 // Of every 8 pairs of scores, this many take the FMA-pipe exponential; the MUFU
 // (16 results per clock per SM) would otherwise pace the softmax at the same
 // rate as the tensor core's MMAs.
@@ -62,7 +75,6 @@ struct AttnArgs {
   // Phase 1
   int32_t n_blocks, mt;   // blocks; 128-row q-tiles per block
   int32_t n_anchor;       // 128-column tiles covering the anchor b_0
-  int32_t anchor_tail;    // visible columns of the last anchor tile
   __nv_bfloat16* o;       // [b, L, Hq, d]
   float* lse;             // [b, Hq, L] or null
   // Phase-2 query
@@ -75,9 +87,9 @@ struct AttnArgs {
 struct Bars {
   uint64_t q_full;
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2];
-  uint64_t p_full;
-  uint64_t o_bar;
+  uint64_t s_full[2];  // per Q tile: S_q(j) (and every earlier MMA) complete
+  uint64_t p_full[2];  // per Q tile: P_q(j) written to TMEM
+  uint64_t o_bar[2];   // per Q tile: the last O_q += P V complete
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -86,13 +98,13 @@ struct Bars {
 // What one CTA computes.
 struct Item {
   int bb, kvh;
-  int32_t qc1, qc2;  // Q tile coordinates: head (dim 1), token (dim 2)
   int n_tiles;
+  int32_t qc1[2], qc2[2];  // Q tile coordinates: head (dim 1), token (dim 2)
   // Phase 1
-  int h, n_anchor, rows_valid;
-  int64_t bstart, t0;
+  int h[2], rows_valid[2], n_anchor;
+  int64_t bstart, t0[2];
   // query
-  int split, tok0;
+  int split, tok0[2];
   bool cache;
   int64_t k0, k1;
 };
@@ -102,33 +114,59 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a) {
   Item it{};
   int64_t r = blockIdx.x;
   if constexpr (M == Mode::kPhase1) {
-    const int hg = static_cast<int>(r % a.G);
-    r /= a.G;
-    const int mp = static_cast<int>(r % a.mt);
-    r /= a.mt;
-    const int ip = static_cast<int>(r % a.n_blocks);
-    r /= a.n_blocks;
-    it.kvh = static_cast<int>(r % a.hkv);
-    it.bb = static_cast<int>(r / a.hkv);
-    const int i = (ip + 1) % a.n_blocks;  // blocks 1..n-1 first, b_0 (cheapest) last
-    const int m = a.mt - 1 - mp;          // longest q-tiles first
-    it.h = it.kvh * a.G + hg;
+    int i, m0, m1;
+    if (a.G >= 2) {
+      const int npair = a.G / 2;
+      const int hp = static_cast<int>(r % npair);
+      r /= npair;
+      const int mp = static_cast<int>(r % a.mt);
+      r /= a.mt;
+      const int ip = static_cast<int>(r % a.n_blocks);
+      r /= a.n_blocks;
+      it.kvh = static_cast<int>(r % a.hkv);
+      it.bb = static_cast<int>(r / a.hkv);
+      i = (ip + 1) % a.n_blocks;  // blocks 1..n-1 first, b_0 (cheapest) last
+      m0 = m1 = a.mt - 1 - mp;    // longest q-tiles first
+      it.h[0] = it.kvh * a.G + 2 * hp;
+      it.h[1] = it.h[0] + 1;
+    } else {
+      const int mt2 = (a.mt + 1) / 2;
+      const int mp = static_cast<int>(r % mt2);
+      r /= mt2;
+      const int ip = static_cast<int>(r % a.n_blocks);
+      r /= a.n_blocks;
+      it.kvh = static_cast<int>(r % a.hkv);
+      it.bb = static_cast<int>(r / a.hkv);
+      i = (ip + 1) % a.n_blocks;
+      m0 = 2 * (mt2 - 1 - mp);
+      m1 = m0 + 1;
+      it.h[0] = it.h[1] = it.kvh;
+    }
     it.bstart = static_cast<int64_t>(i) * a.B;
     const int64_t bend = min(a.L, it.bstart + a.B);
-    it.t0 = it.bstart + 128 * static_cast<int64_t>(m);
-    it.rows_valid = it.t0 >= bend ? 0 : static_cast<int>(bend - it.t0 < 128 ? bend - it.t0 : 128);
+    it.t0[0] = it.bstart + 128 * static_cast<int64_t>(m0);
+    it.t0[1] = it.bstart + 128 * static_cast<int64_t>(m1);
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      it.rows_valid[q] = it.t0[q] >= bend ? 0 : static_cast<int>(bend - it.t0[q] < 128 ? bend - it.t0[q] : 128);
+    const int m_last = it.rows_valid[1] > 0 ? m1 : m0;
     it.n_anchor = i > 0 ? a.n_anchor : 0;
-    it.n_tiles = it.rows_valid > 0 ? it.n_anchor + m + 1 : 0;
-    it.qc1 = it.h;
-    it.qc2 = static_cast<int32_t>(it.t0);
+    it.n_tiles = it.rows_valid[0] > 0 ? it.n_anchor + m_last + 1 : 0;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      it.qc1[q] = it.h[q];
+      it.qc2[q] = static_cast<int32_t>(it.t0[q]);
+    }
   } else {
-    const int qt = static_cast<int>(r % a.n_qt);
-    r /= a.n_qt;
+    const int npair = (a.n_qt + 1) / 2;
+    const int qp = static_cast<int>(r % npair);
+    r /= npair;
     it.split = static_cast<int>(r % a.n_splits);
     r /= a.n_splits;
     it.kvh = static_cast<int>(r % a.hkv);
     it.bb = static_cast<int>(r / a.hkv);
-    it.tok0 = qt * (128 / a.G);
+    it.tok0[0] = 2 * qp * (128 / a.G);
+    it.tok0[1] = it.tok0[0] + 128 / a.G;  // may lie past Lq: zero rows, never stored
     it.cache = it.split == a.n_ctx;
     if (!it.cache) {
       const int64_t blk = it.split / a.spb;
@@ -142,8 +180,11 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a) {
       it.k1 = a.lq;
     }
     it.n_tiles = static_cast<int>((it.k1 - it.k0 + 127) / 128);
-    it.qc1 = it.kvh * a.G;
-    it.qc2 = it.tok0;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      it.qc1[q] = it.kvh * a.G;
+      it.qc2[q] = it.tok0[q];
+    }
   }
   return it;
 }
@@ -165,6 +206,37 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ba
   }
 }
 
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Columns [0, limit) of K/V tile j are visible to a softmax row whose token is
+// `tok` (Phase 1: absolute context position; query: query-token index).
+template <Mode M>
+__device__ __forceinline__ int visible_prefix(const Item& it, const AttnArgs& a, int64_t tok,
+                                              int j) {
+  int64_t lim;
+  if constexpr (M == Mode::kPhase1) {
+    if (j < it.n_anchor) {
+      lim = a.B - 128 * static_cast<int64_t>(j);  // the anchor ends at B
+    } else {
+      const int64_t kv0 = it.bstart + 128 * static_cast<int64_t>(j - it.n_anchor);
+      lim = tok - kv0 + 1;  // causal inside the own block
+    }
+  } else {
+    if (it.cache)
+      lim = tok - 128 * static_cast<int64_t>(j) + 1;  // query token sees cache rows <= itself
+    else
+      lim = it.k1 - it.k0 - 128 * static_cast<int64_t>(j);  // end of the chunk
+  }
+  return lim < 0 ? 0 : (lim > 128 ? 128 : static_cast<int>(lim));
+}
+
 template <int D, Mode M>
 __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
     const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -176,8 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sq = base;
-  uint8_t* sk = sq + kTileBytes;      // [2][kTileBytes]
+  uint8_t* sq = base;                 // [2][kTileBytes]
+  uint8_t* sk = sq + 2 * kTileBytes;  // [2][kTileBytes]
   uint8_t* sv = sk + 2 * kTileBytes;  // [2][kTileBytes]
   Bars* bars = reinterpret_cast<Bars*>(sv + 2 * kTileBytes);
 
@@ -185,11 +257,11 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
   if (it.n_tiles == 0) {
     if constexpr (M == Mode::kQuery) {
       // A chunk past the end of a short last block: an empty partial.
-      for (int idx = threadIdx.x; idx < 128 * D; idx += kThreads) {
+      for (int idx = threadIdx.x; idx < 256 * D; idx += kThreads) {
         const int row = idx / D, e = idx % D;
-        const int tok = it.tok0 + row / a.G;
+        const int tok = it.tok0[row >> 7] + (row & 127) / a.G;
         if (tok >= a.lq) continue;
-        const int hq = it.kvh * a.G + row % a.G;
+        const int hq = it.kvh * a.G + (row & 127) % a.G;
         const int64_t prow = static_cast<int64_t>(it.split) * a.b + it.bb;
         a.o_parts[((prow * a.lq + tok) * a.hq + hq) * D + e] = 0.f;
         if (e == 0) a.lse_parts[(prow * a.hq + hq) * a.lq + tok] = -INFINITY;
@@ -201,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int wg = warp >> 2;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -211,9 +284,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->p_full[s], 128);
+      mbar_init(&bars->o_bar[s], 1);
     }
-    mbar_init(&bars->p_full, 128);
-    mbar_init(&bars->o_bar, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_barrier_init();
@@ -227,9 +300,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (wg == 0) {
+    setmaxnreg_dec<kRegsLow>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------ TMA producer
       const CUtensorMap* mk = &tk;
       const CUtensorMap* mv = &tv;
       if constexpr (M == Mode::kQuery) {
@@ -241,10 +315,13 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(mk);
       tma_prefetch_desc(mv);
-      mbar_arrive_expect_tx(&bars->q_full, kTileBytes);
+      mbar_arrive_expect_tx(&bars->q_full, 2 * kTileBytes);
 #pragma unroll
-      for (int c = 0; c < CH; ++c)
-        tma_load_4d(sq + c * kChunkBytes, &tq, &bars->q_full, c * 64, it.qc1, it.qc2, it.bb);
+      for (int q = 0; q < 2; ++q)
+#pragma unroll
+        for (int c = 0; c < CH; ++c)
+          tma_load_4d(sq + q * kTileBytes + c * kChunkBytes, &tq, &bars->q_full, c * 64, it.qc1[q],
+                      it.qc2[q], it.bb);
       int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j & 1;
@@ -276,91 +353,110 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         if (last_k[s] >= 0) mbar_wait(&bars->k_full[s], (last_k[s] >> 1) & 1, a.status);
         if (last_v[s] >= 0) mbar_wait(&bars->v_full[s], (last_v[s] >> 1) & 1, a.status);
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t kIdescQK = make_idesc_bf16(128, 128, false, false);
       constexpr uint32_t kIdescPV = make_idesc_bf16(128, D, false, true);
       const uint32_t sq_addr = smem_u32(sq);
-      auto issue_pv = [&](int jp) -> bool {
-        const int sp = jp & 1;
-        if (!wait_or_abort(&bars->p_full, jp & 1, bars, a.status)) return false;
-        if (!wait_or_abort(&bars->v_full[sp], (jp >> 1) & 1, bars, a.status)) return false;
-        tc_fence_after();
-        const uint32_t sv_addr = smem_u32(sv + sp * kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk) {
-          // B = V tile, MN-major (d contiguous): 16 kv rows per step; the next 64
-          // columns of d sit one chunk (LBO) away, the next 8 kv rows 1024 B (SBO).
-          tc_mma_ts(tmem + 256, tmem + sp * 128 + kk * 8,
-                    make_sdesc(sv_addr + kk * 2048, kChunkBytes, 1024), kIdescPV,
-                    (jp > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&bars->o_bar);
-        tc_commit(&bars->v_empty[sp]);
-        return true;
-      };
-      bool ok = wait_or_abort(&bars->q_full, 0, bars, a.status);
-      tc_fence_after();
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j & 1;
-        if (!wait_or_abort(&bars->k_full[s], (j >> 1) & 1, bars, a.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t sk_addr = smem_u32(sk + s * kTileBytes);
+      const uint32_t sk_addr = smem_u32(sk);
+      const uint32_t sv_addr = smem_u32(sv);
+      // S_q = Q_q K_j^T: A = Q, B = K, both K-major 128-byte swizzled (16 columns = 32 bytes a step).
+      auto issue_s = [&](int q, int j) {
+        const uint32_t qa = sq_addr + q * kTileBytes;
+        const uint32_t ka = sk_addr + (j & 1) * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          // A = Q, B = K, both K-major 128-byte swizzled: 16 columns = 32 bytes per step.
           const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          tc_mma_ss(tmem + s * 128, make_sdesc(sq_addr + off, 16, 1024),
-                    make_sdesc(sk_addr + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+          tc_mma_ss(tmem + q * 128, make_sdesc(qa + off, 16, 1024), make_sdesc(ka + off, 16, 1024),
+                    kIdescQK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&bars->s_full[s]);
-        tc_commit(&bars->k_empty[s]);
-        if (j >= 1 && !issue_pv(j - 1)) ok = false;
+        tc_commit(&bars->s_full[q]);
+      };
+      // O_q += P_q V_j: P from TMEM (bf16 pairs over S_q's columns); V MN-major
+      // (d contiguous): 16 kv rows a step, the next 64 columns of d one chunk (LBO)
+      // away, the next 8 kv rows 1024 B (SBO) away.
+      auto issue_pv = [&](int q, int j) {
+        const uint32_t va = sv_addr + (j & 1) * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          tc_mma_ts(tmem + 256 + q * D, tmem + q * 128 + kk * 8,
+                    make_sdesc(va + kk * 2048, kChunkBytes, 1024), kIdescPV,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait_or_abort(&bars->q_full, 0, bars, a.status) &&
+                wait_or_abort(&bars->k_full[0], 0, bars, a.status);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        tc_commit(&bars->k_empty[0]);
       }
-      if (ok) issue_pv(n_tiles - 1);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j & 1;
+        const bool more = j + 1 < n_tiles;
+        ok = wait_or_abort(&bars->v_full[s], (j >> 1) & 1, bars, a.status) &&
+             wait_or_abort(&bars->p_full[0], j & 1, bars, a.status);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (!more) tc_commit(&bars->o_bar[0]);
+        if (more) {
+          ok = wait_or_abort(&bars->k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, bars, a.status);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        ok = wait_or_abort(&bars->p_full[1], j & 1, bars, a.status);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        tc_commit(&bars->v_empty[s]);
+        if (!more) tc_commit(&bars->o_bar[1]);
+        if (more) {
+          issue_s(1, j + 1);
+          tc_commit(&bars->k_empty[(j + 1) & 1]);
+        }
+      }
       // Every MMA this thread issued has completed before TMEM is released.
       tc_commit(&bars->drain);
       mbar_wait(&bars->drain, 0, a.status);
     }
   } else {
-    // ------------------------------------------------------------ softmax warps
+    // ------------------------------------------------------------ softmax warpgroups
+    setmaxnreg_inc<kRegsHigh>();
+    const int q = wg - 1;  // the Q tile this warpgroup owns
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const uint32_t s_col = q * 128;
+    const uint32_t o_col = 256 + q * D;
+    // This tile's scalars (selected, so that Item stays in registers).
+    int64_t row_tok;  // Phase 1: context position of this row; query: query-token index
+    int head, rows_valid;
+    if constexpr (M == Mode::kPhase1) {
+      row_tok = (q ? it.t0[1] : it.t0[0]) + row;
+      head = q ? it.h[1] : it.h[0];
+      rows_valid = q ? it.rows_valid[1] : it.rows_valid[0];
+    } else {
+      row_tok = (q ? it.tok0[1] : it.tok0[0]) + row / a.G;
+      head = it.kvh * a.G + row % a.G;
+      rows_valid = 0;
+    }
     const float sl2 = a.scale_log2;
     float m_run = -INFINITY;
     float l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      const int s = j & 1;
       // Waits are per thread; the tcgen05 loads/stores below are warp-wide, so
       // the warp proceeds only if every lane's wait succeeded.
-      ok = __all_sync(0xffffffffu, wait_or_abort(&bars->s_full[s], (j >> 1) & 1, bars, a.status));
+      ok = __all_sync(0xffffffffu, wait_or_abort(&bars->s_full[q], j & 1, bars, a.status));
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + s * 128 + c * 32, sr[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + s_col + c * 32, sr[c]);
       tmem_wait_ld();
-      // Columns [0, limit) of this tile are visible to this row.
-      int limit = 128;
-      if constexpr (M == Mode::kPhase1) {
-        if (j == n_tiles - 1) limit = row + 1;                  // diagonal: causal
-        else if (j == it.n_anchor - 1) limit = a.anchor_tail;  // partial last anchor tile
-      } else {
-        if (it.cache) {
-          const int64_t lim = it.tok0 + row / a.G - 128 * j + 1;  // token j sees cache rows <= j
-          limit = lim < 0 ? 0 : (lim > 128 ? 128 : static_cast<int>(lim));
-        } else {
-          const int64_t lim = it.k1 - it.k0 - 128 * j;            // end of the chunk
-          limit = lim > 128 ? 128 : static_cast<int>(lim);
-        }
-      }
+      const int limit = visible_prefix<M>(it, a, row_tok, j);
       // Most tiles are fully visible: mask only when some row of the warp needs it.
       if (__any_sync(0xffffffffu, limit < 128)) {
 #pragma unroll
@@ -411,73 +507,69 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         }
       const float psum = (ps[0].x + ps[0].y) + (ps[1].x + ps[1].y);
       l_run = l_run * alpha + psum;
-      if (j >= 1) {
-        // PV of the previous tile must be done before O is rescaled and P overwritten.
-        ok = __all_sync(0xffffffffu, wait_or_abort(&bars->o_bar, (j - 1) & 1, bars, a.status));
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
+      // S_q(j) complete implies O_q += P_q(j-1) V complete: O may be rescaled now.
+      if (j >= 1 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ob[32];
-            tmem_ld32(lane_addr + 256 + c * 32, ob);
-            tmem_wait_ld();
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ob[32];
+          tmem_ld32(lane_addr + o_col + c * 32, ob);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * alpha);
-            tmem_st32(lane_addr + 256 + c * 32, ob);
-          }
+          for (int e = 0; e < 32; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * alpha);
+          tmem_st32(lane_addr + o_col + c * 32, ob);
         }
       }
-      tmem_st32(lane_addr + s * 128, pk[0]);
-      tmem_st32(lane_addr + s * 128 + 32, pk[1]);
+      tmem_st32(lane_addr + s_col, pk[0]);
+      tmem_st32(lane_addr + s_col + 32, pk[1]);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->p_full);
+      mbar_arrive(&bars->p_full[q]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&bars->o_bar, (n_tiles - 1) & 1, bars, a.status));
+    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&bars->o_bar[q], 0, bars, a.status));
     tc_fence_after();
     if (ok) {
       const bool has = l_run > 0.f;
       const float inv = has ? 1.f / l_run : 0.f;
       const float lse2 = has ? m_run * sl2 + log2f(l_run) : -INFINITY;
       if constexpr (M == Mode::kPhase1) {
-        const int64_t t = it.t0 + row;
-        __nv_bfloat16* dst = a.o + ((static_cast<int64_t>(it.bb) * a.L + t) * a.hq + it.h) * D;
+        const int64_t t = row_tok;
+        const bool valid = row < rows_valid;
+        __nv_bfloat16* dst = a.o + ((static_cast<int64_t>(it.bb) * a.L + t) * a.hq + head) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ob[32];
-          tmem_ld32(lane_addr + 256 + c * 32, ob);
+          tmem_ld32(lane_addr + o_col + c * 32, ob);
           tmem_wait_ld();
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             w[e] = pack_bf16x2(__uint_as_float(ob[2 * e]) * inv, __uint_as_float(ob[2 * e + 1]) * inv);
-          if (row < it.rows_valid) {
+          if (valid) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              d4[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            for (int u = 0; u < 4; ++u)
+              d4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
           }
         }
-        if (a.lse && row < it.rows_valid)
-          a.lse[(static_cast<int64_t>(it.bb) * a.hq + it.h) * a.L + t] = lse2 * 0.69314718055994531f;
+        if (a.lse && valid)
+          a.lse[(static_cast<int64_t>(it.bb) * a.hq + head) * a.L + t] = lse2 * 0.69314718055994531f;
       } else {
-        const int tok = it.tok0 + row / a.G;
-        const int hq = it.kvh * a.G + row % a.G;
+        const int tok = static_cast<int>(row_tok);
+        const int hq = head;
         const bool valid = tok < a.lq;
         const int64_t prow = static_cast<int64_t>(it.split) * a.b + it.bb;
         float* dst = a.o_parts + ((prow * a.lq + tok) * a.hq + hq) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ob[32];
-          tmem_ld32(lane_addr + 256 + c * 32, ob);
+          tmem_ld32(lane_addr + o_col + c * 32, ob);
           tmem_wait_ld();
           if (valid) {
             float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              d4[q] = make_float4(__uint_as_float(ob[4 * q]) * inv, __uint_as_float(ob[4 * q + 1]) * inv,
-                                  __uint_as_float(ob[4 * q + 2]) * inv, __uint_as_float(ob[4 * q + 3]) * inv);
+            for (int u = 0; u < 8; ++u)
+              d4[u] = make_float4(__uint_as_float(ob[4 * u]) * inv, __uint_as_float(ob[4 * u + 1]) * inv,
+                                  __uint_as_float(ob[4 * u + 2]) * inv, __uint_as_float(ob[4 * u + 3]) * inv);
           }
         }
         if (valid) a.lse_parts[(prow * a.hq + hq) * a.lq + tok] = lse2 * 0.69314718055994531f;
@@ -509,9 +601,9 @@ AttnArgs base_args(const Shape& s) {
 template <int D, Mode M>
 cudaError_t launch(const AttnArgs& a, const CUtensorMap (&m)[5], int64_t items, cudaStream_t st) {
   constexpr uint32_t kTileBytes = (D / 64) * kChunkBytes;
-  // 5 tiles (Q, 2 K, 2 V) + barriers + alignment slack; at least 120 KB so that
+  // 6 tiles (2 Q, 2 K, 2 V) + barriers + alignment slack; at least 120 KB so that
   // only one CTA (and one 512-column TMEM allocation) lives on an SM.
-  size_t smem = 5 * kTileBytes + sizeof(Bars) + 1024;
+  size_t smem = 6 * kTileBytes + sizeof(Bars) + 1024;
   if (smem < 120 * 1024) smem = 120 * 1024;
   auto kern = attention_kernel<D, M>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -538,10 +630,10 @@ cudaError_t launch_phase1_t(const Shape& s, const void* q, const void* k, const 
   a.n_blocks = static_cast<int32_t>(s.n_blocks());
   a.mt = static_cast<int32_t>((s.B + 127) / 128);
   a.n_anchor = a.mt;
-  a.anchor_tail = static_cast<int32_t>(s.B - 128 * static_cast<int64_t>(a.n_anchor - 1));
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
-  const int64_t items = static_cast<int64_t>(s.b) * s.hkv * a.n_blocks * a.mt * a.G;
+  const int64_t pairs_per_block = a.G >= 2 ? static_cast<int64_t>(a.mt) * (a.G / 2) : (a.mt + 1) / 2;
+  const int64_t items = static_cast<int64_t>(s.b) * s.hkv * a.n_blocks * pairs_per_block;
   return launch<D, Mode::kPhase1>(a, m, items, st);
 }
 
@@ -566,10 +658,10 @@ cudaError_t launch_query_t(const Shape& s, const SplitPlan& p, const void* q, in
   a.spb = p.spb;
   a.n_ctx = p.n_ctx;
   a.n_splits = p.n_splits;
-  a.n_qt = static_cast<int32_t>((lq * G + 127) / 128);
+  a.n_qt = static_cast<int32_t>(query_tiles(s, lq));
   a.o_parts = o_parts;
   a.lse_parts = lse_parts;
-  const int64_t items = static_cast<int64_t>(s.b) * s.hkv * a.n_splits * a.n_qt;
+  const int64_t items = static_cast<int64_t>(s.b) * s.hkv * a.n_splits * ((a.n_qt + 1) / 2);
   return launch<D, Mode::kQuery>(a, m, items, st);
 }
 

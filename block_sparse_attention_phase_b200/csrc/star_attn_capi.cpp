@@ -75,9 +75,10 @@ void count_launch(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxe
 SplitPlan decode_plan(const Shape& s) { return make_plan(s, int64_t{kSMs} * kDecodeCtasPerSM); }
 
 SplitPlan query_plan(const Shape& s, int64_t lq) {
-  // One tensor-core CTA per SM; aim at about two waves over (splits x q-tiles).
-  const int64_t qt = query_tiles(s, lq);
-  return make_plan(s, 2 * int64_t{kSMs} / qt);
+  // One tensor-core CTA per SM, each taking two q-tiles; aim at about two waves
+  // over (splits x pairs of q-tiles).
+  const int64_t pairs = (query_tiles(s, lq) + 1) / 2;
+  return make_plan(s, 2 * int64_t{kSMs} / pairs);
 }
 
 size_t partial_bytes(const Shape& s, const SplitPlan& p, int64_t rows) {
