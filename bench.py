@@ -53,26 +53,31 @@ def load_peaks():
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
 
-    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
-              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
-              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    FIELDS = ["timestamp", "index", "clocks.sm", "clocks.max.sm", "power.draw",
+              "clocks_event_reasons.active", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
 
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
 
     def start(self):
+        """Start sampling (call before the warm-up; stop() keeps the timed window only)."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(self.dev)],
+                 "-lms", "20", "-i", str(self.dev)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t_begin: float = None, t_end: float = None):
+        """Samples whose timestamp lies in [t_begin, t_end] (host wall time, seconds)."""
+        import datetime
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        time.sleep(0.05)
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
@@ -87,12 +92,15 @@ class ClockSampler:
             if len(parts) != len(self.FIELDS):
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-                power.append(float(parts[3]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if t_begin is not None and not (t_begin - 0.025 <= ts <= t_end + 0.025):
+                    continue
+                sm.append(float(parts[2]))
+                smax.append(float(parts[3]))
+                power.append(float(parts[4]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:]):
+            for n, v in zip(names, parts[6:]):
                 if v.lower() == "active":
                     reasons.add(n)
         under = [s for s, p in zip(sm, power) if p > 0.35 * max(power or [1])] or sm
@@ -365,6 +373,8 @@ def main(argv=None):
     step = Step(w, x, device)
     peaks = load_peaks()
 
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()  # sampling starts early; only the timed window's samples are kept
     for _ in range(args.warmup):
         step.run()
     if not args.eager:
@@ -376,24 +386,24 @@ def main(argv=None):
         step.launches_per_step = sa.launch_count() - n0
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(torch.cuda.current_device())
-    clocks.start()
     recorded = []
     barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    wall0 = time.time()
     t0.record()
     for _ in range(args.steps):
         step.run(record=True)
         recorded.append(step.events)  # read after the timed region
     t1.record()
     torch.cuda.synchronize()
+    wall1 = time.time()
     barrier(world)
     # Kernels launched in the timed region: each step replays (or re-issues) the
     # same launches the library counted when the step was first issued.
     launches = step.launches_per_step * args.steps
-    clk = clocks.stop()
+    clk = clocks.stop(wall0, wall1)
     elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world, device)
 
     phases = []

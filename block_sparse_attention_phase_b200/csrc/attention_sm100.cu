@@ -52,10 +52,11 @@ constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;          // lazy-rescale threshold (log2 units)
 // Register split: 384 threads launch with 168 registers each (64512); warpgroup 0
-// gives back down to 56, the two softmax warpgroups take 224: 128*56 + 256*224 = 64512.
+// gives back down to 104, the two softmax warpgroups take 200: 128*104 + 256*200 = 64512
+// (the split with the least spilling in either region).
 constexpr int kLaunchRegs = 168;
-constexpr int kRegsLow = 56;
-constexpr int kRegsHigh = 224;
+constexpr int kRegsLow = 104;
+constexpr int kRegsHigh = 200;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
 // Of every 8 pairs of scores, this many take the FMA-pipe exponential; the MUFU
 // (16 results per clock per SM) would otherwise pace the softmax at the same
@@ -452,27 +453,33 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       ok = __all_sync(0xffffffffu, wait_or_abort(&bars->s_full[q], j & 1, bars, a.status));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + s_col + c * 32, sr[c]);
-      tmem_wait_ld();
       const int limit = visible_prefix<M>(it, a, row_tok, j);
       // Most tiles are fully visible: mask only when some row of the warp needs it.
-      if (__any_sync(0xffffffffu, limit < 128)) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c * 32 + e >= limit) sr[c][e] = __float_as_uint(-INFINITY);
-      }
-      // Row max with four independent 3-input max chains.
+      const bool masked = __any_sync(0xffffffffu, limit < 128);
+      // S in two halves: the max over the first 64 scores overlaps the TMEM read
+      // of the second 64. Row max with independent 3-input max chains.
+      uint32_t sr[4][32];
       float mc[4];
+      tmem_ld32(lane_addr + s_col, sr[0]);
+      tmem_ld32(lane_addr + s_col + 32, sr[1]);
+      tmem_wait_ld();
+      tmem_ld32(lane_addr + s_col + 64, sr[2]);
+      tmem_ld32(lane_addr + s_col + 96, sr[3]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        mc[c] = fmaxf(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]));
+      for (int half = 0; half < 2; ++half) {
+        if (half == 1) tmem_wait_ld();
 #pragma unroll
-        for (int e = 2; e < 32; e += 2)
-          mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+        for (int c = 2 * half; c < 2 * half + 2; ++c) {
+          if (masked) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (c * 32 + e >= limit) sr[c][e] = __float_as_uint(-INFINITY);
+          }
+          mc[c] = fmaxf(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]));
+#pragma unroll
+          for (int e = 2; e < 32; e += 2)
+            mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+        }
       }
       const float mt = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
       const bool need = (m_run == -INFINITY) || ((mt - m_run) * sl2 > kRescaleLog2);
@@ -485,9 +492,11 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       const float2 sl2v = make_float2(sl2, sl2);
       const float2 nms = make_float2(-ms, -ms);
       float2 ps[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      uint32_t pk[2][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 4; ++c) {
+        // Chunk c (32 scores) -> 16 bf16 pairs, stored to TMEM columns [16c, 16c+16)
+        // at once (S is all in registers already), so few P words are ever live.
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const float2 x = ffma2(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])),
@@ -503,8 +512,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
             p1 = ex2_approx(x.y);
           }
           ps[(e >> 1) & 1] = fadd2(ps[(e >> 1) & 1], make_float2(p0, p1));
-          pk[c >> 1][(c & 1) * 16 + e / 2] = pack_bf16x2(p0, p1);
+          pk[e / 2] = pack_bf16x2(p0, p1);
         }
+        tmem_st16(lane_addr + s_col + c * 16, pk);
+      }
       const float psum = (ps[0].x + ps[0].y) + (ps[1].x + ps[1].y);
       l_run = l_run * alpha + psum;
       // S_q(j) complete implies O_q += P_q(j-1) V complete: O may be rescaled now.
@@ -519,8 +530,6 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
           tmem_st32(lane_addr + o_col + c * 32, ob);
         }
       }
-      tmem_st32(lane_addr + s_col, pk[0]);
-      tmem_st32(lane_addr + s_col + 32, pk[1]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full[q]);
