@@ -49,6 +49,36 @@ def load_peaks():
                 "source": "fallback"}
 
 
+# ------------------------------------------------------------------ recorded DRAM traffic
+# profiles/traffic.json holds dram__bytes_read.sum + dram__bytes_write.sum per launch
+# from an ncu capture, with the SHA-256 of the sources the kernel was built from;
+# a figure is reported only while those sources are unchanged.
+KERNEL_SOURCES = {
+    "phase1": ["attention_sm100.cu", "common.cuh"],
+    "decode": ["decode.cu", "merge.cu", "common.cuh"],
+}
+
+
+def sources_sha256(kind: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, "block_sparse_attention_phase_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kind: str, workload: str):
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            entry = json.load(f)[workload][kind]
+    except Exception:
+        return None
+    if entry.get("sources_sha256") != sources_sha256(kind):
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
@@ -432,14 +462,16 @@ def main(argv=None):
              "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
              "frac": p1_tflops / peaks["bf16_tflops_sustained"],
              "frac_of_burst": p1_tflops / peaks["bf16_tflops"],
-             "peak_kind": f"bf16 sustained ({peaks['source']})", "traffic": None,
+             "peak_kind": f"bf16 sustained ({peaks['source']})",
+             "traffic": recorded_traffic("phase1", w.name),
              "algorithmic_per_launch": flops, "avg_launch_ms": p1_avg}
     # Decode: per-step duration inside the timed region (partials + merge, consecutive
     # steps overlapping through programmatic launch); "cold" = one step timed alone
     # right after an L2 flush, launch latency included.
     rl_dec = {"bound": "hbm", "kernel": "phase2_decode (partials + merge)", "achieved": dec_gbs,
               "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
-              "peak_kind": f"HBM copy ({peaks['source']})", "traffic": None,
+              "peak_kind": f"HBM copy ({peaks['source']})",
+              "traffic": recorded_traffic("decode", w.name),
               "algorithmic_per_launch": statistics.mean(kv_bytes), "avg_launch_ms": dec_avg,
               "cold_gbs": dec_cold_gbs, "cold_avg_launch_ms": dec_cold_avg,
               "cold_frac": dec_cold_gbs / peaks["hbm_gbs"]}
