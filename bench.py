@@ -375,6 +375,59 @@ def run_reference(args, w, world, rank):
     return 0
 
 
+def block_sweep(args):
+    """Phase-1 throughput against block size, next to dense causal attention (B = L,
+    the same kernel with one block) on the same GPU: B = L/2 .. L/32 at the
+    workload's L (the pages' Figure 5 setting), and a fixed B of 32768 as L grows
+    to 1M (the pages' Figure 6 / Table 5 setting). Prints one JSON line."""
+    import block_sparse_attention_phase_b200 as sa
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    base = workloads.get(args.workload)
+
+    def time_phase1(L, B, reps):
+        w = workloads.Workload("sweep", base.batch, base.num_q_heads, base.num_kv_heads,
+                               base.head_dim, L, B, 1, 1, 0, 0)
+        x = workloads.make_inputs(w, device=device, parts=("ctx",))
+        o = torch.empty_like(x["q_ctx"])
+        for _ in range(3):
+            sa.phase1(x["q_ctx"], x["k_ctx"], x["v_ctx"], B, o=o, want_lse=False)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        torch.cuda.synchronize()
+        ev[0].record()
+        for _ in range(reps):
+            sa.phase1(x["q_ctx"], x["k_ctx"], x["v_ctx"], B, o=o, want_lse=False)
+        ev[1].record()
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[1]) / reps
+        del x, o
+        torch.cuda.empty_cache()
+        return ms, w.phase1_flops()
+
+    rows = []
+    L = base.ctx_len
+    dense_ms, dense_flops = time_phase1(L, L, args.steps)
+    for div in (1, 2, 4, 8, 16, 32):
+        B = L // div
+        ms, flops = (dense_ms, dense_flops) if div == 1 else time_phase1(L, B, args.steps)
+        rows.append({"L": L, "B": B, "n_blocks": div, "ms": ms, "tflops": flops / ms / 1e9,
+                     "ctx_tok_s": base.batch * L / ms * 1e3, "speedup_vs_dense": dense_ms / ms})
+    fixed = []
+    for L2 in (131072, 262144, 524288, 1048576):
+        reps = max(1, args.steps // 4)
+        d_ms, d_fl = time_phase1(L2, L2, reps)
+        s_ms, s_fl = time_phase1(L2, 32768, reps)
+        fixed.append({"L": L2, "B": 32768, "ms": s_ms, "dense_ms": d_ms, "tflops": s_fl / s_ms / 1e9,
+                      "dense_tflops": d_fl / d_ms / 1e9, "speedup_vs_dense": d_ms / s_ms})
+    print(json.dumps({"metric": "Phase-1 time vs block size (dense causal = one block)",
+                      "unit": "ms", "config": {"workload": base.name, "batch": base.batch,
+                                               "num_q_heads": base.num_q_heads,
+                                               "num_kv_heads": base.num_kv_heads,
+                                               "head_dim": base.head_dim},
+                      "block_fraction_sweep": rows, "fixed_block_32k": fixed}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -385,6 +438,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=10.0)
+    ap.add_argument("--block-sweep", action="store_true",
+                    help="time Phase 1 against block size and dense causal attention instead")
     ap.add_argument("--eager", action="store_true",
                     help="issue every call from Python instead of replaying CUDA graphs")
     args = ap.parse_args(argv)
@@ -393,6 +448,8 @@ def main(argv=None):
 
     world, rank, local = setup_dist(args)
     w = workloads.get(args.workload)
+    if args.block_sweep:
+        return block_sweep(args) if rank == 0 else 0
     if args.impl == "reference":
         return run_reference(args, w, world, rank)
 
