@@ -33,7 +33,9 @@ STATUS_NAMES = {0: "STAR_OK", 1: "STAR_ERR_INVALID_ARG", 2: "STAR_ERR_UNSUPPORTE
 
 # Every symbol the header declares; tests check that the library exports them all.
 EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase2_query",
-            "star_attn_phase2_decode", "star_attn_phase2_decode_noalloc", "star_attn_lse_merge", "star_attn_simple_phase1",
+            "star_attn_phase2_decode", "star_attn_phase2_query_paged",
+            "star_attn_phase2_decode_paged", "star_attn_phase2_decode_noalloc",
+            "star_attn_lse_merge", "star_attn_simple_phase1",
             "star_attn_simple_phase2", "star_attn_get_device_status",
             "star_attn_selftest_wait_timeout", "star_attn_selftest_exp2", "star_attn_launch_count",
             "star_attn_status_string", "star_attn_version"]
@@ -71,6 +73,10 @@ def lib() -> ctypes.CDLL:
         "star_attn_phase1": (I32, [SP, P, P, P, P, P, P]),
         "star_attn_phase2_query": (I32, [SP, P, P, P, I64, P, P, P, P, I64, P, P, P, SZ, P]),
         "star_attn_phase2_decode": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P, SZ, P]),
+        "star_attn_phase2_query_paged": (I32, [SP, P, P, P, I64, P, P, P, P, I32, I32, P, I32,
+                                                P, P, P, SZ, P]),
+        "star_attn_phase2_decode_paged": (I32, [SP, P, P, P, P, P, P, P, I32, I32, P, I32, I64,
+                                                 P, P, P, SZ, P]),
         "star_attn_phase2_decode_noalloc": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P]),
         "star_attn_lse_merge": (I32, [P, P, I32, I32, I64, I32, I32, P, P, P]),
         "star_attn_simple_phase1": (I32, [SP, P, P, P, P, P, P]),
@@ -190,6 +196,65 @@ def phase2_decode(q, k, v, k_ctx, v_ctx, k_cache, v_cache, cache_len: int, block
         ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_cache),
         _ptr(v_cache), int(cache_len), k_cache.shape[1], _ptr(o), _ptr(lse), _ptr(workspace),
         workspace.numel(), _stream()), "star_attn_phase2_decode")
+    return o, lse
+
+
+def _page_pool(k_pages, v_pages, page_table):
+    for t, n in ((k_pages, "k_pages"), (v_pages, "v_pages")):
+        _bf16(t, n, 4)
+    if k_pages.shape != v_pages.shape:
+        raise ValueError("k_pages and v_pages must have the same shape")
+    if (not isinstance(page_table, torch.Tensor) or page_table.dtype != torch.int32
+            or page_table.dim() != 2 or not page_table.is_contiguous()
+            or page_table.device != k_pages.device):
+        raise TypeError("page_table must be a contiguous int32 [batch, max_pages] tensor "
+                        "on the pool's device")
+    num_pages, page_size = k_pages.shape[0], k_pages.shape[1]
+    return page_size, num_pages, page_table.shape[1]
+
+
+def phase2_query_paged(q, k, v, k_ctx, v_ctx, k_pages, v_pages, page_table, block_size: int,
+                       scale: Optional[float] = None, o=None, lse=None, workspace=None):
+    """phase2_query() with the query-local cache in a page pool: k_pages/v_pages
+    [num_pages, page_size, Hkv, d] bf16, page_table [b, max_pages] int32; cache row r of
+    sequence i lives in row r % page_size of page page_table[i, r // page_size]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (k_ctx, "k_ctx"), (v_ctx, "v_ctx")):
+        _bf16(t, n, 4)
+    page_size, num_pages, max_pages = _page_pool(k_pages, v_pages, page_table)
+    b, lq, hq, d = q.shape
+    shape = make_shape(b, hq, k_ctx.shape[2], d, k_ctx.shape[1], block_size, scale)
+    workspace = _ws(shape, STAR_PHASE2_QUERY, lq, q.device, workspace)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((b, hq, lq), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_phase2_query_paged(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), lq, _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(k_pages), _ptr(v_pages), page_size, num_pages, _ptr(page_table), max_pages,
+        _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(), _stream()),
+        "star_attn_phase2_query_paged")
+    return o, lse
+
+
+def phase2_decode_paged(q, k, v, k_ctx, v_ctx, k_pages, v_pages, page_table, cache_len: int,
+                        block_size: int, scale: Optional[float] = None, o=None, lse=None,
+                        workspace=None):
+    """phase2_decode() with the query-local cache in a page pool (see phase2_query_paged)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (k_ctx, "k_ctx"), (v_ctx, "v_ctx")):
+        _bf16(t, n, 4)
+    page_size, num_pages, max_pages = _page_pool(k_pages, v_pages, page_table)
+    b, _, hq, d = q.shape
+    shape = make_shape(b, hq, k_ctx.shape[2], d, k_ctx.shape[1], block_size, scale)
+    workspace = _ws(shape, STAR_PHASE2_DECODE, 1, q.device, workspace)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((b, hq, 1), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_phase2_decode_paged(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(k_pages), _ptr(v_pages), page_size, num_pages, _ptr(page_table), max_pages,
+        int(cache_len), _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(), _stream()),
+        "star_attn_phase2_decode_paged")
     return o, lse
 
 

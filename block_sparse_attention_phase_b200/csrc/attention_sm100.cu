@@ -83,6 +83,9 @@ struct AttnArgs {
   int32_t spb, n_ctx, n_splits, n_qt;
   float* o_parts;    // [S, b, Lq, Hq, d]
   float* lse_parts;  // [S, b, Hq, Lq]
+  // paged query-local cache (page_table == null: contiguous)
+  const int32_t* page_table;  // [b, max_pages]
+  int32_t page_size, max_pages;
 };
 
 struct Bars {
@@ -333,17 +336,26 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         } else {
           kv0 = static_cast<int32_t>(it.k0 + 128 * j);
         }
+        // Outer TMA coordinate: the sequence, or for a paged cache the page holding
+        // this 128-row tile (page sizes are multiples of 128).
+        int32_t c3 = it.bb;
+        if constexpr (M == Mode::kQuery) {
+          if (it.cache && a.page_table) {
+            c3 = a.page_table[static_cast<int64_t>(it.bb) * a.max_pages + kv0 / a.page_size];
+            kv0 %= a.page_size;
+          }
+        }
         if (j >= 2 && !wait_or_abort(&bars->k_empty[s], ph ^ 1, bars, a.status)) break;
         mbar_arrive_expect_tx(&bars->k_full[s], kTileBytes);
 #pragma unroll
         for (int c = 0; c < CH; ++c)
-          tma_load_4d(sk + s * kTileBytes + c * kChunkBytes, mk, &bars->k_full[s], c * 64, it.kvh, kv0, it.bb);
+          tma_load_4d(sk + s * kTileBytes + c * kChunkBytes, mk, &bars->k_full[s], c * 64, it.kvh, kv0, c3);
         last_k[s] = j;
         if (j >= 2 && !wait_or_abort(&bars->v_empty[s], ph ^ 1, bars, a.status)) break;
         mbar_arrive_expect_tx(&bars->v_full[s], kTileBytes);
 #pragma unroll
         for (int c = 0; c < CH; ++c)
-          tma_load_4d(sv + s * kTileBytes + c * kChunkBytes, mv, &bars->v_full[s], c * 64, it.kvh, kv0, it.bb);
+          tma_load_4d(sv + s * kTileBytes + c * kChunkBytes, mv, &bars->v_full[s], c * 64, it.kvh, kv0, c3);
         last_v[s] = j;
       }
       // Every copy this thread issued has landed before the CTA may exit (on the
@@ -648,20 +660,30 @@ cudaError_t launch_phase1_t(const Shape& s, const void* q, const void* k, const 
 
 template <int D>
 cudaError_t launch_query_t(const Shape& s, const SplitPlan& p, const void* q, int64_t lq,
-                           const void* kc, const void* vc, const void* k_cache,
-                           const void* v_cache, int64_t cap, float* o_parts, float* lse_parts,
-                           cudaStream_t st) {
+                           const void* kc, const void* vc, const CacheRef& c, float* o_parts,
+                           float* lse_parts, cudaStream_t st) {
   const int G = s.group();
   alignas(64) CUtensorMap m[5];
-  if (!encode_tma_bf16_4d(&m[0], q, D, s.hq, lq, lq, s.b, 64, G, 128 / G, true) ||
-      !encode_tma_bf16_4d(&m[1], kc, D, s.hkv, s.L, s.L, s.b, 64, 1, 128, true) ||
-      !encode_tma_bf16_4d(&m[2], vc, D, s.hkv, s.L, s.L, s.b, 64, 1, 128, true) ||
-      // only the Lq rows written by this call are in bounds: rows past them
-      // (unwritten, any bytes) read as zeros, so P = 0 never meets a NaN there
-      !encode_tma_bf16_4d(&m[3], k_cache, D, s.hkv, lq, cap, s.b, 64, 1, 128, true) ||
-      !encode_tma_bf16_4d(&m[4], v_cache, D, s.hkv, lq, cap, s.b, 64, 1, 128, true))
-    return cudaErrorInvalidValue;
+  bool ok = encode_tma_bf16_4d(&m[0], q, D, s.hq, lq, lq, s.b, 64, G, 128 / G, true) &&
+            encode_tma_bf16_4d(&m[1], kc, D, s.hkv, s.L, s.L, s.b, 64, 1, 128, true) &&
+            encode_tma_bf16_4d(&m[2], vc, D, s.hkv, s.L, s.L, s.b, 64, 1, 128, true);
+  if (c.paged()) {
+    // the page pool [pages, P, Hkv, d]; rows past Lq in the last page were zeroed
+    // by the cache write of this call
+    ok = ok &&
+         encode_tma_bf16_4d(&m[3], c.k, D, s.hkv, c.page_size, c.page_size, c.num_pages, 64, 1, 128, true) &&
+         encode_tma_bf16_4d(&m[4], c.v, D, s.hkv, c.page_size, c.page_size, c.num_pages, 64, 1, 128, true);
+  } else {
+    // only the Lq rows written by this call are in bounds: rows past them
+    // (unwritten, any bytes) read as zeros, so P = 0 never meets a NaN there
+    ok = ok && encode_tma_bf16_4d(&m[3], c.k, D, s.hkv, lq, c.cap, s.b, 64, 1, 128, true) &&
+         encode_tma_bf16_4d(&m[4], c.v, D, s.hkv, lq, c.cap, s.b, 64, 1, 128, true);
+  }
+  if (!ok) return cudaErrorInvalidValue;
   AttnArgs a = base_args(s);
+  a.page_table = c.page_table;
+  a.page_size = c.page_size;
+  a.max_pages = c.max_pages;
   a.lq = lq;
   a.chunk = p.chunk;
   a.spb = p.spb;
@@ -685,13 +707,10 @@ cudaError_t launch_phase1_sm100(const Shape& s, const void* q, const void* k, co
 }
 
 cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q, int64_t lq,
-                              const void* kc, const void* vc, const void* k_cache,
-                              const void* v_cache, int64_t cap, float* o_parts, float* lse_parts,
-                              void* o, float* lse, cudaStream_t st) {
-  cudaError_t e = s.d == 128 ? launch_query_t<128>(s, p, q, lq, kc, vc, k_cache, v_cache, cap,
-                                                   o_parts, lse_parts, st)
-                             : launch_query_t<64>(s, p, q, lq, kc, vc, k_cache, v_cache, cap,
-                                                  o_parts, lse_parts, st);
+                              const void* kc, const void* vc, const CacheRef& c, float* o_parts,
+                              float* lse_parts, void* o, float* lse, cudaStream_t st) {
+  cudaError_t e = s.d == 128 ? launch_query_t<128>(s, p, q, lq, kc, vc, c, o_parts, lse_parts, st)
+                             : launch_query_t<64>(s, p, q, lq, kc, vc, c, o_parts, lse_parts, st);
   if (e != cudaSuccess) return e;
   return launch_merge(o_parts, lse_parts, p.n_splits, s.b, lq, s.hq, s.d, o, lse, st);
 }

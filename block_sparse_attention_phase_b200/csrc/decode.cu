@@ -41,6 +41,9 @@ struct DecodeArgs {
   float* o_parts;    // [S, b, 1, Hq, D]
   float* lse_parts;  // [S, b, Hq, 1]
   uint32_t* status;
+  // paged query-local cache (page_table == null: contiguous [b, cap, Hkv, D])
+  const int32_t* page_table;  // [b, max_pages]; pool [num_pages, page_size, Hkv, D]
+  int32_t page_size, max_pages, num_pages;
 };
 
 constexpr int kTile = 64;      // tokens per TMA tile
@@ -107,11 +110,39 @@ __global__ void __launch_bounds__((kWarps + 1) * 32) decode_partials_kernel(
   if (warp == kWarps) {
     // ---------------- producer warp: the cache append, then TMA loads ----------------
     if (is_cache && lane < D / 8) {
-      const int64_t src = (static_cast<int64_t>(bb) * a.hkv + kvh) * D + lane * 8;
-      const int64_t dst = ((static_cast<int64_t>(bb) * a.cap + a.cache_len) * a.hkv + kvh) * D + lane * 8;
-      *reinterpret_cast<uint4*>(a.k_cache + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
-      *reinterpret_cast<uint4*>(a.v_cache + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
-      fence_proxy_async_global();  // the TMA loads below read this row
+      // Cache row of (this sequence, row r): contiguous [b, cap, Hkv, D], or row
+      // r % P of page table[b][r / P] in the pool [num_pages, P, Hkv, D]. A page id
+      // outside the pool is refused (bounds flag, no write).
+      int64_t page = 0;
+      if (a.page_table) {
+        page = a.page_table[static_cast<int64_t>(bb) * a.max_pages + a.cache_len / a.page_size];
+        if (page < 0 || page >= a.num_pages) {
+          if (lane == 0) atomicOr(a.status, kBoundsFlag);
+          page = -1;
+        }
+      }
+      auto row_off = [&](int64_t r) -> int64_t {
+        const int64_t prow = a.page_table ? page * a.page_size + r % a.page_size
+                                          : static_cast<int64_t>(bb) * a.cap + r;
+        return (prow * a.hkv + kvh) * D + lane * 8;
+      };
+      if (page >= 0) {
+        const int64_t src = (static_cast<int64_t>(bb) * a.hkv + kvh) * D + lane * 8;
+        const int64_t dst = row_off(a.cache_len);
+        *reinterpret_cast<uint4*>(a.k_cache + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
+        *reinterpret_cast<uint4*>(a.v_cache + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
+        if (a.page_table && a.cache_len % a.page_size == 0) {
+          // The append opens a new page: zero its other rows (for this kv-head), so
+          // that tiles reaching past the last valid row read zeros, never stale bytes.
+          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+          for (int64_t r = a.cache_len + 1; r < a.cache_len + a.page_size; ++r) {
+            const int64_t off = row_off(r);
+            *reinterpret_cast<uint4*>(a.k_cache + off) = z;
+            *reinterpret_cast<uint4*>(a.v_cache + off) = z;
+          }
+        }
+      }
+      fence_proxy_async_global();  // the TMA loads below read these rows
     }
     __syncwarp();
     if (lane == 0 && ntiles > 0) {
@@ -122,11 +153,16 @@ __global__ void __launch_bounds__((kWarps + 1) * 32) decode_partials_kernel(
         const uint32_t ph = (i / kStages) & 1;
         if (i >= kStages && !mbar_wait(&empty[stg], ph ^ 1, a.status)) break;
         mbar_arrive_expect_tx(&full[stg], 2 * kTileBytes);
-        const int32_t t0 = static_cast<int32_t>(k0 + static_cast<int64_t>(i) * kTile);
+        int32_t t0 = static_cast<int32_t>(k0 + static_cast<int64_t>(i) * kTile);
+        int32_t c3 = bb;  // the sequence, or for a paged cache the page holding this tile
+        if (is_cache && a.page_table) {
+          c3 = a.page_table[static_cast<int64_t>(bb) * a.max_pages + t0 / a.page_size];
+          t0 %= a.page_size;
+        }
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-          tma_load_4d(kbuf + stg * kTileBytes + c * kChunk, mk, &full[stg], c * 64, kvh, t0, bb);
-          tma_load_4d(vbuf + stg * kTileBytes + c * kChunk, mv, &full[stg], c * 64, kvh, t0, bb);
+          tma_load_4d(kbuf + stg * kTileBytes + c * kChunk, mk, &full[stg], c * 64, kvh, t0, c3);
+          tma_load_4d(vbuf + stg * kTileBytes + c * kChunk, mv, &full[stg], c * 64, kvh, t0, c3);
         }
       }
     }
@@ -288,15 +324,23 @@ __global__ void __launch_bounds__((kWarps + 1) * 32) decode_partials_kernel(
 
 template <int D, int G>
 cudaError_t launch_decode_t(const Shape& s, const SplitPlan& p, const DecodeArgs& a,
-                            const void* kc, const void* vc, cudaStream_t st) {
+                            const void* kc, const void* vc, int32_t num_pages, cudaStream_t st) {
   alignas(64) CUtensorMap m[4];
-  // The cache map covers the cached rows and the new one; rows past them read as zeros.
-  const uint64_t cache_rows = static_cast<uint64_t>(a.cache_len + 1);
-  const bool ok =
-      encode_tma_bf16_4d(&m[0], kc, D, s.hkv, s.L, s.L, s.b, 64, 1, kTile, true) &&
-      encode_tma_bf16_4d(&m[1], vc, D, s.hkv, s.L, s.L, s.b, 64, 1, kTile, true) &&
-      encode_tma_bf16_4d(&m[2], a.k_cache, D, s.hkv, cache_rows, a.cap, s.b, 64, 1, kTile, true) &&
-      encode_tma_bf16_4d(&m[3], a.v_cache, D, s.hkv, cache_rows, a.cap, s.b, 64, 1, kTile, true);
+  bool ok = encode_tma_bf16_4d(&m[0], kc, D, s.hkv, s.L, s.L, s.b, 64, 1, kTile, true) &&
+            encode_tma_bf16_4d(&m[1], vc, D, s.hkv, s.L, s.L, s.b, 64, 1, kTile, true);
+  if (a.page_table) {
+    // The page pool [pages, P, Hkv, D]; rows past the valid ones in a sequence's
+    // last page hold zeros (written when the page was opened).
+    ok = ok &&
+         encode_tma_bf16_4d(&m[2], a.k_cache, D, s.hkv, a.page_size, a.page_size, num_pages, 64, 1, kTile, true) &&
+         encode_tma_bf16_4d(&m[3], a.v_cache, D, s.hkv, a.page_size, a.page_size, num_pages, 64, 1, kTile, true);
+  } else {
+    // The cache map covers the cached rows and the new one; rows past them read as zeros.
+    const uint64_t cache_rows = static_cast<uint64_t>(a.cache_len + 1);
+    ok = ok &&
+         encode_tma_bf16_4d(&m[2], a.k_cache, D, s.hkv, cache_rows, a.cap, s.b, 64, 1, kTile, true) &&
+         encode_tma_bf16_4d(&m[3], a.v_cache, D, s.hkv, cache_rows, a.cap, s.b, 64, 1, kTile, true);
+  }
   if (!ok) return cudaErrorInvalidValue;
   const size_t smem = 2 * kStages * (D / 64) * kTile * 128 + 2 * kStages * sizeof(uint64_t) + 1024;
   auto kern = decode_partials_kernel<D, G>;
@@ -314,17 +358,20 @@ cudaError_t launch_decode_t(const Shape& s, const SplitPlan& p, const DecodeArgs
 
 cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const void* q,
                                    const void* k_new, const void* v_new, const void* kc,
-                                   const void* vc, void* k_cache, void* v_cache, int64_t cache_len,
-                                   int64_t cap, float* o_parts, float* lse_parts,
-                                   cudaStream_t st) {
+                                   const void* vc, const CacheRef& c, int64_t cache_len,
+                                   float* o_parts, float* lse_parts, cudaStream_t st) {
   DecodeArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k_new = static_cast<const __nv_bfloat16*>(k_new);
   a.v_new = static_cast<const __nv_bfloat16*>(v_new);
-  a.k_cache = static_cast<__nv_bfloat16*>(k_cache);
-  a.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  a.k_cache = static_cast<__nv_bfloat16*>(c.k);
+  a.v_cache = static_cast<__nv_bfloat16*>(c.v);
   a.cache_len = cache_len;
-  a.cap = cap;
+  a.cap = c.cap;
+  a.page_table = c.page_table;
+  a.page_size = c.page_size;
+  a.max_pages = c.max_pages;
+  a.num_pages = c.num_pages;
   a.L = s.L;
   a.B = s.B;
   a.chunk = p.chunk;
@@ -339,7 +386,7 @@ cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const voi
   a.status = device_status_word();
   const int G = s.group();
 #define STAR_DECODE_CASE(DD, GG) \
-  if (s.d == DD && G == GG) return launch_decode_t<DD, GG>(s, p, a, kc, vc, st);
+  if (s.d == DD && G == GG) return launch_decode_t<DD, GG>(s, p, a, kc, vc, c.num_pages, st);
   STAR_DECODE_CASE(128, 1) STAR_DECODE_CASE(128, 2) STAR_DECODE_CASE(128, 4)
   STAR_DECODE_CASE(128, 8) STAR_DECODE_CASE(64, 1) STAR_DECODE_CASE(64, 2)
   STAR_DECODE_CASE(64, 4) STAR_DECODE_CASE(64, 8)

@@ -66,6 +66,63 @@ SplitPlan make_plan(const Shape& s, int64_t target_ctas) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Page-pool arguments: a tile (128 query-pass rows, 64 decode rows) must never
+// straddle two pages, and TMA coordinates of a page are 32-bit.
+star_status_t check_pages(int32_t page_size, int32_t num_pages, const int32_t* page_table,
+                          int32_t max_pages) {
+  if (page_size < 128 || page_size % 128 != 0) return STAR_ERR_INVALID_ARG;
+  if (num_pages < 1 || max_pages < 1 || !page_table) return STAR_ERR_INVALID_ARG;
+  if (!aligned4(page_table)) return STAR_ERR_INVALID_ARG;
+  return STAR_OK;
+}
+
+CacheRef paged_ref(void* k, void* v, int32_t page_size, int32_t num_pages,
+                   const int32_t* page_table, int32_t max_pages) {
+  CacheRef c;
+  c.k = k;
+  c.v = v;
+  c.page_table = page_table;
+  c.page_size = page_size;
+  c.num_pages = num_pages;
+  c.max_pages = max_pages;
+  return c;
+}
+
+// Workspace = [o_parts (256-B aligned)][lse_parts].
+float* lse_parts_of(void* workspace, const Shape& s, const SplitPlan& p, int64_t rows) {
+  const size_t per = static_cast<size_t>(p.n_splits) * s.b * rows * s.hq;
+  return reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                  align256(per * s.d * sizeof(float)));
+}
+
+// Phase-2 query pass on validated arguments: cache append, then partials + merge.
+star_status_t run_query(const Shape& s, const void* q, const void* k, const void* v,
+                        int64_t query_len, const void* k_ctx, const void* v_ctx,
+                        const CacheRef& c, void* o, float* lse, void* workspace,
+                        cudaStream_t cs) {
+  const SplitPlan plan = query_plan(s, query_len);
+  cudaError_t e = launch_cache_write(s, k, v, query_len, c, cs);
+  if (e != cudaSuccess) return STAR_ERR_CUDA;
+  e = launch_query_path(s, plan, q, query_len, k_ctx, v_ctx, c, static_cast<float*>(workspace),
+                        lse_parts_of(workspace, s, plan, query_len), o, lse, cs);
+  return e == cudaSuccess ? STAR_OK : STAR_ERR_CUDA;
+}
+
+// Phase-2 decode step on validated arguments: partials (with the append) + merge.
+star_status_t run_decode(const Shape& s, const void* q, const void* k, const void* v,
+                         const void* k_ctx, const void* v_ctx, const CacheRef& c,
+                         int64_t cache_len, void* o, float* lse, void* workspace,
+                         cudaStream_t cs) {
+  const SplitPlan plan = decode_plan(s);
+  float* o_parts = static_cast<float*>(workspace);
+  float* lse_parts = lse_parts_of(workspace, s, plan, 1);
+  cudaError_t e = launch_decode_partials(s, plan, q, k, v, k_ctx, v_ctx, c, cache_len, o_parts,
+                                         lse_parts, cs);
+  if (e != cudaSuccess) return STAR_ERR_CUDA;
+  e = launch_merge(o_parts, lse_parts, plan.n_splits, s.b, 1, s.hq, s.d, o, lse, cs);
+  return e == cudaSuccess ? STAR_OK : STAR_ERR_CUDA;
+}
+
 std::atomic<uint64_t> g_launches{0};
 
 }  // namespace
@@ -153,19 +210,14 @@ STAR_ATTN_API star_status_t star_attn_phase2_query(
     if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
   if (!star::aligned4(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
   if (query_len > cache_capacity) return STAR_ERR_CACHE_FULL;
-  const star::SplitPlan plan = star::query_plan(s, query_len);
-  const size_t need = star::partial_bytes(s, plan, query_len);
+  const size_t need = star::partial_bytes(s, star::query_plan(s, query_len), query_len);
   if (!workspace || workspace_bytes < need) return STAR_ERR_WORKSPACE;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = star::launch_cache_write(s, k, v, query_len, k_cache, v_cache, cache_capacity, 0, cs);
-  if (e != cudaSuccess) return STAR_ERR_CUDA;
-  float* o_parts = static_cast<float*>(workspace);
-  const size_t per = static_cast<size_t>(plan.n_splits) * s.b * query_len * s.hq;
-  float* lse_parts = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                              ((per * s.d * sizeof(float) + 255) & ~size_t(255)));
-  e = star::launch_query_path(s, plan, q, query_len, k_ctx, v_ctx, k_cache, v_cache,
-                              cache_capacity, o_parts, lse_parts, o, lse, cs);
-  return star::cuda_status(e);
+  star::CacheRef c;
+  c.k = k_cache;
+  c.v = v_cache;
+  c.cap = cache_capacity;
+  return star::run_query(s, q, k, v, query_len, k_ctx, v_ctx, c, o, lse, workspace,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 STAR_ATTN_API star_status_t star_attn_phase2_decode(
@@ -182,19 +234,62 @@ STAR_ATTN_API star_status_t star_attn_phase2_decode(
     if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
   if (!star::aligned4(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
   if (cache_len + 1 > cache_capacity) return STAR_ERR_CACHE_FULL;
-  const star::SplitPlan plan = star::decode_plan(s);
-  const size_t need = star::partial_bytes(s, plan, 1);
+  if (!workspace || workspace_bytes < star::partial_bytes(s, star::decode_plan(s), 1))
+    return STAR_ERR_WORKSPACE;
+  star::CacheRef c;
+  c.k = k_cache;
+  c.v = v_cache;
+  c.cap = cache_capacity;
+  return star::run_decode(s, q, k, v, k_ctx, v_ctx, c, cache_len, o, lse, workspace,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+STAR_ATTN_API star_status_t star_attn_phase2_query_paged(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
+    int64_t query_len, const void* k_ctx, const void* v_ctx, void* k_pages, void* v_pages,
+    int32_t page_size, int32_t num_pages, const int32_t* page_table, int32_t max_pages, void* o,
+    float* lse, void* workspace, size_t workspace_bytes, star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (query_len < 1) return STAR_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, k_ctx, v_ctx, k_pages, v_pages, o};
+  for (const void* p : ptrs)
+    if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned4(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
+  st = star::check_pages(page_size, num_pages, page_table, max_pages);
+  if (st != STAR_OK) return st;
+  if ((query_len + page_size - 1) / page_size > max_pages) return STAR_ERR_CACHE_FULL;
+  const size_t need = star::partial_bytes(s, star::query_plan(s, query_len), query_len);
   if (!workspace || workspace_bytes < need) return STAR_ERR_WORKSPACE;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  float* o_parts = static_cast<float*>(workspace);
-  const size_t per = static_cast<size_t>(plan.n_splits) * s.b * s.hq;
-  float* lse_parts = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                              ((per * s.d * sizeof(float) + 255) & ~size_t(255)));
-  cudaError_t e = star::launch_decode_partials(s, plan, q, k, v, k_ctx, v_ctx, k_cache, v_cache,
-                                               cache_len, cache_capacity, o_parts, lse_parts, cs);
-  if (e != cudaSuccess) return STAR_ERR_CUDA;
-  e = star::launch_merge(o_parts, lse_parts, plan.n_splits, s.b, 1, s.hq, s.d, o, lse, cs);
-  return star::cuda_status(e);
+  const star::CacheRef c = star::paged_ref(k_pages, v_pages, page_size, num_pages, page_table,
+                                           max_pages);
+  return star::run_query(s, q, k, v, query_len, k_ctx, v_ctx, c, o, lse, workspace,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+STAR_ATTN_API star_status_t star_attn_phase2_decode_paged(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
+    const void* k_ctx, const void* v_ctx, void* k_pages, void* v_pages, int32_t page_size,
+    int32_t num_pages, const int32_t* page_table, int32_t max_pages, int64_t cache_len, void* o,
+    float* lse, void* workspace, size_t workspace_bytes, star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (cache_len < 0) return STAR_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, k_ctx, v_ctx, k_pages, v_pages, o};
+  for (const void* p : ptrs)
+    if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned4(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
+  st = star::check_pages(page_size, num_pages, page_table, max_pages);
+  if (st != STAR_OK) return st;
+  if (cache_len / page_size + 1 > max_pages) return STAR_ERR_CACHE_FULL;
+  if (!workspace || workspace_bytes < star::partial_bytes(s, star::decode_plan(s), 1))
+    return STAR_ERR_WORKSPACE;
+  const star::CacheRef c = star::paged_ref(k_pages, v_pages, page_size, num_pages, page_table,
+                                           max_pages);
+  return star::run_decode(s, q, k, v, k_ctx, v_ctx, c, cache_len, o, lse, workspace,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 STAR_ATTN_API star_status_t star_attn_lse_merge(const float* o_parts, const float* lse_parts,

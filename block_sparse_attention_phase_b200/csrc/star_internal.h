@@ -64,6 +64,18 @@ cudaError_t launch_programmatic(void (*kern)(Params...), dim3 grid, dim3 block, 
 }
 #endif
 
+// Where the query-local cache rows live: one contiguous [b, cap, Hkv, d] buffer
+// (page_table == nullptr), or pages of a pool [num_pages, page_size, Hkv, d] with
+// page_table [b, max_pages].
+struct CacheRef {
+  void* k = nullptr;
+  void* v = nullptr;
+  int64_t cap = 0;               // contiguous: rows per sequence
+  const int32_t* page_table = nullptr;
+  int32_t page_size = 0, num_pages = 0, max_pages = 0;
+  bool paged() const { return page_table != nullptr; }
+};
+
 // Device status word of the current device (address valid on that device).
 uint32_t* device_status_word();
 
@@ -77,20 +89,20 @@ cudaError_t launch_simple_phase2(const Shape& s, const void* q, int64_t rows, co
 cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int32_t n_splits,
                          int32_t b, int64_t tokens, int32_t heads, int32_t d, void* o,
                          float* lse, cudaStream_t st);
+// Cache rows [0, rows) <- k, v [b, rows, Hkv, d]; for a paged cache, also zero
+// the rest of the page holding row rows-1.
 cudaError_t launch_cache_write(const Shape& s, const void* k, const void* v, int64_t rows,
-                               void* kc, void* vc, int64_t cap, int64_t row0, cudaStream_t st);
+                               const CacheRef& c, cudaStream_t st);
 cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const void* q,
                                    const void* k_new, const void* v_new, const void* kc,
-                                   const void* vc, void* k_cache, void* v_cache, int64_t cache_len,
-                                   int64_t cap, float* o_parts, float* lse_parts,
-                                   cudaStream_t st);
+                                   const void* vc, const CacheRef& c, int64_t cache_len,
+                                   float* o_parts, float* lse_parts, cudaStream_t st);
 cudaError_t launch_phase1_sm100(const Shape& s, const void* q, const void* k, const void* v,
                                 void* o, float* lse, cudaStream_t st);
 // Phase-2 query tokens after their KV is in the cache: partials + merge into o/lse.
 cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q, int64_t lq,
-                              const void* kc, const void* vc, const void* k_cache,
-                              const void* v_cache, int64_t cap, float* o_parts, float* lse_parts,
-                              void* o, float* lse, cudaStream_t st);
+                              const void* kc, const void* vc, const CacheRef& c, float* o_parts,
+                              float* lse_parts, void* o, float* lse, cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t wait_ns, cudaStream_t st);
 cudaError_t launch_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t st);
 

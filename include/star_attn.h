@@ -145,6 +145,37 @@ STAR_ATTN_API star_status_t star_attn_phase2_decode(
     star_stream_t stream);
 
 /*
+ * Paged query-local cache (paperhub.cn page, the authors' response to Reviewer
+ * dKGV, item 3 "Compatibility with Parallelism Methods and Serving Frameworks":
+ * PagedAttention-style memory management applies within each host to its local
+ * KV cache). Same computation as star_attn_phase2_query() /
+ * star_attn_phase2_decode(); only where the cache rows live differs:
+ *   k_pages, v_pages [num_pages, page_size, Hkv, d] bf16 — a pool shared by the batch;
+ *   page_table [batch, max_pages] int32 (device) — cache row r of sequence b is row
+ *     r % page_size of page page_table[b * max_pages + r / page_size].
+ * page_size must be a positive multiple of 128 (a tile never straddles pages);
+ * every page id a call touches must lie in [0, num_pages) and each sequence's pages
+ * must be distinct. Rows past the valid ones in a sequence's last page are written
+ * with zeros by these calls (the query call zero-fills the rest of the page holding
+ * its last row; a decode step that starts a new page zero-fills that page), so the
+ * pool needs no initialisation.
+ * Errors: STAR_ERR_CACHE_FULL if the rows to append need more than max_pages pages;
+ * STAR_ERR_INVALID_ARG for a bad page_size, num_pages or max_pages.
+ * No counterpart on the pages beyond the reference to PagedAttention.
+ */
+STAR_ATTN_API star_status_t star_attn_phase2_query_paged(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
+    int64_t query_len, const void* k_ctx, const void* v_ctx, void* k_pages, void* v_pages,
+    int32_t page_size, int32_t num_pages, const int32_t* page_table, int32_t max_pages, void* o,
+    float* lse, void* workspace, size_t workspace_bytes, star_stream_t stream);
+
+STAR_ATTN_API star_status_t star_attn_phase2_decode_paged(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
+    const void* k_ctx, const void* v_ctx, void* k_pages, void* v_pages, int32_t page_size,
+    int32_t num_pages, const int32_t* page_table, int32_t max_pages, int64_t cache_len, void* o,
+    float* lse, void* workspace, size_t workspace_bytes, star_stream_t stream);
+
+/*
  * The decode step of star_attn_phase2_decode() for callers that cannot allocate
  * device memory where they decode (a serving runtime whose pooled allocator owns
  * all of the GPU's memory, code that must avoid the implicit synchronisation of

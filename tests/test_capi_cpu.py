@@ -106,3 +106,34 @@ def test_binding_checks_tensors_before_calling():
     q = torch.zeros(1, 8, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         sa.phase1(q, q, q, 4)  # CPU tensors are refused: there is no CPU path
+
+
+def test_paged_entry_points_reject_bad_pools():
+    L = sa.lib()
+    s = sa.make_shape(1, 4, 2, 128, 100, 10)
+    F = ctypes.c_void_p(FAKE)
+    needd = sa.workspace_bytes(s, sa.STAR_PHASE2_DECODE)
+    needq = sa.workspace_bytes(s, sa.STAR_PHASE2_QUERY, 200)
+
+    def dec(page_size, num_pages, table, max_pages, cache_len, ws=needd):
+        return L.star_attn_phase2_decode_paged(ctypes.byref(s), F, F, F, F, F, F, F, page_size,
+                                               num_pages, table, max_pages, cache_len, F, None,
+                                               F, ws, None)
+
+    def qry(lq, page_size, num_pages, table, max_pages, ws=needq):
+        return L.star_attn_phase2_query_paged(ctypes.byref(s), F, F, F, lq, F, F, F, F,
+                                              page_size, num_pages, table, max_pages, F, None,
+                                              F, ws, None)
+
+    T = ctypes.c_void_p(FAKE)
+    assert dec(100, 4, T, 2, 0) == 1          # page size not a multiple of 128
+    assert dec(64, 4, T, 2, 0) == 1
+    assert dec(128, 0, T, 2, 0) == 1          # empty pool
+    assert dec(128, 4, None, 2, 0) == 1       # no page table
+    assert dec(128, 4, ctypes.c_void_p(FAKE + 2), 2, 0) == 1  # misaligned table
+    assert dec(128, 4, T, 0, 0) == 1          # no page slots
+    assert dec(128, 4, T, 2, 256) == 4        # row 256 needs a third page
+    assert dec(128, 4, T, 2, 255, needd - 1) == 3
+    assert qry(200, 128, 4, T, 1) == 4        # 200 rows need two pages
+    assert qry(200, 256, 4, T, 1, 0) == 3     # fits one page, but no workspace
+    assert qry(0, 128, 4, T, 2) == 1
