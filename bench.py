@@ -55,7 +55,8 @@ def load_peaks():
 # a figure is reported only while those sources are unchanged.
 KERNEL_SOURCES = {
     "phase1": ["attention_sm100.cu", "common.cuh"],
-    "decode": ["decode.cu", "merge.cu", "common.cuh"],
+    "decode": ["decode.cu", "common.cuh"],
+    "decode_separate": ["decode.cu", "merge.cu", "common.cuh"],
 }
 
 
@@ -144,12 +145,13 @@ class ClockSampler:
 class Step:
     """One whole hot-path pass over resident inputs, with CUDA events per phase."""
 
-    def __init__(self, w, x, device):
+    def __init__(self, w, x, device, fused_decode: bool = True):
         import block_sparse_attention_phase_b200 as sa
         self.sa = sa
         self.w, self.x = w, x
         self.layer = sa.StarAttentionLayer(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim,
-                                           w.ctx_len, w.block_size, w.cache_capacity, device=device)
+                                           w.ctx_len, w.block_size, w.cache_capacity, device=device,
+                                           fused_decode=fused_decode)
         b, L, hq, d = w.batch, w.ctx_len, w.num_q_heads, w.head_dim
         self.o_ctx = torch.empty((b, L, hq, d), dtype=torch.bfloat16, device=device)
         self.lse_ctx = torch.empty((b, hq, L), dtype=torch.float32, device=device)
@@ -440,6 +442,8 @@ def main(argv=None):
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     ap.add_argument("--block-sweep", action="store_true",
                     help="time Phase 1 against block size and dense causal attention instead")
+    ap.add_argument("--decode-merge", default="fused", choices=["fused", "separate"],
+                    help="decode step as one kernel (last-CTA merge) or partials + merge kernel")
     ap.add_argument("--eager", action="store_true",
                     help="issue every call from Python instead of replaying CUDA graphs")
     args = ap.parse_args(argv)
@@ -457,7 +461,8 @@ def main(argv=None):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     x = workloads.make_inputs(w, device=device, seed=w.seed + rank)
-    step = Step(w, x, device)
+    fused = args.decode_merge == "fused"
+    step = Step(w, x, device, fused_decode=fused)
     peaks = load_peaks()
 
     clocks = ClockSampler(torch.cuda.current_device())
@@ -525,10 +530,12 @@ def main(argv=None):
     # Decode: per-step duration inside the timed region (partials + merge, consecutive
     # steps overlapping through programmatic launch); "cold" = one step timed alone
     # right after an L2 flush, launch latency included.
-    rl_dec = {"bound": "hbm", "kernel": "phase2_decode (partials + merge)", "achieved": dec_gbs,
+    dec_kernel = ("phase2_decode (one kernel: partials + last-CTA merge)" if fused else
+                  "phase2_decode (partials kernel + merge kernel)")
+    rl_dec = {"bound": "hbm", "kernel": dec_kernel, "achieved": dec_gbs,
               "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
               "peak_kind": f"HBM copy ({peaks['source']})",
-              "traffic": recorded_traffic("decode", w.name),
+              "traffic": recorded_traffic("decode" if fused else "decode_separate", w.name),
               "algorithmic_per_launch": statistics.mean(kv_bytes), "avg_launch_ms": dec_avg,
               "cold_gbs": dec_cold_gbs, "cold_avg_launch_ms": dec_cold_avg,
               "cold_frac": dec_cold_gbs / peaks["hbm_gbs"]}
@@ -559,6 +566,7 @@ def main(argv=None):
                        "query_len": w.query_len, "decode_steps": w.decode_steps,
                        "planted_pairs": w.planted_pairs, "parallelism": f"replicas{world}",
                        "launch": "eager" if args.eager else "cuda-graph replay per phase",
+                       "decode_merge": args.decode_merge,
                        "l2": "256 MiB write before every step; every decode step reads "
                              f"{w.decode_kv_bytes(0) / 1e6:.1f} MB of KV"},
             "phase1": {"ms": p1_avg, "tok_s": tokens / (p1_avg / 1e3), "tflops": p1_tflops,

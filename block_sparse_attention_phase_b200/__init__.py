@@ -26,14 +26,15 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libstarattn.so")
 
-STAR_PHASE1, STAR_PHASE2_QUERY, STAR_PHASE2_DECODE = 1, 2, 3
+STAR_PHASE1, STAR_PHASE2_QUERY, STAR_PHASE2_DECODE, STAR_PHASE2_DECODE_FUSED = 1, 2, 3, 4
 STATUS_NAMES = {0: "STAR_OK", 1: "STAR_ERR_INVALID_ARG", 2: "STAR_ERR_UNSUPPORTED",
                 3: "STAR_ERR_WORKSPACE", 4: "STAR_ERR_CACHE_FULL", 5: "STAR_ERR_CUDA",
                 6: "STAR_ERR_TIMEOUT"}
 
 # Every symbol the header declares; tests check that the library exports them all.
 EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase2_query",
-            "star_attn_phase2_decode", "star_attn_phase2_query_paged",
+            "star_attn_phase2_decode", "star_attn_phase2_decode_fused",
+            "star_attn_phase2_query_paged",
             "star_attn_phase2_decode_paged", "star_attn_phase2_decode_noalloc",
             "star_attn_lse_merge", "star_attn_simple_phase1",
             "star_attn_simple_phase2", "star_attn_get_device_status",
@@ -73,6 +74,8 @@ def lib() -> ctypes.CDLL:
         "star_attn_phase1": (I32, [SP, P, P, P, P, P, P]),
         "star_attn_phase2_query": (I32, [SP, P, P, P, I64, P, P, P, P, I64, P, P, P, SZ, P]),
         "star_attn_phase2_decode": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P, SZ, P]),
+        "star_attn_phase2_decode_fused": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P, SZ,
+                                                 P]),
         "star_attn_phase2_query_paged": (I32, [SP, P, P, P, I64, P, P, P, P, I32, I32, P, I32,
                                                 P, P, P, SZ, P]),
         "star_attn_phase2_decode_paged": (I32, [SP, P, P, P, P, P, P, P, I32, I32, P, I32, I64,
@@ -258,6 +261,41 @@ def phase2_decode_paged(q, k, v, k_ctx, v_ctx, k_pages, v_pages, page_table, cac
     return o, lse
 
 
+def fused_decode_workspace(batch, num_q_heads, num_kv_heads, head_dim, ctx_len, block_size,
+                           device, scale: Optional[float] = None) -> torch.Tensor:
+    """A zeroed workspace for phase2_decode_fused() (reusable across its steps)."""
+    shape = make_shape(batch, num_q_heads, num_kv_heads, head_dim, ctx_len, block_size, scale)
+    need = workspace_bytes(shape, STAR_PHASE2_DECODE_FUSED)
+    if need == 0:
+        raise ValueError("unsupported shape")
+    return torch.zeros(need, dtype=torch.uint8, device=device)
+
+
+def phase2_decode_fused(q, k, v, k_ctx, v_ctx, k_cache, v_cache, cache_len: int,
+                        block_size: int, scale: Optional[float] = None, o=None, lse=None,
+                        workspace=None):
+    """phase2_decode() as one kernel (partials + last-CTA merge). `workspace` must come
+    from fused_decode_workspace() (zeroed once, left zeroed by every call); one is made
+    when it is None."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (k_ctx, "k_ctx"), (v_ctx, "v_ctx"),
+                 (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _bf16(t, n, 4)
+    b, _, hq, d = q.shape
+    shape = make_shape(b, hq, k_ctx.shape[2], d, k_ctx.shape[1], block_size, scale)
+    if workspace is None:
+        workspace = fused_decode_workspace(b, hq, k_ctx.shape[2], d, k_ctx.shape[1],
+                                           block_size, q.device, scale)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((b, hq, 1), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_phase2_decode_fused(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_cache),
+        _ptr(v_cache), int(cache_len), k_cache.shape[1], _ptr(o), _ptr(lse), _ptr(workspace),
+        workspace.numel(), _stream()), "star_attn_phase2_decode_fused")
+    return o, lse
+
+
 def lse_merge(o_parts: torch.Tensor, lse_parts: torch.Tensor):
     """o_parts [S, b, T, H, d] fp32, lse_parts [S, b, H, T] fp32 -> (o bf16 [b, T, H, d], lse)."""
     S, b, T, H, d = o_parts.shape
@@ -339,7 +377,8 @@ class StarAttentionLayer:
     """
 
     def __init__(self, batch, num_q_heads, num_kv_heads, head_dim, ctx_len, block_size,
-                 cache_capacity, device="cuda", scale: Optional[float] = None):
+                 cache_capacity, device="cuda", scale: Optional[float] = None,
+                 fused_decode: bool = True):
         self.shape = make_shape(batch, num_q_heads, num_kv_heads, head_dim, ctx_len, block_size,
                                 scale)
         self.block_size = block_size
@@ -349,8 +388,16 @@ class StarAttentionLayer:
         self.v_cache = torch.empty_like(self.k_cache)
         self.cache_len = 0
         self.k_ctx = self.v_ctx = None
-        self.ws_decode = torch.empty(max(256, workspace_bytes(self.shape, STAR_PHASE2_DECODE)),
-                                     dtype=torch.uint8, device=device)
+        # Decode steps run as one kernel each (partials + last-CTA merge) unless
+        # fused_decode is False (partial kernel, then a merge kernel).
+        self.fused_decode = fused_decode
+        if fused_decode:
+            self.ws_decode = fused_decode_workspace(batch, num_q_heads, num_kv_heads, head_dim,
+                                                    ctx_len, block_size, device, scale)
+        else:
+            self.ws_decode = torch.empty(
+                max(256, workspace_bytes(self.shape, STAR_PHASE2_DECODE)), dtype=torch.uint8,
+                device=device)
         self.ws_query = None
 
     def prefill(self, q, k, v, o=None, lse=None):
@@ -369,8 +416,8 @@ class StarAttentionLayer:
         return out
 
     def decode(self, q, k, v, o=None, lse=None):
-        out = phase2_decode(q, k, v, self.k_ctx, self.v_ctx, self.k_cache, self.v_cache,
-                            self.cache_len, self.block_size, self.scale, o=o, lse=lse,
-                            workspace=self.ws_decode)
+        fn = phase2_decode_fused if self.fused_decode else phase2_decode
+        out = fn(q, k, v, self.k_ctx, self.v_ctx, self.k_cache, self.v_cache, self.cache_len,
+                 self.block_size, self.scale, o=o, lse=lse, workspace=self.ws_decode)
         self.cache_len += 1
         return out

@@ -44,12 +44,171 @@ struct DecodeArgs {
   // paged query-local cache (page_table == null: contiguous [b, cap, Hkv, D])
   const int32_t* page_table;  // [b, max_pages]; pool [num_pages, page_size, Hkv, D]
   int32_t page_size, max_pages, num_pages;
+  // fused merge (counters == null: partials only, a separate merge kernel follows)
+  __nv_bfloat16* o;    // [b, 1, Hq, D]
+  float* lse;          // [b, Hq, 1]
+  uint32_t* counters;  // [b * Hkv], zero between calls
 };
 
 constexpr int kTile = 64;      // tokens per TMA tile
 constexpr int kWarps = 4;      // consumer warps (16 tokens of each tile apiece)
 constexpr int kStages = 3;
 constexpr float kRescaleLog2 = 8.f;
+
+// The fused merge reuses the KV ring: S x G split weights, then one fp32 sum of
+// the G x D outputs per consumer warp.
+STAR_HD constexpr size_t ring_bytes(int d) { return size_t{2} * kStages * (d / 64) * kTile * 128; }
+STAR_HD constexpr size_t fused_weights_bytes(int64_t n_splits, int g) {
+  return (static_cast<size_t>(n_splits) * g * 4 + 15) & ~size_t(15);
+}
+STAR_HD constexpr size_t fused_merge_bytes(int64_t n_splits, int g, int d) {
+  return fused_weights_bytes(n_splits, g) + size_t{kWarps} * g * d * 4;
+}
+
+// Fused merge, run by the consumer threads of every CTA after it has stored its
+// partial: the CTA that completes the count of its (sequence, kv-head) is the
+// last one, all the other splits' partials are in memory, and it combines them
+// (the query host's aggregation: M = max lse_s, W = sum exp(lse_s - M),
+// o = sum exp(lse_s - M) o_s / W, lse = M + ln W) for its G heads. It also puts
+// the counter back to zero for the next call.
+//
+// The combine is bound by L2 latency, so it is spread wide: the S x G split
+// LSEs are staged in shared memory in one pass and turned into weights there;
+// then the 4 warps take the splits in turn (warp w: splits w, w + 4, ...), each
+// lane owning float4 columns of the split's contiguous G x D partial block, with
+// several splits' loads in flight; the warps' sums meet in shared memory.
+template <int D, int G>
+__device__ __forceinline__ void merge_if_last(const DecodeArgs& a, int bb, int kvh,
+                                              uint8_t* smem) {
+  __shared__ int s_last;
+  __shared__ float s_red[kWarps][G];
+  __shared__ float s_m[G], s_w[G];
+  __threadfence();  // this thread's partial stores, before the count
+  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
+  const int tid = threadIdx.x;  // 0 .. 127 (the consumer warps)
+  if (tid == 0) {
+    uint32_t* ctr = a.counters + blockIdx.y;
+    const uint32_t prev = atomicAdd(ctr, 1u);
+    const int last = prev == gridDim.x - 1;
+    if (last) atomicExch(ctr, 0u);  // every split of this launch has counted
+    s_last = last;
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
+  if (!s_last) return;
+  __threadfence();
+
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int S = gridDim.x;
+  const int64_t row0 = static_cast<int64_t>(bb) * a.hq + kvh * G;  // split 0, first head
+  const int64_t stride = static_cast<int64_t>(a.b) * a.hq;         // rows per split
+  float* wts = reinterpret_cast<float*>(smem);                     // [S][G]
+  float4* red = reinterpret_cast<float4*>(smem + fused_weights_bytes(S, G));  // [kWarps][G*D/4]
+
+  // 1. the LSEs -> shared memory; per-head maximum
+  float m[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) m[h] = -INFINITY;
+  for (int i = tid; i < S * G; i += kWarps * 32) {
+    const int sp = i / G, h = i % G;
+    const float l = __ldcg(a.lse_parts + row0 + sp * stride + h);
+    wts[i] = l;
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh)
+      if (hh == h) m[hh] = fmaxf(m[hh], l);
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], off));
+    if (lane == 0) s_red[warp][h] = m[h];
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
+  if (tid < G) {
+    float mm = s_red[0][tid];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) mm = fmaxf(mm, s_red[w][tid]);
+    s_m[tid] = mm;
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
+
+  // 2. weights exp(lse_s - M) in place (0 for an empty split or an all-empty head); sums
+  float wsum[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) wsum[h] = 0.f;
+  for (int i = tid; i < S * G; i += kWarps * 32) {
+    const int h = i % G;
+    const float M = s_m[h];
+    const float wv = M == -INFINITY ? 0.f : expf(wts[i] - M);
+    wts[i] = wv;
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh)
+      if (hh == h) wsum[hh] += wv;
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) wsum[h] += __shfl_xor_sync(0xffffffffu, wsum[h], off);
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");  // s_red reads above are done
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+    if (lane == 0) s_red[warp][h] = wsum[h];
+
+  // 3. weighted sums of the partial outputs
+  constexpr int F = G * D / 4;          // float4 columns of one split's G x D block
+  constexpr int KPL = (F + 31) / 32;    // per lane
+  float4 acc[KPL];
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int sp = warp; sp < S; sp += kWarps) {
+    const float4* src = reinterpret_cast<const float4*>(a.o_parts + (row0 + sp * stride) * D);
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) {
+      const int f = lane + 32 * k;
+      if (F % 32 == 0 || f < F) {
+        const float wv = wts[sp * G + f / (D / 4)];
+        const float4 x = __ldcg(src + f);
+        acc[k].x += wv * x.x;
+        acc[k].y += wv * x.y;
+        acc[k].z += wv * x.z;
+        acc[k].w += wv * x.w;
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < KPL; ++k) {
+    const int f = lane + 32 * k;
+    if (F % 32 == 0 || f < F) red[warp * F + f] = acc[k];
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
+  if (tid < G) {
+    float W = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) W += s_red[w][tid];
+    s_w[tid] = W;
+    if (a.lse) a.lse[row0 + tid] = W > 0.f ? s_m[tid] + logf(W) : -INFINITY;
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
+  for (int f = tid; f < F; f += kWarps * 32) {
+    float4 x = red[f];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+      const float4 y = red[w * F + f];
+      x.x += y.x;
+      x.y += y.y;
+      x.z += y.z;
+      x.w += y.w;
+    }
+    const float W = s_w[f / (D / 4)];
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    uint2 packed;
+    packed.x = pack_bf16x2(x.x * inv, x.y * inv);
+    packed.y = pack_bf16x2(x.z * inv, x.w * inv);
+    *reinterpret_cast<uint2*>(a.o + row0 * D + 4 * f) = packed;  // G heads are contiguous
+  }
+}
 
 template <int D, int G>
 __global__ void __launch_bounds__((kWarps + 1) * 32) decode_partials_kernel(
@@ -109,6 +268,11 @@ __global__ void __launch_bounds__((kWarps + 1) * 32) decode_partials_kernel(
 
   if (warp == kWarps) {
     // ---------------- producer warp: the cache append, then TMA loads ----------------
+    // With the fused merge the previous decode step is a kernel of this same kind,
+    // which may still be appending its own row: the cache split waits for it to
+    // finish before it writes or reads any cache row. (Context splits read only
+    // the context, written long before.)
+    if (is_cache && a.counters) pdl_wait();
     if (is_cache && lane < D / 8) {
       // Cache row of (this sequence, row r): contiguous [b, cap, Hkv, D], or row
       // r % P of page table[b][r / P] in the pool [num_pages, P, Hkv, D]. A page id
@@ -319,6 +483,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32) decode_partials_kernel(
             lsum > 0.f ? (M * sl2 + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
       }
     }
+    if (a.counters) merge_if_last<D, G>(a, bb, kvh, base);
   }
 }
 
@@ -342,7 +507,8 @@ cudaError_t launch_decode_t(const Shape& s, const SplitPlan& p, const DecodeArgs
          encode_tma_bf16_4d(&m[3], a.v_cache, D, s.hkv, cache_rows, a.cap, s.b, 64, 1, kTile, true);
   }
   if (!ok) return cudaErrorInvalidValue;
-  const size_t smem = 2 * kStages * (D / 64) * kTile * 128 + 2 * kStages * sizeof(uint64_t) + 1024;
+  if (a.counters && fused_merge_bytes(p.n_splits, G, D) > ring_bytes(D)) return cudaErrorInvalidValue;
+  const size_t smem = ring_bytes(D) + 2 * kStages * sizeof(uint64_t) + 1024;
   auto kern = decode_partials_kernel<D, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -356,11 +522,19 @@ cudaError_t launch_decode_t(const Shape& s, const SplitPlan& p, const DecodeArgs
 
 }  // namespace
 
+bool decode_fused_fits(const Shape& s, const SplitPlan& p) {
+  return fused_merge_bytes(p.n_splits, s.group(), s.d) <= ring_bytes(s.d);
+}
+
 cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const void* q,
                                    const void* k_new, const void* v_new, const void* kc,
                                    const void* vc, const CacheRef& c, int64_t cache_len,
-                                   float* o_parts, float* lse_parts, cudaStream_t st) {
+                                   float* o_parts, float* lse_parts, const FusedMerge* fm,
+                                   cudaStream_t st) {
   DecodeArgs a;
+  a.o = fm ? static_cast<__nv_bfloat16*>(fm->o) : nullptr;
+  a.lse = fm ? fm->lse : nullptr;
+  a.counters = fm ? fm->counters : nullptr;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k_new = static_cast<const __nv_bfloat16*>(k_new);
   a.v_new = static_cast<const __nv_bfloat16*>(v_new);

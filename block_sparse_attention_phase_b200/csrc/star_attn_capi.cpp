@@ -117,10 +117,15 @@ star_status_t run_decode(const Shape& s, const void* q, const void* k, const voi
   float* o_parts = static_cast<float*>(workspace);
   float* lse_parts = lse_parts_of(workspace, s, plan, 1);
   cudaError_t e = launch_decode_partials(s, plan, q, k, v, k_ctx, v_ctx, c, cache_len, o_parts,
-                                         lse_parts, cs);
+                                         lse_parts, nullptr, cs);
   if (e != cudaSuccess) return STAR_ERR_CUDA;
   e = launch_merge(o_parts, lse_parts, plan.n_splits, s.b, 1, s.hq, s.d, o, lse, cs);
   return e == cudaSuccess ? STAR_OK : STAR_ERR_CUDA;
+}
+
+// Fused decode workspace = [o_parts][lse_parts][counters: b * Hkv uint32].
+size_t fused_decode_bytes(const Shape& s) {
+  return partial_bytes(s, decode_plan(s), 1) + align256(static_cast<size_t>(s.b) * s.hkv * 4);
 }
 
 std::atomic<uint64_t> g_launches{0};
@@ -178,6 +183,7 @@ STAR_ATTN_API size_t star_attn_workspace_bytes(const star_attn_shape_t* shape, i
       if (rows < 1) return 0;
       return star::partial_bytes(s, star::query_plan(s, rows), rows);
     case STAR_PHASE2_DECODE: return star::partial_bytes(s, star::decode_plan(s), 1);
+    case STAR_PHASE2_DECODE_FUSED: return star::fused_decode_bytes(s);
     default: return 0;
   }
 }
@@ -242,6 +248,39 @@ STAR_ATTN_API star_status_t star_attn_phase2_decode(
   c.cap = cache_capacity;
   return star::run_decode(s, q, k, v, k_ctx, v_ctx, c, cache_len, o, lse, workspace,
                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+STAR_ATTN_API star_status_t star_attn_phase2_decode_fused(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
+    const void* k_ctx, const void* v_ctx, void* k_cache, void* v_cache, int64_t cache_len,
+    int64_t cache_capacity, void* o, float* lse, void* workspace, size_t workspace_bytes,
+    star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (cache_len < 0 || cache_capacity < 1) return STAR_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, k_ctx, v_ctx, k_cache, v_cache, o};
+  for (const void* p : ptrs)
+    if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned4(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
+  if (cache_len + 1 > cache_capacity) return STAR_ERR_CACHE_FULL;
+  if (!workspace || workspace_bytes < star::fused_decode_bytes(s)) return STAR_ERR_WORKSPACE;
+  const star::SplitPlan plan = star::decode_plan(s);
+  star::CacheRef c;
+  c.k = k_cache;
+  c.v = v_cache;
+  c.cap = cache_capacity;
+  if (!star::decode_fused_fits(s, plan))  // very many splits: partials + merge kernel
+    return star::run_decode(s, q, k, v, k_ctx, v_ctx, c, cache_len, o, lse, workspace,
+                            reinterpret_cast<cudaStream_t>(stream));
+  const size_t parts = star::partial_bytes(s, plan, 1);
+  star::FusedMerge fm;
+  fm.o = o;
+  fm.lse = lse;
+  fm.counters = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + parts);
+  return star::cuda_status(star::launch_decode_partials(
+      s, plan, q, k, v, k_ctx, v_ctx, c, cache_len, static_cast<float*>(workspace),
+      star::lse_parts_of(workspace, s, plan, 1), &fm, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 STAR_ATTN_API star_status_t star_attn_phase2_query_paged(

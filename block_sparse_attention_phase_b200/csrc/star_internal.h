@@ -93,10 +93,21 @@ cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int32_t n
 // the rest of the page holding row rows-1.
 cudaError_t launch_cache_write(const Shape& s, const void* k, const void* v, int64_t rows,
                                const CacheRef& c, cudaStream_t st);
+// Outputs of a decode step whose partial kernel also merges (the last CTA of each
+// (sequence, kv-head) combines the splits); counters [b * Hkv] must be zero before
+// the launch and are zero again after it.
+struct FusedMerge {
+  void* o;
+  float* lse;
+  uint32_t* counters;
+};
 cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const void* q,
                                    const void* k_new, const void* v_new, const void* kc,
                                    const void* vc, const CacheRef& c, int64_t cache_len,
-                                   float* o_parts, float* lse_parts, cudaStream_t st);
+                                   float* o_parts, float* lse_parts, const FusedMerge* fm,
+                                   cudaStream_t st);
+// Whether the fused merge's weights and sums fit in the decode kernel's shared memory.
+bool decode_fused_fits(const Shape& s, const SplitPlan& p);
 cudaError_t launch_phase1_sm100(const Shape& s, const void* q, const void* k, const void* v,
                                 void* o, float* lse, cudaStream_t st);
 // Phase-2 query tokens after their KV is in the cache: partials + merge into o/lse.

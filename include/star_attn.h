@@ -74,13 +74,16 @@ typedef struct {
 } star_attn_shape_t;
 
 /* Phase selectors for star_attn_workspace_bytes(). */
-enum { STAR_PHASE1 = 1, STAR_PHASE2_QUERY = 2, STAR_PHASE2_DECODE = 3 };
+enum { STAR_PHASE1 = 1, STAR_PHASE2_QUERY = 2, STAR_PHASE2_DECODE = 3,
+       STAR_PHASE2_DECODE_FUSED = 4 };
 
 /*
  * Workspace (device scratch) a call needs, in bytes; 0 if none.
- * phase: STAR_PHASE1, STAR_PHASE2_QUERY (rows = query_len) or STAR_PHASE2_DECODE
- * (rows ignored). The workspace holds the per-split fp32 partial outputs and
- * LSEs of Phase 2 before they are merged. Returns 0 for an invalid shape.
+ * phase: STAR_PHASE1, STAR_PHASE2_QUERY (rows = query_len), STAR_PHASE2_DECODE or
+ * STAR_PHASE2_DECODE_FUSED (rows ignored). The workspace holds the per-split fp32
+ * partial outputs and LSEs of Phase 2 before they are merged (and, for the fused
+ * decode, one 32-bit counter per (sequence, kv-head)). Returns 0 for an invalid
+ * shape.
  */
 STAR_ATTN_API size_t star_attn_workspace_bytes(const star_attn_shape_t* shape, int32_t phase,
                                                int64_t rows);
@@ -139,6 +142,30 @@ STAR_ATTN_API star_status_t star_attn_phase2_query(
  * Errors: STAR_ERR_CACHE_FULL if cache_len + 1 > cache_capacity.
  */
 STAR_ATTN_API star_status_t star_attn_phase2_decode(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
+    const void* k_ctx, const void* v_ctx, void* k_cache, void* v_cache, int64_t cache_len,
+    int64_t cache_capacity, void* o, float* lse, void* workspace, size_t workspace_bytes,
+    star_stream_t stream);
+
+/*
+ * star_attn_phase2_decode() in ONE kernel launch: the split-KV partial kernel also
+ * does the exact merge (hotaipapers.com page, Phase 2 paragraph: the query host
+ * aggregates one vector and one scalar per block). Every CTA stores its partial
+ * and counts itself on a per-(sequence, kv-head) counter; the CTA that completes
+ * the count combines all splits of its GQA group and resets the counter.
+ * Same arguments, results and errors as star_attn_phase2_decode(), except:
+ *   workspace: at least star_attn_workspace_bytes(shape, STAR_PHASE2_DECODE_FUSED, 1)
+ *     bytes, ALL ZERO before the first call that uses it (e.g. cudaMemsetAsync once
+ *     after allocation). Each call leaves its counter words zero again, so steps
+ *     can reuse the workspace without clearing it; a workspace that another call
+ *     (query pass, unfused decode) has written must be zeroed again first.
+ *   The result equals star_attn_phase2_decode()'s to fp32 rounding of the merge
+ *     (summation order differs); it is deterministic.
+ *   Shapes with so many splits that the merge's weights do not fit in the kernel's
+ *     shared memory (thousands of context blocks) run as partials + merge kernel,
+ *     with the same results and without touching the counters.
+ */
+STAR_ATTN_API star_status_t star_attn_phase2_decode_fused(
     const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
     const void* k_ctx, const void* v_ctx, void* k_cache, void* v_cache, int64_t cache_len,
     int64_t cache_capacity, void* o, float* lse, void* workspace, size_t workspace_bytes,

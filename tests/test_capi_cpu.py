@@ -137,3 +137,19 @@ def test_paged_entry_points_reject_bad_pools():
     assert qry(200, 128, 4, T, 1) == 4        # 200 rows need two pages
     assert qry(200, 256, 4, T, 1, 0) == 3     # fits one page, but no workspace
     assert qry(0, 128, 4, T, 2) == 1
+
+
+def test_fused_decode_workspace_and_validation():
+    L = sa.lib()
+    s = sa.make_shape(2, 32, 8, 128, 32768, 4096)
+    split = sa.workspace_bytes(s, sa.STAR_PHASE2_DECODE)
+    fused = sa.workspace_bytes(s, sa.STAR_PHASE2_DECODE_FUSED)
+    assert fused == split + 256  # one uint32 counter per (sequence, kv-head), 256-B aligned
+    F = ctypes.c_void_p(FAKE)
+    args = [F, F, F, F, F, F, F]
+    assert L.star_attn_phase2_decode_fused(ctypes.byref(s), *args, 3, 8, F, None, F, split,
+                                           None) == 3  # room for partials but not counters
+    assert L.star_attn_phase2_decode_fused(ctypes.byref(s), *args, 8, 8, F, None, F, fused,
+                                           None) == 4  # cache full
+    assert L.star_attn_phase2_decode_fused(ctypes.byref(s), *args, -1, 8, F, None, F, fused,
+                                           None) == 1

@@ -184,11 +184,16 @@ def _phase2_sampled(w, x, heads, steps):
     vc = torch.zeros_like(kc)
     oq, lql = m.phase2_query(x["q_qry"], x["k_qry"], x["v_qry"], x["k_ctx"], x["v_ctx"], kc, vc,
                              w.block_size)
-    outs = {}
+    kc2, vc2 = kc.clone(), vc.clone()
+    ws = m.fused_decode_workspace(b, w.num_q_heads, hkv, d, w.ctx_len, w.block_size, "cuda")
+    outs, outs_fused = {}, {}
     for t in range(max(steps) + 1):
-        outs[t] = m.phase2_decode(x["q_dec"][t], x["k_dec"][t], x["v_dec"][t], x["k_ctx"],
-                                  x["v_ctx"], kc, vc, lq + t, w.block_size)
+        args = (x["q_dec"][t], x["k_dec"][t], x["v_dec"][t], x["k_ctx"], x["v_ctx"])
+        outs[t] = m.phase2_decode(*args, kc, vc, lq + t, w.block_size)
+        outs_fused[t] = m.phase2_decode_fused(*args, kc2, vc2, lq + t, w.block_size,
+                                              workspace=ws)
     torch.cuda.synchronize()
+    assert torch.equal(kc, kc2) and torch.equal(vc, vc2)
     for bb in range(b):
         for h in heads:
             g = oracle.kv_head_of(h, w.num_q_heads, hkv)
@@ -207,9 +212,10 @@ def _phase2_sampled(w, x, heads, steps):
                     x["q_dec"][t, bb, 0, h].float().cpu().numpy(), kctx, vctx,
                     np.concatenate([kq, kd[:t]]), np.concatenate([vq, vd[:t]]), kd[t], vd[t],
                     w.softmax_scale)
-                od, ld = outs[t]
-                check_rows(to_np(od[bb, 0, h])[None], ro[None], to_np(ld[bb, h, 0:1]),
-                           np.array([rl]), f"{w.name} decode t={t} b={bb} h={h}")
+                for kind, res in (("split", outs), ("fused", outs_fused)):
+                    od, ld = res[t]
+                    check_rows(to_np(od[bb, 0, h])[None], ro[None], to_np(ld[bb, h, 0:1]),
+                               np.array([rl]), f"{w.name} {kind} decode t={t} b={bb} h={h}")
 
 
 FULL = ["llama8b-32k", "llama8b-128k", "70b-128k", "1m"]
