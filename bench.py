@@ -220,14 +220,21 @@ class Step:
                 ev[2].elapsed_time(ev[3]) / self.w.decode_steps)
 
 
+COLD_SPIN_CYCLES = 400_000  # ~0.2 ms of GPU time at 1.9 GHz
+
+
 def decode_cold_ms(step: Step, reps: int = 1):
-    """Each decode call timed alone after an L2 flush (events on the launching stream)."""
+    """Each decode call timed alone after an L2 flush (events on the launching stream).
+    A short GPU spin after the flush keeps the GPU busy while the host issues the
+    call, so the time is the step's own from a cold L2 (launch latency included),
+    not the host's Python overhead."""
     w, x, layer = step.w, step.x, step.layer
     layer.prefill(x["q_ctx"], x["k_ctx"], x["v_ctx"], o=step.o_ctx, lse=step.lse_ctx)
     layer.query(x["q_qry"], x["k_qry"], x["v_qry"], o=step.o_q, lse=step.lse_q)
     times = []
     for t in range(w.decode_steps):
         step.flush.fill_(2)
+        torch.cuda._sleep(COLD_SPIN_CYCLES)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record()

@@ -88,10 +88,13 @@ def main(argv=None) -> int:
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true", help="print registers / spills per kernel")
+    ap.add_argument("-D", dest="defines", action="append", default=[],
+                    help="NAME=VALUE passed to the compiler (tuning constants)")
     args = ap.parse_args(argv)
     extra = ["-Xptxas", "-v"] if args.ptxas_info else []
-    path = build(force=args.force or args.ptxas_info, verbose=args.verbose or args.ptxas_info,
-                 extra=extra)
+    extra += [f"-D{d}" for d in args.defines]
+    path = build(force=args.force or args.ptxas_info or bool(args.defines),
+                 verbose=args.verbose or args.ptxas_info, extra=extra)
     print(path)
     return 0
 

@@ -52,12 +52,17 @@ struct DecodeArgs {
 
 constexpr int kTile = 64;      // tokens per TMA tile
 constexpr int kWarps = 4;      // consumer warps (16 tokens of each tile apiece)
-constexpr int kStages = 3;
+// Ring depth: 3 stages (96 KB at d = 128, two CTAs per SM) keep enough bytes in
+// flight for long splits. For short splits the whole step is only a few tiles
+// per CTA and the gaps between consecutive steps dominate, so 2 stages are used:
+// three CTAs then fit on an SM, and the next step's CTAs (launched early through
+// programmatic launch) start streaming in the free slot while this step drains.
+constexpr int64_t kShortChunk = 2048;  // keys per split at or below which 2 stages are used
 constexpr float kRescaleLog2 = 8.f;
 
-// The fused merge reuses the KV ring: S x G split weights, then one fp32 sum of
-// the G x D outputs per consumer warp.
-STAR_HD constexpr size_t ring_bytes(int d) { return size_t{2} * kStages * (d / 64) * kTile * 128; }
+STAR_HD constexpr size_t ring_bytes(int d, int stages) {
+  return size_t{2} * stages * (d / 64) * kTile * 128;
+}
 STAR_HD constexpr size_t fused_weights_bytes(int64_t n_splits, int g) {
   return (static_cast<size_t>(n_splits) * g * 4 + 15) & ~size_t(15);
 }
@@ -210,8 +215,8 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, int bb, int k
   }
 }
 
-template <int D, int G>
-__global__ void __launch_bounds__((kWarps + 1) * 32) decode_partials_kernel(
+template <int D, int G, int kStages>
+__global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decode_partials_kernel(
     const __grid_constant__ CUtensorMap mk_ctx, const __grid_constant__ CUtensorMap mv_ctx,
     const __grid_constant__ CUtensorMap mk_cache, const __grid_constant__ CUtensorMap mv_cache,
     const DecodeArgs a) {
@@ -487,7 +492,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32) decode_partials_kernel(
   }
 }
 
-template <int D, int G>
+template <int D, int G, int kStages>
 cudaError_t launch_decode_t(const Shape& s, const SplitPlan& p, const DecodeArgs& a,
                             const void* kc, const void* vc, int32_t num_pages, cudaStream_t st) {
   alignas(64) CUtensorMap m[4];
@@ -507,9 +512,10 @@ cudaError_t launch_decode_t(const Shape& s, const SplitPlan& p, const DecodeArgs
          encode_tma_bf16_4d(&m[3], a.v_cache, D, s.hkv, cache_rows, a.cap, s.b, 64, 1, kTile, true);
   }
   if (!ok) return cudaErrorInvalidValue;
-  if (a.counters && fused_merge_bytes(p.n_splits, G, D) > ring_bytes(D)) return cudaErrorInvalidValue;
-  const size_t smem = ring_bytes(D) + 2 * kStages * sizeof(uint64_t) + 1024;
-  auto kern = decode_partials_kernel<D, G>;
+  if (a.counters && fused_merge_bytes(p.n_splits, G, D) > ring_bytes(D, kStages))
+    return cudaErrorInvalidValue;
+  const size_t smem = ring_bytes(D, kStages) + 2 * kStages * sizeof(uint64_t) + 1024;
+  auto kern = decode_partials_kernel<D, G, kStages>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -520,10 +526,12 @@ cudaError_t launch_decode_t(const Shape& s, const SplitPlan& p, const DecodeArgs
   return cudaGetLastError();
 }
 
+int decode_stages(const SplitPlan& p) { return p.chunk <= kShortChunk ? 2 : 3; }
+
 }  // namespace
 
 bool decode_fused_fits(const Shape& s, const SplitPlan& p) {
-  return fused_merge_bytes(p.n_splits, s.group(), s.d) <= ring_bytes(s.d);
+  return fused_merge_bytes(p.n_splits, s.group(), s.d) <= ring_bytes(s.d, decode_stages(p));
 }
 
 cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const void* q,
@@ -559,8 +567,11 @@ cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const voi
   a.lse_parts = lse_parts;
   a.status = device_status_word();
   const int G = s.group();
-#define STAR_DECODE_CASE(DD, GG) \
-  if (s.d == DD && G == GG) return launch_decode_t<DD, GG>(s, p, a, kc, vc, c.num_pages, st);
+  const bool two = decode_stages(p) == 2;
+#define STAR_DECODE_CASE(DD, GG)                                                              \
+  if (s.d == DD && G == GG)                                                                   \
+    return two ? launch_decode_t<DD, GG, 2>(s, p, a, kc, vc, c.num_pages, st)                 \
+               : launch_decode_t<DD, GG, 3>(s, p, a, kc, vc, c.num_pages, st);
   STAR_DECODE_CASE(128, 1) STAR_DECODE_CASE(128, 2) STAR_DECODE_CASE(128, 4)
   STAR_DECODE_CASE(128, 8) STAR_DECODE_CASE(64, 1) STAR_DECODE_CASE(64, 2)
   STAR_DECODE_CASE(64, 4) STAR_DECODE_CASE(64, 8)

@@ -14,7 +14,10 @@ namespace star {
 namespace {
 
 constexpr int kSMs = 148;              // B200
-constexpr int kDecodeCtasPerSM = 2;
+#ifndef STAR_DECODE_CTAS_PER_SM
+#define STAR_DECODE_CTAS_PER_SM 2
+#endif
+constexpr int kDecodeCtasPerSM = STAR_DECODE_CTAS_PER_SM;
 constexpr int64_t kMinChunk = 64;      // one TMA tile of keys
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
