@@ -32,7 +32,8 @@ STATUS_NAMES = {0: "STAR_OK", 1: "STAR_ERR_INVALID_ARG", 2: "STAR_ERR_UNSUPPORTE
                 6: "STAR_ERR_TIMEOUT"}
 
 # Every symbol the header declares; tests check that the library exports them all.
-EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase2_query",
+EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase1_varlen",
+            "star_attn_phase2_query",
             "star_attn_phase2_decode", "star_attn_phase2_decode_fused",
             "star_attn_phase2_query_paged",
             "star_attn_phase2_decode_paged", "star_attn_phase2_decode_noalloc",
@@ -72,6 +73,7 @@ def lib() -> ctypes.CDLL:
     sig = {
         "star_attn_workspace_bytes": (SZ, [SP, I32, I64]),
         "star_attn_phase1": (I32, [SP, P, P, P, P, P, P]),
+        "star_attn_phase1_varlen": (I32, [SP, ctypes.POINTER(I64), P, P, P, P, P, P]),
         "star_attn_phase2_query": (I32, [SP, P, P, P, I64, P, P, P, P, I64, P, P, P, SZ, P]),
         "star_attn_phase2_decode": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P, SZ, P]),
         "star_attn_phase2_decode_fused": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P, SZ,
@@ -150,6 +152,30 @@ def phase1(q, k, v, block_size: int, scale: Optional[float] = None, o=None, lse=
         lse = torch.empty((b, hq, L), dtype=torch.float32, device=q.device)
     _check(lib().star_attn_phase1(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                   _ptr(lse), _stream()), "star_attn_phase1")
+    return o, lse
+
+
+def _cu_array(cu_seqlens):
+    vals = [int(x) for x in cu_seqlens]
+    return (ctypes.c_int64 * len(vals))(*vals), vals
+
+
+def phase1_varlen(q, k, v, cu_seqlens, block_size: int, scale: Optional[float] = None,
+                  o=None, lse=None, want_lse: bool = True):
+    """Phase 1 over sequences packed along tokens: q [total, Hq, d], k/v [total, Hkv, d],
+    cu_seqlens = host offsets [n + 1] (list/array/CPU tensor). Returns (o [total, Hq, d],
+    lse [Hq, total]); each sequence is computed as if alone."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bf16(t, n, 3)
+    cu, vals = _cu_array(cu_seqlens)
+    total, hq, d = q.shape
+    shape = make_shape(len(vals) - 1, hq, k.shape[1], d, total, block_size, scale)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((hq, total), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_phase1_varlen(ctypes.byref(shape), cu, _ptr(q), _ptr(k), _ptr(v),
+                                         _ptr(o), _ptr(lse), _stream()), "star_attn_phase1_varlen")
     return o, lse
 
 

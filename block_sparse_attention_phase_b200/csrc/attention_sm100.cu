@@ -107,6 +107,8 @@ struct Item {
   // Phase 1
   int h[2], rows_valid[2], n_anchor;
   int64_t bstart, t0[2];
+  int64_t L, B;       // this sequence's length and block size
+  int64_t tok_base;   // first token of this sequence in packed (varlen) tensors, else 0
   // query
   int split, tok0[2];
   bool cache;
@@ -114,52 +116,71 @@ struct Item {
 };
 
 template <Mode M>
-__device__ __forceinline__ Item decode_item(const AttnArgs& a) {
+__device__ __forceinline__ Item decode_item(const AttnArgs& a, const VarSeqs& vs) {
   Item it{};
   int64_t r = blockIdx.x;
+  it.L = a.L;
+  it.B = a.B;
   if constexpr (M == Mode::kPhase1) {
+    int n_blocks = a.n_blocks, mt = a.mt, n_anchor = a.n_anchor;
+    if (vs.n > 0) {
+      // Varlen batch: the sequence whose work items hold this one (the last with
+      // item0 <= r; empty sequences own no item), then its own block plan.
+      int lo = 0, hi = vs.n;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (vs.item0[mid] <= r) lo = mid; else hi = mid;
+      }
+      r -= vs.item0[lo];
+      it.tok_base = vs.start[lo];
+      it.L = vs.start[lo + 1] - vs.start[lo];
+      it.B = min(a.B, it.L);
+      n_blocks = static_cast<int>((it.L + it.B - 1) / it.B);
+      mt = static_cast<int>((it.B + 127) / 128);
+      n_anchor = mt;
+    }
     int i, m0, m1;
     if (a.G >= 2) {
       const int npair = a.G / 2;
       const int hp = static_cast<int>(r % npair);
       r /= npair;
-      const int mp = static_cast<int>(r % a.mt);
-      r /= a.mt;
-      const int ip = static_cast<int>(r % a.n_blocks);
-      r /= a.n_blocks;
+      const int mp = static_cast<int>(r % mt);
+      r /= mt;
+      const int ip = static_cast<int>(r % n_blocks);
+      r /= n_blocks;
       it.kvh = static_cast<int>(r % a.hkv);
       it.bb = static_cast<int>(r / a.hkv);
-      i = (ip + 1) % a.n_blocks;  // blocks 1..n-1 first, b_0 (cheapest) last
-      m0 = m1 = a.mt - 1 - mp;    // longest q-tiles first
+      i = (ip + 1) % n_blocks;  // blocks 1..n-1 first, b_0 (cheapest) last
+      m0 = m1 = mt - 1 - mp;    // longest q-tiles first
       it.h[0] = it.kvh * a.G + 2 * hp;
       it.h[1] = it.h[0] + 1;
     } else {
-      const int mt2 = (a.mt + 1) / 2;
+      const int mt2 = (mt + 1) / 2;
       const int mp = static_cast<int>(r % mt2);
       r /= mt2;
-      const int ip = static_cast<int>(r % a.n_blocks);
-      r /= a.n_blocks;
+      const int ip = static_cast<int>(r % n_blocks);
+      r /= n_blocks;
       it.kvh = static_cast<int>(r % a.hkv);
       it.bb = static_cast<int>(r / a.hkv);
-      i = (ip + 1) % a.n_blocks;
+      i = (ip + 1) % n_blocks;
       m0 = 2 * (mt2 - 1 - mp);
       m1 = m0 + 1;
       it.h[0] = it.h[1] = it.kvh;
     }
-    it.bstart = static_cast<int64_t>(i) * a.B;
-    const int64_t bend = min(a.L, it.bstart + a.B);
+    it.bstart = static_cast<int64_t>(i) * it.B;
+    const int64_t bend = min(it.L, it.bstart + it.B);
     it.t0[0] = it.bstart + 128 * static_cast<int64_t>(m0);
     it.t0[1] = it.bstart + 128 * static_cast<int64_t>(m1);
 #pragma unroll
     for (int q = 0; q < 2; ++q)
       it.rows_valid[q] = it.t0[q] >= bend ? 0 : static_cast<int>(bend - it.t0[q] < 128 ? bend - it.t0[q] : 128);
     const int m_last = it.rows_valid[1] > 0 ? m1 : m0;
-    it.n_anchor = i > 0 ? a.n_anchor : 0;
+    it.n_anchor = i > 0 ? n_anchor : 0;
     it.n_tiles = it.rows_valid[0] > 0 ? it.n_anchor + m_last + 1 : 0;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       it.qc1[q] = it.h[q];
-      it.qc2[q] = static_cast<int32_t>(it.t0[q]);
+      it.qc2[q] = static_cast<int32_t>(it.tok_base + it.t0[q]);
     }
   } else {
     const int npair = (a.n_qt + 1) / 2;
@@ -227,7 +248,7 @@ __device__ __forceinline__ int visible_prefix(const Item& it, const AttnArgs& a,
   int64_t lim;
   if constexpr (M == Mode::kPhase1) {
     if (j < it.n_anchor) {
-      lim = a.B - 128 * static_cast<int64_t>(j);  // the anchor ends at B
+      lim = it.B - 128 * static_cast<int64_t>(j);  // the anchor ends at B
     } else {
       const int64_t kv0 = it.bstart + 128 * static_cast<int64_t>(j - it.n_anchor);
       lim = tok - kv0 + 1;  // causal inside the own block
@@ -245,7 +266,7 @@ template <int D, Mode M>
 __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
     const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tk2,
-    const __grid_constant__ CUtensorMap tv2, const AttnArgs a) {
+    const __grid_constant__ CUtensorMap tv2, const AttnArgs a, const __grid_constant__ VarSeqs vs) {
   constexpr int CH = D / 64;
   constexpr uint32_t kTileBytes = CH * kChunkBytes;
 
@@ -257,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
   uint8_t* sv = sk + 2 * kTileBytes;  // [2][kTileBytes]
   Bars* bars = reinterpret_cast<Bars*>(sv + 2 * kTileBytes);
 
-  const Item it = decode_item<M>(a);
+  const Item it = decode_item<M>(a, vs);
   if (it.n_tiles == 0) {
     if constexpr (M == Mode::kQuery) {
       // A chunk past the end of a short last block: an empty partial.
@@ -332,7 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         const uint32_t ph = (j >> 1) & 1;
         int32_t kv0;
         if constexpr (M == Mode::kPhase1) {
-          kv0 = j < it.n_anchor ? j * 128 : static_cast<int32_t>(it.bstart + 128 * (j - it.n_anchor));
+          kv0 = static_cast<int32_t>(it.tok_base) +
+                (j < it.n_anchor ? j * 128 : static_cast<int32_t>(it.bstart + 128 * (j - it.n_anchor)));
         } else {
           kv0 = static_cast<int32_t>(it.k0 + 128 * j);
         }
@@ -555,7 +577,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       if constexpr (M == Mode::kPhase1) {
         const int64_t t = row_tok;
         const bool valid = row < rows_valid;
-        __nv_bfloat16* dst = a.o + ((static_cast<int64_t>(it.bb) * a.L + t) * a.hq + head) * D;
+        // uniform: row bb * L + t of [b, L, Hq, d]; varlen: row tok_base + t of [total, Hq, d]
+        __nv_bfloat16* dst = a.o + ((static_cast<int64_t>(it.bb) * a.L + it.tok_base + t) * a.hq + head) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ob[32];
@@ -573,7 +596,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
           }
         }
         if (a.lse && valid)
-          a.lse[(static_cast<int64_t>(it.bb) * a.hq + head) * a.L + t] = lse2 * 0.69314718055994531f;
+          a.lse[(static_cast<int64_t>(it.bb) * a.hq + head) * a.L + it.tok_base + t] =
+              lse2 * 0.69314718055994531f;
       } else {
         const int tok = static_cast<int>(row_tok);
         const int hq = head;
@@ -620,7 +644,8 @@ AttnArgs base_args(const Shape& s) {
 }
 
 template <int D, Mode M>
-cudaError_t launch(const AttnArgs& a, const CUtensorMap (&m)[5], int64_t items, cudaStream_t st) {
+cudaError_t launch(const AttnArgs& a, const CUtensorMap (&m)[5], int64_t items, const VarSeqs& vs,
+                   cudaStream_t st) {
   constexpr uint32_t kTileBytes = (D / 64) * kChunkBytes;
   // 6 tiles (2 Q, 2 K, 2 V) + barriers + alignment slack; at least 120 KB so that
   // only one CTA (and one 512-column TMEM allocation) lives on an SM.
@@ -632,7 +657,7 @@ cudaError_t launch(const AttnArgs& a, const CUtensorMap (&m)[5], int64_t items, 
   if (e != cudaSuccess) return e;
   if (items <= 0) return cudaSuccess;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
-  kern<<<static_cast<unsigned>(items), kThreads, smem, st>>>(m[0], m[1], m[2], m[3], m[4], a);
+  kern<<<static_cast<unsigned>(items), kThreads, smem, st>>>(m[0], m[1], m[2], m[3], m[4], a, vs);
   count_launch();
   return cudaGetLastError();
 }
@@ -655,7 +680,48 @@ cudaError_t launch_phase1_t(const Shape& s, const void* q, const void* k, const 
   a.lse = lse;
   const int64_t pairs_per_block = a.G >= 2 ? static_cast<int64_t>(a.mt) * (a.G / 2) : (a.mt + 1) / 2;
   const int64_t items = static_cast<int64_t>(s.b) * s.hkv * a.n_blocks * pairs_per_block;
-  return launch<D, Mode::kPhase1>(a, m, items, st);
+  VarSeqs vs;
+  vs.n = 0;
+  return launch<D, Mode::kPhase1>(a, m, items, vs, st);
+}
+
+// Work items of one Phase-1 sequence of length L (blocks x q-tile pairs x kv-heads).
+int64_t phase1_items(int64_t L, int64_t B, int G, int hkv) {
+  if (L <= 0) return 0;
+  const int64_t Bi = B < L ? B : L;
+  const int64_t n_blocks = (L + Bi - 1) / Bi;
+  const int64_t mt = (Bi + 127) / 128;
+  const int64_t pairs = G >= 2 ? mt * (G / 2) : (mt + 1) / 2;
+  return n_blocks * pairs * hkv;
+}
+
+template <int D>
+cudaError_t launch_phase1_varlen_t(const Shape& s, const int64_t* cu, const void* q, const void* k,
+                                   const void* v, void* o, float* lse, cudaStream_t st) {
+  const int64_t total = cu[s.b];
+  alignas(64) CUtensorMap m[5];
+  if (!encode_tma_bf16_4d(&m[0], q, D, s.hq, total, total, 1, 64, 1, 128, true) ||
+      !encode_tma_bf16_4d(&m[1], k, D, s.hkv, total, total, 1, 64, 1, 128, true) ||
+      !encode_tma_bf16_4d(&m[2], v, D, s.hkv, total, total, 1, 64, 1, 128, true))
+    return cudaErrorInvalidValue;
+  m[3] = m[1];
+  m[4] = m[2];
+  AttnArgs a = base_args(s);
+  a.L = total;  // row stride of the packed outputs (o rows, lse per head)
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  VarSeqs vs;
+  vs.n = s.b;
+  int64_t items = 0;
+  for (int i = 0; i < s.b; ++i) {
+    vs.item0[i] = static_cast<int32_t>(items);
+    vs.start[i] = static_cast<int32_t>(cu[i]);
+    items += phase1_items(cu[i + 1] - cu[i], s.B, a.G, s.hkv);
+    if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+  }
+  vs.item0[s.b] = static_cast<int32_t>(items);
+  vs.start[s.b] = static_cast<int32_t>(total);
+  return launch<D, Mode::kPhase1>(a, m, items, vs, st);
 }
 
 template <int D>
@@ -693,7 +759,9 @@ cudaError_t launch_query_t(const Shape& s, const SplitPlan& p, const void* q, in
   a.o_parts = o_parts;
   a.lse_parts = lse_parts;
   const int64_t items = static_cast<int64_t>(s.b) * s.hkv * a.n_splits * ((a.n_qt + 1) / 2);
-  return launch<D, Mode::kQuery>(a, m, items, st);
+  VarSeqs vs;
+  vs.n = 0;
+  return launch<D, Mode::kQuery>(a, m, items, vs, st);
 }
 
 }  // namespace
@@ -704,6 +772,13 @@ cudaError_t launch_phase1_sm100(const Shape& s, const void* q, const void* k, co
                                 void* o, float* lse, cudaStream_t st) {
   if (s.d == 128) return launch_phase1_t<128>(s, q, k, v, o, lse, st);
   return launch_phase1_t<64>(s, q, k, v, o, lse, st);
+}
+
+cudaError_t launch_phase1_varlen(const Shape& s, const int64_t* cu_seqlens, const void* q,
+                                 const void* k, const void* v, void* o, float* lse,
+                                 cudaStream_t st) {
+  if (s.d == 128) return launch_phase1_varlen_t<128>(s, cu_seqlens, q, k, v, o, lse, st);
+  return launch_phase1_varlen_t<64>(s, cu_seqlens, q, k, v, o, lse, st);
 }
 
 cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q, int64_t lq,

@@ -205,6 +205,25 @@ STAR_ATTN_API star_status_t star_attn_phase1(const star_attn_shape_t* shape, con
       star::launch_phase1_sm100(s, q, k, v, o, lse, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+STAR_ATTN_API star_status_t star_attn_phase1_varlen(const star_attn_shape_t* shape,
+                                                    const int64_t* cu_seqlens, const void* q,
+                                                    const void* k, const void* v, void* o,
+                                                    float* lse, star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (!cu_seqlens || !q || !k || !v || !o) return STAR_ERR_INVALID_ARG;
+  if (s.b > star::kMaxVarSeqs) return STAR_ERR_UNSUPPORTED;
+  if (cu_seqlens[0] != 0 || cu_seqlens[s.b] != s.L) return STAR_ERR_INVALID_ARG;
+  for (int i = 0; i < s.b; ++i)
+    if (cu_seqlens[i + 1] < cu_seqlens[i]) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned16(q) || !star::aligned16(k) || !star::aligned16(v) || !star::aligned16(o) ||
+      !star::aligned4(lse))
+    return STAR_ERR_INVALID_ARG;
+  return star::cuda_status(star::launch_phase1_varlen(s, cu_seqlens, q, k, v, o, lse,
+                                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 STAR_ATTN_API star_status_t star_attn_phase2_query(
     const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
     int64_t query_len, const void* k_ctx, const void* v_ctx, void* k_cache, void* v_cache,

@@ -76,6 +76,16 @@ struct CacheRef {
   bool paged() const { return page_table != nullptr; }
 };
 
+// A varlen batch as the kernels see it (passed by value as a kernel parameter):
+// sequence i owns work items [item0[i], item0[i+1]) and tokens
+// [start[i], start[i+1]) of the packed tensors. n = 0: a uniform batch.
+constexpr int kMaxVarSeqs = 128;
+struct VarSeqs {
+  int32_t n;
+  int32_t item0[kMaxVarSeqs + 1];
+  int32_t start[kMaxVarSeqs + 1];
+};
+
 // Device status word of the current device (address valid on that device).
 uint32_t* device_status_word();
 
@@ -110,6 +120,11 @@ cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const voi
 bool decode_fused_fits(const Shape& s, const SplitPlan& p);
 cudaError_t launch_phase1_sm100(const Shape& s, const void* q, const void* k, const void* v,
                                 void* o, float* lse, cudaStream_t st);
+// Phase 1 over a varlen batch: s.b sequences packed along tokens, s.L = total tokens,
+// cu_seqlens (host) [s.b + 1]; o [total, Hq, d], lse [Hq, total].
+cudaError_t launch_phase1_varlen(const Shape& s, const int64_t* cu_seqlens, const void* q,
+                                 const void* k, const void* v, void* o, float* lse,
+                                 cudaStream_t st);
 // Phase-2 query tokens after their KV is in the cache: partials + merge into o/lse.
 cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q, int64_t lq,
                               const void* kc, const void* vc, const CacheRef& c, float* o_parts,

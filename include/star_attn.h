@@ -107,6 +107,27 @@ STAR_ATTN_API star_status_t star_attn_phase1(const star_attn_shape_t* shape, con
                                              star_stream_t stream);
 
 /*
+ * Phase 1 over a varlen batch: shape->batch sequences of different lengths,
+ * packed back to back along the token axis; each sequence is its own context
+ * with its own blocks and its own anchor (its first block), exactly as if it
+ * were run alone through star_attn_phase1() with batch 1.
+ *   cu_seqlens: HOST array of batch + 1 int64 offsets, cu_seqlens[0] = 0,
+ *     non-decreasing, cu_seqlens[batch] = shape->ctx_len (the total token count).
+ *     Sequence i is tokens [cu_seqlens[i], cu_seqlens[i+1]); empty sequences are
+ *     allowed. Read during the call only.
+ *   A sequence shorter than block_size is one block (plain causal attention).
+ * q [total, Hq, d]; k, v [total, Hkv, d]; o [total, Hq, d]; lse [Hq, total] or NULL.
+ * Errors: STAR_ERR_UNSUPPORTED for more than 128 sequences; STAR_ERR_INVALID_ARG
+ * for offsets that are not as above.
+ * No counterpart on the pages (serving-side batching of documents of different
+ * lengths; the per-sequence computation is Phase 1's).
+ */
+STAR_ATTN_API star_status_t star_attn_phase1_varlen(const star_attn_shape_t* shape,
+                                                    const int64_t* cu_seqlens, const void* q,
+                                                    const void* k, const void* v, void* o,
+                                                    float* lse, star_stream_t stream);
+
+/*
  * Phase 2, query tokens (abstract: query tokens attend to all prior cached
  * tokens; hotaipapers.com page, Phase 2 paragraph).
  *

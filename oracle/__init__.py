@@ -31,6 +31,7 @@ from .star_oracle import (  # noqa: F401
     lse_merge,
     phase1_head,
     phase1,
+    phase1_varlen,
     phase2_query_head,
     phase2_query_head_blockwise,
     phase2_query,

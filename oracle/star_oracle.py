@@ -169,6 +169,24 @@ def phase1(q, k, v, block_size: int, scale: float = None):
     return o, lse
 
 
+def phase1_varlen(q, k, v, cu_seqlens: Sequence[int], block_size: int, scale: float = None):
+    """Phase 1 over a varlen batch: sequences packed along the token axis,
+    q [total, Hq, d], k, v [total, Hkv, d], sequence i = tokens
+    [cu_seqlens[i], cu_seqlens[i+1]). Each sequence is its own context (its own
+    blocks and anchor), so this is Phase 1 applied to each slice on its own.
+    Returns o [total, Hq, d] and lse [Hq, total] in float64."""
+    total, Hq, d = q.shape
+    o = np.zeros((total, Hq, d), dtype=F64)
+    lse = np.zeros((Hq, total), dtype=F64)
+    for a, e in zip(cu_seqlens[:-1], cu_seqlens[1:]):
+        if e == a:
+            continue
+        oi, li = phase1(q[None, a:e], k[None, a:e], v[None, a:e], block_size, scale)
+        o[a:e] = oi[0]
+        lse[:, a:e] = li[0]
+    return o, lse
+
+
 def phase2_query_head(q, k_ctx, v_ctx, k_qry, v_qry, scale: float):
     """Phase-2 query tokens by the definition: sequence-global attention
     (abstract: query and response tokens attend to all prior cached tokens).

@@ -153,3 +153,21 @@ def test_fused_decode_workspace_and_validation():
                                            None) == 4  # cache full
     assert L.star_attn_phase2_decode_fused(ctypes.byref(s), *args, -1, 8, F, None, F, fused,
                                            None) == 1
+
+
+def test_phase1_varlen_rejects_bad_offsets():
+    L = sa.lib()
+    F = ctypes.c_void_p(FAKE)
+
+    def call(cu, total, batch=None):
+        n = len(cu) - 1 if batch is None else batch
+        s = sa.make_shape(n, 4, 2, 128, total, 64)
+        arr = (ctypes.c_int64 * len(cu))(*cu)
+        return L.star_attn_phase1_varlen(ctypes.byref(s), arr, F, F, F, F, None, None)
+
+    assert call([1, 5, 9], 9) == 1        # does not start at 0
+    assert call([0, 5, 4], 4) == 1        # decreasing
+    assert call([0, 5, 9], 10) == 1       # last offset != ctx_len
+    assert call([0] + list(range(1, 130)), 129) == 2  # 129 sequences: more than 128
+    s = sa.make_shape(2, 4, 2, 128, 9, 64)
+    assert L.star_attn_phase1_varlen(ctypes.byref(s), None, F, F, F, F, None, None) == 1

@@ -267,11 +267,32 @@ def check_decode_matches_query_rows(seed=8):
         np.testing.assert_allclose(lse[:, :, 0], full_lse[:, :, pos], atol=1e-12)
 
 
+def check_phase1_varlen_per_sequence(seed=9):
+    """Varlen Phase 1 = each packed sequence on its own. Every sequence here has at
+    most two blocks, so its Phase 1 is plain causal attention (torch SDPA)."""
+    rng = np.random.default_rng(seed)
+    B, Hq, Hkv, d = 8, 4, 2, 16
+    lens = [5, 0, 16, 11, 1, 8]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(int)
+    total = int(cu[-1])
+    q, k, v = rand(rng, total, Hq, d), rand(rng, total, Hkv, d), rand(rng, total, Hkv, d)
+    scale = 0.3
+    o, lse = oracle.phase1_varlen(q, k, v, list(cu), B, scale)
+    assert o.shape == (total, Hq, d) and lse.shape == (Hq, total)
+    for a, e in zip(cu[:-1], cu[1:]):
+        if e == a:
+            continue
+        ro, rl = sdpa_causal_gqa(q[a:e], k[a:e], v[a:e], scale)
+        np.testing.assert_allclose(o[a:e], ro, atol=1e-12)
+        np.testing.assert_allclose(lse[:, a:e], rl, atol=1e-12)
+
+
 ALL_CHECKS = [check_single_block_is_causal, check_two_blocks_is_full_causal,
               check_phase1_keysets_golden, check_first_and_last_row_of_block,
               check_block_independence, check_gqa_mapping, check_closed_forms,
               check_phase2_query_is_global, check_phase2_keysets_golden,
-              check_merge_split_invariance, check_decode_matches_query_rows]
+              check_merge_split_invariance, check_decode_matches_query_rows,
+              check_phase1_varlen_per_sequence]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda c: c.__name__)
@@ -331,7 +352,14 @@ def _mut_merge_unweighted(o_parts, lse_parts):
     return o, np.log(np.exp(lse_parts).sum(0))
 
 
+def _mut_varlen_one_context(q, k, v, cu_seqlens, block_size, scale=None):
+    # the packed batch treated as one long context (blocks and anchor shared)
+    o, lse = so.phase1(q[None], k[None], v[None], block_size, scale)
+    return o[0], lse[0]
+
+
 MUTANTS = {
+    "varlen_one_context": ("phase1_varlen", _mut_varlen_one_context),
     "anchor_is_previous_block": ("phase1_visible", _mut_anchor_previous),
     "no_anchor": ("phase1_visible", _mut_no_anchor),
     "strict_causal": ("phase1_visible", _mut_strict_causal),
