@@ -35,6 +35,7 @@ STATUS_NAMES = {0: "STAR_OK", 1: "STAR_ERR_INVALID_ARG", 2: "STAR_ERR_UNSUPPORTE
 EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase1_varlen",
             "star_attn_phase2_query",
             "star_attn_phase2_decode", "star_attn_phase2_decode_fused",
+            "star_attn_phase2_decode_varlen", "star_attn_decode_varlen_workspace_bytes",
             "star_attn_phase2_query_paged",
             "star_attn_phase2_decode_paged", "star_attn_phase2_decode_noalloc",
             "star_attn_lse_merge", "star_attn_simple_phase1",
@@ -78,6 +79,10 @@ def lib() -> ctypes.CDLL:
         "star_attn_phase2_decode": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P, SZ, P]),
         "star_attn_phase2_decode_fused": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P, SZ,
                                                  P]),
+        "star_attn_phase2_decode_varlen": (I32, [SP, ctypes.POINTER(I64), ctypes.POINTER(I64),
+                                                  P, P, P, P, P, P, P, I64, P, I32, I32, I32,
+                                                  P, P, P, SZ, P]),
+        "star_attn_decode_varlen_workspace_bytes": (SZ, [SP, ctypes.POINTER(I64)]),
         "star_attn_phase2_query_paged": (I32, [SP, P, P, P, I64, P, P, P, P, I32, I32, P, I32,
                                                 P, P, P, SZ, P]),
         "star_attn_phase2_decode_paged": (I32, [SP, P, P, P, P, P, P, P, I32, I32, P, I32, I64,
@@ -319,6 +324,57 @@ def phase2_decode_fused(q, k, v, k_ctx, v_ctx, k_cache, v_cache, cache_len: int,
         ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_cache),
         _ptr(v_cache), int(cache_len), k_cache.shape[1], _ptr(o), _ptr(lse), _ptr(workspace),
         workspace.numel(), _stream()), "star_attn_phase2_decode_fused")
+    return o, lse
+
+
+def decode_varlen_workspace(batch, num_q_heads, num_kv_heads, head_dim, cu_ctx, block_size,
+                            device, scale: Optional[float] = None) -> torch.Tensor:
+    """A zeroed workspace for phase2_decode_varlen() with these context offsets."""
+    cu, vals = _cu_array(cu_ctx)
+    shape = make_shape(batch, num_q_heads, num_kv_heads, head_dim, vals[-1], block_size, scale)
+    need = int(lib().star_attn_decode_varlen_workspace_bytes(ctypes.byref(shape), cu))
+    if need == 0:
+        raise ValueError("unsupported shape or offsets")
+    return torch.zeros(need, dtype=torch.uint8, device=device)
+
+
+def phase2_decode_varlen(q, k, v, k_ctx, v_ctx, cu_ctx, k_cache, v_cache, cache_lens,
+                         block_size: int, page_table=None, scale: Optional[float] = None,
+                         o=None, lse=None, workspace=None):
+    """One decode step for a batch of sequences at different lengths: q [b, 1, Hq, d],
+    k/v [b, 1, Hkv, d]; packed contexts k_ctx/v_ctx [total, Hkv, d] with host offsets
+    cu_ctx [b + 1]; caches [b, cap, Hkv, d] (or page pools with page_table [b, max_pages])
+    holding cache_lens[i] rows (host). Appends each new token's KV at row cache_lens[i]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bf16(t, n, 4)
+    _bf16(k_ctx, "k_ctx", 3)
+    _bf16(v_ctx, "v_ctx", 3)
+    cu, vals = _cu_array(cu_ctx)
+    lens, lvals = _cu_array(cache_lens)
+    b, _, hq, d = q.shape
+    if len(vals) != b + 1 or len(lvals) != b:
+        raise ValueError("cu_ctx needs batch + 1 offsets and cache_lens batch entries")
+    shape = make_shape(b, hq, k_ctx.shape[1], d, vals[-1], block_size, scale)
+    if workspace is None:
+        workspace = decode_varlen_workspace(b, hq, k_ctx.shape[1], d, vals, block_size, q.device,
+                                            scale)
+    if page_table is not None:
+        page_size, num_pages, max_pages = _page_pool(k_cache, v_cache, page_table)
+        cap = 0
+    else:
+        _bf16(k_cache, "k_cache", 4)
+        _bf16(v_cache, "v_cache", 4)
+        page_size = num_pages = max_pages = 0
+        cap = k_cache.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((b, hq, 1), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_phase2_decode_varlen(
+        ctypes.byref(shape), cu, lens, _ptr(q), _ptr(k), _ptr(v), _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(k_cache), _ptr(v_cache), cap, _ptr(page_table), page_size, num_pages, max_pages,
+        _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(), _stream()),
+        "star_attn_phase2_decode_varlen")
     return o, lse
 
 

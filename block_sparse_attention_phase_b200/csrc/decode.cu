@@ -70,6 +70,84 @@ STAR_HD constexpr size_t fused_merge_bytes(int64_t n_splits, int g, int d) {
   return fused_weights_bytes(n_splits, g) + size_t{kWarps} * g * d * 4;
 }
 
+template <class VL>
+constexpr bool kIsVarlen = sizeof(VL) == sizeof(DecVarlen);
+
+// The split a CTA streams, for a uniform batch (grid = splits x (batch * Hkv)) or a
+// varlen one (1-D grid; the sequence found by binary search in the CTA table).
+struct Split {
+  int bb, kvh, split, n_splits;
+  bool is_cache;
+  int64_t k0, k1;         // key range: context tokens of the sequence, or cache rows
+  int32_t ctx_tok, ctx_c3;  // context-map coordinate offset (packed varlen) and outer coordinate
+  int64_t cache_len;
+  int64_t prow;           // partial row (in units of Hq rows) of this split
+  int64_t prow0, pstride; // partial row of the sequence's split 0; step between splits
+  int ctr;                // fused-merge counter of (sequence, kv-head)
+};
+
+// A uniform batch needs no table: its launches carry this instead of DecVarlen.
+struct NoVarlen {
+  int32_t n;
+};
+
+template <class VL>
+__device__ __forceinline__ Split locate(const DecodeArgs& a, const VL& dv) {
+  Split w;
+  int64_t L = a.L, B = a.B, chunk = a.chunk;
+  int spb = a.spb, n_ctx = a.n_ctx;
+  if constexpr (!kIsVarlen<VL>) {
+    w.split = blockIdx.x;
+    w.bb = blockIdx.y / a.hkv;
+    w.kvh = blockIdx.y % a.hkv;
+    w.n_splits = gridDim.x;
+    w.cache_len = a.cache_len;
+    w.ctx_tok = 0;
+    w.ctx_c3 = w.bb;
+    w.prow = static_cast<int64_t>(w.split) * a.b + w.bb;
+    w.prow0 = w.bb;
+    w.pstride = a.b;
+    w.ctr = blockIdx.y;
+  } else {
+    const int r0 = blockIdx.x;
+    int lo = 0, hi = dv.n;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (dv.cta0[mid] <= r0) lo = mid; else hi = mid;
+    }
+    const int r = r0 - dv.cta0[lo];
+    w.n_splits = dv.split0[lo + 1] - dv.split0[lo];
+    w.kvh = r / w.n_splits;
+    w.split = r % w.n_splits;
+    w.bb = lo;
+    n_ctx = w.n_splits - 1;
+    L = dv.ctx0[lo + 1] - dv.ctx0[lo];
+    B = min(a.B, L);
+    spb = dv.spb[lo];
+    chunk = L > 0 ? (B + spb - 1) / spb : 1;
+    w.cache_len = dv.cache_len[lo];
+    w.ctx_tok = dv.ctx0[lo];
+    w.ctx_c3 = 0;
+    w.prow = dv.split0[lo] + w.split;
+    w.prow0 = dv.split0[lo];
+    w.pstride = 1;
+    w.ctr = lo * a.hkv + w.kvh;
+  }
+  w.is_cache = w.split == n_ctx;
+  if (!w.is_cache) {
+    const int64_t blk = w.split / spb;
+    const int64_t sub = w.split % spb;
+    const int64_t bstart = blk * B;
+    const int64_t bend = min(L, bstart + B);
+    w.k0 = min(bend, bstart + sub * chunk);
+    w.k1 = min(bend, w.k0 + chunk);
+  } else {
+    w.k0 = 0;
+    w.k1 = w.cache_len + 1;  // the cached rows and the new token, appended by the CTA
+  }
+  return w;
+}
+
 // Fused merge, run by the consumer threads of every CTA after it has stored its
 // partial: the CTA that completes the count of its (sequence, kv-head) is the
 // last one, all the other splits' partials are in memory, and it combines them
@@ -83,8 +161,7 @@ STAR_HD constexpr size_t fused_merge_bytes(int64_t n_splits, int g, int d) {
 // lane owning float4 columns of the split's contiguous G x D partial block, with
 // several splits' loads in flight; the warps' sums meet in shared memory.
 template <int D, int G>
-__device__ __forceinline__ void merge_if_last(const DecodeArgs& a, int bb, int kvh,
-                                              uint8_t* smem) {
+__device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const Split& w, uint8_t* smem) {
   __shared__ int s_last;
   __shared__ float s_red[kWarps][G];
   __shared__ float s_m[G], s_w[G];
@@ -92,9 +169,9 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, int bb, int k
   asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
   const int tid = threadIdx.x;  // 0 .. 127 (the consumer warps)
   if (tid == 0) {
-    uint32_t* ctr = a.counters + blockIdx.y;
+    uint32_t* ctr = a.counters + w.ctr;
     const uint32_t prev = atomicAdd(ctr, 1u);
-    const int last = prev == gridDim.x - 1;
+    const int last = prev == static_cast<uint32_t>(w.n_splits - 1);
     if (last) atomicExch(ctr, 0u);  // every split of this launch has counted
     s_last = last;
   }
@@ -104,9 +181,10 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, int bb, int k
 
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const int S = gridDim.x;
-  const int64_t row0 = static_cast<int64_t>(bb) * a.hq + kvh * G;  // split 0, first head
-  const int64_t stride = static_cast<int64_t>(a.b) * a.hq;         // rows per split
+  const int S = w.n_splits;
+  const int64_t row0 = w.prow0 * a.hq + w.kvh * G;  // partial row: split 0, first head
+  const int64_t stride = w.pstride * a.hq;         // rows between splits
+  const int64_t orow0 = static_cast<int64_t>(w.bb) * a.hq + w.kvh * G;  // output row
   float* wts = reinterpret_cast<float*>(smem);                     // [S][G]
   float4* red = reinterpret_cast<float4*>(smem + fused_weights_bytes(S, G));  // [kWarps][G*D/4]
 
@@ -193,7 +271,7 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, int bb, int k
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) W += s_red[w][tid];
     s_w[tid] = W;
-    if (a.lse) a.lse[row0 + tid] = W > 0.f ? s_m[tid] + logf(W) : -INFINITY;
+    if (a.lse) a.lse[orow0 + tid] = W > 0.f ? s_m[tid] + logf(W) : -INFINITY;
   }
   asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
   for (int f = tid; f < F; f += kWarps * 32) {
@@ -211,15 +289,15 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, int bb, int k
     uint2 packed;
     packed.x = pack_bf16x2(x.x * inv, x.y * inv);
     packed.y = pack_bf16x2(x.z * inv, x.w * inv);
-    *reinterpret_cast<uint2*>(a.o + row0 * D + 4 * f) = packed;  // G heads are contiguous
+    *reinterpret_cast<uint2*>(a.o + orow0 * D + 4 * f) = packed;  // G heads are contiguous
   }
 }
 
-template <int D, int G, int kStages>
+template <int D, int G, int kStages, class VL>
 __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decode_partials_kernel(
     const __grid_constant__ CUtensorMap mk_ctx, const __grid_constant__ CUtensorMap mv_ctx,
     const __grid_constant__ CUtensorMap mk_cache, const __grid_constant__ CUtensorMap mv_cache,
-    const DecodeArgs a) {
+    const DecodeArgs a, const __grid_constant__ VL dv) {
   constexpr int CH = D / 64;                        // 64-column chunks of a row
   constexpr uint32_t kChunk = kTile * 128;          // one chunk of a tile: 64 rows x 128 B
   constexpr uint32_t kTileBytes = CH * kChunk;
@@ -235,24 +313,17 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
-  const int bb = blockIdx.y / a.hkv;
-  const int kvh = blockIdx.y % a.hkv;
-  const bool is_cache = split == a.n_ctx;
-
-  int64_t k0, k1;
-  if (!is_cache) {
-    const int64_t blk = split / a.spb;
-    const int64_t sub = split % a.spb;
-    const int64_t bstart = blk * a.B;
-    const int64_t bend = min(a.L, bstart + a.B);
-    k0 = min(bend, bstart + sub * a.chunk);
-    k1 = min(bend, k0 + a.chunk);
-  } else {
-    k0 = 0;
-    k1 = a.cache_len + 1;  // the cached rows and the new token, appended below
-  }
+  const Split w = locate(a, dv);
+  const int bb = w.bb;
+  const int kvh = w.kvh;
+  const bool is_cache = w.is_cache;
+  const int64_t k0 = w.k0, k1 = w.k1;
+  const int64_t cache_len = w.cache_len;
   const int ntiles = static_cast<int>((k1 - k0 + kTile - 1) / kTile);
+  // Varlen batches with a contiguous cache cannot end each sequence's cache map at
+  // its own length, so rows past k1 in the cache's last tile are zeroed in shared
+  // memory instead (those rows may hold any bytes; P = 0 times NaN would be NaN).
+  const bool zero_tail = kIsVarlen<VL> && is_cache && !a.page_table;
 
   if (threadIdx.x == 0) {
 #pragma unroll
@@ -284,7 +355,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
       // outside the pool is refused (bounds flag, no write).
       int64_t page = 0;
       if (a.page_table) {
-        page = a.page_table[static_cast<int64_t>(bb) * a.max_pages + a.cache_len / a.page_size];
+        page = a.page_table[static_cast<int64_t>(bb) * a.max_pages + cache_len / a.page_size];
         if (page < 0 || page >= a.num_pages) {
           if (lane == 0) atomicOr(a.status, kBoundsFlag);
           page = -1;
@@ -297,14 +368,14 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
       };
       if (page >= 0) {
         const int64_t src = (static_cast<int64_t>(bb) * a.hkv + kvh) * D + lane * 8;
-        const int64_t dst = row_off(a.cache_len);
+        const int64_t dst = row_off(cache_len);
         *reinterpret_cast<uint4*>(a.k_cache + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
         *reinterpret_cast<uint4*>(a.v_cache + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
-        if (a.page_table && a.cache_len % a.page_size == 0) {
+        if (a.page_table && cache_len % a.page_size == 0) {
           // The append opens a new page: zero its other rows (for this kv-head), so
           // that tiles reaching past the last valid row read zeros, never stale bytes.
           const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-          for (int64_t r = a.cache_len + 1; r < a.cache_len + a.page_size; ++r) {
+          for (int64_t r = cache_len + 1; r < cache_len + a.page_size; ++r) {
             const int64_t off = row_off(r);
             *reinterpret_cast<uint4*>(a.k_cache + off) = z;
             *reinterpret_cast<uint4*>(a.v_cache + off) = z;
@@ -323,8 +394,13 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
         if (i >= kStages && !mbar_wait(&empty[stg], ph ^ 1, a.status)) break;
         mbar_arrive_expect_tx(&full[stg], 2 * kTileBytes);
         int32_t t0 = static_cast<int32_t>(k0 + static_cast<int64_t>(i) * kTile);
-        int32_t c3 = bb;  // the sequence, or for a paged cache the page holding this tile
-        if (is_cache && a.page_table) {
+        // Outer coordinate: the sequence (a packed varlen context: 0, with the
+        // sequence's first token added to t0), or for a paged cache the page.
+        int32_t c3 = bb;
+        if (!is_cache) {
+          t0 += w.ctx_tok;
+          c3 = w.ctx_c3;
+        } else if (a.page_table) {
           c3 = a.page_table[static_cast<int64_t>(bb) * a.max_pages + t0 / a.page_size];
           t0 %= a.page_size;
         }
@@ -373,6 +449,21 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
       if (ok) {
         const uint32_t kt = smem_u32(kbuf + stg * kTileBytes);
         const uint32_t vt = smem_u32(vbuf + stg * kTileBytes);
+        if (zero_tail && i == ntiles - 1) {
+          // this warp's 16 rows at or past k1: zero their K and V (whole 128-byte
+          // swizzle rows of every 64-column chunk)
+          const int64_t first = k1 - (k0 + static_cast<int64_t>(i) * kTile);  // first row to zero
+          for (int u = lane; u < 16 * CH * 8; u += 32) {
+            const int rr = tw0 + u / (CH * 8);
+            const int c = (u / 8) % CH;
+            if (rr >= first) {
+              const uint32_t off = stg * kTileBytes + c * kChunk + rr * 128 + (u % 8) * 16;
+              *reinterpret_cast<uint4*>(kbuf + off) = make_uint4(0u, 0u, 0u, 0u);
+              *reinterpret_cast<uint4*>(vbuf + off) = make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
+          __syncwarp();
+        }
         // ---- S = Q K^T for this warp's 16 tokens (two n-tiles of 8)
         float s[2][4];
 #pragma unroll
@@ -481,65 +572,58 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
         }
       }
       const int hq = kvh * G + h;
-      const int64_t row = static_cast<int64_t>(split) * a.b + bb;
+      const int64_t row = w.prow;
       a.o_parts[(row * a.hq + hq) * D + e] = lsum > 0.f ? acc / lsum : 0.f;
       if (e == 0) {
         a.lse_parts[row * a.hq + hq] =
             lsum > 0.f ? (M * sl2 + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
       }
     }
-    if (a.counters) merge_if_last<D, G>(a, bb, kvh, base);
+    if (a.counters) merge_if_last<D, G>(a, w, base);
   }
 }
 
-template <int D, int G, int kStages>
-cudaError_t launch_decode_t(const Shape& s, const SplitPlan& p, const DecodeArgs& a,
-                            const void* kc, const void* vc, int32_t num_pages, cudaStream_t st) {
+// Context maps: uniform [b, L, Hkv, D], or a packed varlen context [total, Hkv, D]
+// (ctx_batch = 1). Cache maps: the page pool; a contiguous uniform cache whose
+// extent ends after the new row (rows past it read as zeros); or a contiguous varlen
+// cache, all rows in bounds (the kernel zeroes the tail rows in shared memory).
+template <int D, int G, int kStages, class VL>
+cudaError_t launch_decode_t(const Shape& s, const DecodeArgs& a, const VL& dv, dim3 grid,
+                            int64_t max_splits, uint64_t ctx_tokens, uint64_t ctx_batch,
+                            int32_t num_pages, const void* kc, const void* vc, cudaStream_t st) {
   alignas(64) CUtensorMap m[4];
-  bool ok = encode_tma_bf16_4d(&m[0], kc, D, s.hkv, s.L, s.L, s.b, 64, 1, kTile, true) &&
-            encode_tma_bf16_4d(&m[1], vc, D, s.hkv, s.L, s.L, s.b, 64, 1, kTile, true);
+  bool ok = encode_tma_bf16_4d(&m[0], kc, D, s.hkv, ctx_tokens, ctx_tokens, ctx_batch, 64, 1, kTile, true) &&
+            encode_tma_bf16_4d(&m[1], vc, D, s.hkv, ctx_tokens, ctx_tokens, ctx_batch, 64, 1, kTile, true);
   if (a.page_table) {
-    // The page pool [pages, P, Hkv, D]; rows past the valid ones in a sequence's
-    // last page hold zeros (written when the page was opened).
     ok = ok &&
          encode_tma_bf16_4d(&m[2], a.k_cache, D, s.hkv, a.page_size, a.page_size, num_pages, 64, 1, kTile, true) &&
          encode_tma_bf16_4d(&m[3], a.v_cache, D, s.hkv, a.page_size, a.page_size, num_pages, 64, 1, kTile, true);
   } else {
-    // The cache map covers the cached rows and the new one; rows past them read as zeros.
-    const uint64_t cache_rows = static_cast<uint64_t>(a.cache_len + 1);
+    const uint64_t cache_rows = kIsVarlen<VL> ? static_cast<uint64_t>(a.cap) : static_cast<uint64_t>(a.cache_len + 1);
     ok = ok &&
          encode_tma_bf16_4d(&m[2], a.k_cache, D, s.hkv, cache_rows, a.cap, s.b, 64, 1, kTile, true) &&
          encode_tma_bf16_4d(&m[3], a.v_cache, D, s.hkv, cache_rows, a.cap, s.b, 64, 1, kTile, true);
   }
   if (!ok) return cudaErrorInvalidValue;
-  if (a.counters && fused_merge_bytes(p.n_splits, G, D) > ring_bytes(D, kStages))
+  if (a.counters && fused_merge_bytes(max_splits, G, D) > ring_bytes(D, kStages))
     return cudaErrorInvalidValue;
   const size_t smem = ring_bytes(D, kStages) + 2 * kStages * sizeof(uint64_t) + 1024;
-  auto kern = decode_partials_kernel<D, G, kStages>;
+  auto kern = decode_partials_kernel<D, G, kStages, VL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const dim3 grid(p.n_splits, s.b * s.hkv);
-  e = launch_programmatic(kern, grid, dim3((kWarps + 1) * 32), smem, st, m[0], m[1], m[2], m[3], a);
+  e = launch_programmatic(kern, grid, dim3((kWarps + 1) * 32), smem, st, m[0], m[1], m[2], m[3], a,
+                          dv);
   if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();
 }
 
-int decode_stages(const SplitPlan& p) { return p.chunk <= kShortChunk ? 2 : 3; }
+int decode_stages(int64_t chunk) { return chunk <= kShortChunk ? 2 : 3; }
 
-}  // namespace
-
-bool decode_fused_fits(const Shape& s, const SplitPlan& p) {
-  return fused_merge_bytes(p.n_splits, s.group(), s.d) <= ring_bytes(s.d, decode_stages(p));
-}
-
-cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const void* q,
-                                   const void* k_new, const void* v_new, const void* kc,
-                                   const void* vc, const CacheRef& c, int64_t cache_len,
-                                   float* o_parts, float* lse_parts, const FusedMerge* fm,
-                                   cudaStream_t st) {
-  DecodeArgs a;
+DecodeArgs make_args(const Shape& s, const void* q, const void* k_new, const void* v_new,
+                     const CacheRef& c, float* o_parts, float* lse_parts, const FusedMerge* fm) {
+  DecodeArgs a{};
   a.o = fm ? static_cast<__nv_bfloat16*>(fm->o) : nullptr;
   a.lse = fm ? fm->lse : nullptr;
   a.counters = fm ? fm->counters : nullptr;
@@ -548,7 +632,6 @@ cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const voi
   a.v_new = static_cast<const __nv_bfloat16*>(v_new);
   a.k_cache = static_cast<__nv_bfloat16*>(c.k);
   a.v_cache = static_cast<__nv_bfloat16*>(c.v);
-  a.cache_len = cache_len;
   a.cap = c.cap;
   a.page_table = c.page_table;
   a.page_size = c.page_size;
@@ -556,9 +639,6 @@ cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const voi
   a.num_pages = c.num_pages;
   a.L = s.L;
   a.B = s.B;
-  a.chunk = p.chunk;
-  a.spb = p.spb;
-  a.n_ctx = p.n_ctx;
   a.b = s.b;
   a.hq = s.hq;
   a.hkv = s.hkv;
@@ -566,17 +646,100 @@ cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const voi
   a.o_parts = o_parts;
   a.lse_parts = lse_parts;
   a.status = device_status_word();
+  return a;
+}
+
+template <class VL>
+cudaError_t dispatch(const Shape& s, const DecodeArgs& a, const VL& dv, dim3 grid,
+                     int64_t max_splits, int64_t max_chunk, uint64_t ctx_tokens, uint64_t ctx_batch,
+                     int32_t num_pages, const void* kc, const void* vc, cudaStream_t st) {
   const int G = s.group();
-  const bool two = decode_stages(p) == 2;
-#define STAR_DECODE_CASE(DD, GG)                                                              \
-  if (s.d == DD && G == GG)                                                                   \
-    return two ? launch_decode_t<DD, GG, 2>(s, p, a, kc, vc, c.num_pages, st)                 \
-               : launch_decode_t<DD, GG, 3>(s, p, a, kc, vc, c.num_pages, st);
+  const bool two = decode_stages(max_chunk) == 2;
+#define STAR_DECODE_CASE(DD, GG)                                                                  \
+  if (s.d == DD && G == GG)                                                                       \
+    return two ? launch_decode_t<DD, GG, 2, VL>(s, a, dv, grid, max_splits, ctx_tokens,         \
+                                                ctx_batch, num_pages, kc, vc, st)                 \
+               : launch_decode_t<DD, GG, 3, VL>(s, a, dv, grid, max_splits, ctx_tokens,         \
+                                                ctx_batch, num_pages, kc, vc, st);
   STAR_DECODE_CASE(128, 1) STAR_DECODE_CASE(128, 2) STAR_DECODE_CASE(128, 4)
   STAR_DECODE_CASE(128, 8) STAR_DECODE_CASE(64, 1) STAR_DECODE_CASE(64, 2)
   STAR_DECODE_CASE(64, 4) STAR_DECODE_CASE(64, 8)
 #undef STAR_DECODE_CASE
   return cudaErrorNotSupported;
+}
+
+}  // namespace
+
+bool decode_fused_fits(const Shape& s, const SplitPlan& p) {
+  return fused_merge_bytes(p.n_splits, s.group(), s.d) <= ring_bytes(s.d, decode_stages(p.chunk));
+}
+
+cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const void* q,
+                                   const void* k_new, const void* v_new, const void* kc,
+                                   const void* vc, const CacheRef& c, int64_t cache_len,
+                                   float* o_parts, float* lse_parts, const FusedMerge* fm,
+                                   cudaStream_t st) {
+  DecodeArgs a = make_args(s, q, k_new, v_new, c, o_parts, lse_parts, fm);
+  a.cache_len = cache_len;
+  a.chunk = p.chunk;
+  a.spb = p.spb;
+  a.n_ctx = p.n_ctx;
+  NoVarlen dv;
+  dv.n = 0;
+  return dispatch(s, a, dv, dim3(p.n_splits, s.b * s.hkv), p.n_splits, p.chunk, s.L, s.b,
+                  c.num_pages, kc, vc, st);
+}
+
+int64_t plan_decode_varlen(const Shape& s, const int64_t* cu_ctx, const int64_t* cache_lens,
+                           int64_t target_ctas, DecVarlen* dv, int64_t* max_splits,
+                           int64_t* max_chunk) {
+  const int64_t total = cu_ctx[s.b];
+  const int64_t ctx_ctas = target_ctas - static_cast<int64_t>(s.b) * s.hkv;
+  int64_t C = ctx_ctas > 0 ? (total * s.hkv + ctx_ctas - 1) / ctx_ctas : total;
+  if (C < kTile) C = kTile;  // at least one TMA tile of keys per split
+  dv->n = s.b;
+  int64_t splits = 0, ctas = 0;
+  *max_splits = 1;
+  *max_chunk = kTile;
+  for (int i = 0; i < s.b; ++i) {
+    const int64_t L = cu_ctx[i + 1] - cu_ctx[i];
+    int64_t spb = 1, n_ctx = 0;
+    if (L > 0) {
+      const int64_t B = s.B < L ? s.B : L;
+      spb = (B + C - 1) / C;
+      n_ctx = (L + B - 1) / B * spb;
+      const int64_t chunk = (B + spb - 1) / spb;
+      if (chunk > *max_chunk) *max_chunk = chunk;
+    }
+    const int64_t ns = n_ctx + 1;
+    if (ns > *max_splits) *max_splits = ns;
+    dv->cta0[i] = static_cast<int32_t>(ctas);
+    dv->split0[i] = static_cast<int32_t>(splits);
+    dv->ctx0[i] = static_cast<int32_t>(cu_ctx[i]);
+    dv->spb[i] = static_cast<int32_t>(spb);
+    dv->cache_len[i] = static_cast<int32_t>(cache_lens[i]);
+    splits += ns;
+    ctas += ns * s.hkv;
+    if (ctas > 0x7fffffffLL) return -1;
+  }
+  dv->cta0[s.b] = static_cast<int32_t>(ctas);
+  dv->split0[s.b] = static_cast<int32_t>(splits);
+  dv->ctx0[s.b] = static_cast<int32_t>(total);
+  return splits;
+}
+
+cudaError_t launch_decode_varlen(const Shape& s, const DecVarlen& dv, int64_t max_splits,
+                                 int64_t max_chunk, const void* q, const void* k_new,
+                                 const void* v_new, const void* kc, const void* vc,
+                                 const CacheRef& c, float* o_parts, float* lse_parts,
+                                 const FusedMerge& fm, cudaStream_t st) {
+  DecodeArgs a = make_args(s, q, k_new, v_new, c, o_parts, lse_parts, &fm);
+  return dispatch(s, a, dv, dim3(dv.cta0[s.b]), max_splits, max_chunk, dv.ctx0[s.b], 1,
+                  c.num_pages, kc, vc, st);
+}
+
+bool decode_varlen_fused_fits(const Shape& s, int64_t max_splits, int64_t max_chunk) {
+  return fused_merge_bytes(max_splits, s.group(), s.d) <= ring_bytes(s.d, decode_stages(max_chunk));
 }
 
 }  // namespace star

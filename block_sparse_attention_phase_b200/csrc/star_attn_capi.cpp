@@ -6,6 +6,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <vector>
 
 #include "../../include/star_attn.h"
 #include "star_internal.h"
@@ -68,6 +69,30 @@ SplitPlan make_plan(const Shape& s, int64_t target_ctas) {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Host offsets of a varlen batch: cu[0] = 0, non-decreasing, cu[n] = total.
+bool valid_offsets(const int64_t* cu, int n, int64_t total) {
+  if (cu[0] != 0 || cu[n] != total) return false;
+  for (int i = 0; i < n; ++i)
+    if (cu[i + 1] < cu[i]) return false;
+  return true;
+}
+
+int64_t varlen_target_ctas() { return int64_t{kSMs} * kDecodeCtasPerSM; }
+
+// Varlen decode workspace = [o_parts][lse_parts][counters: b * Hkv uint32], each
+// 256-B aligned; partial rows = the plan's splits.
+size_t varlen_decode_bytes(const Shape& s, const int64_t* cu_ctx) {
+  std::vector<int64_t> zeros(static_cast<size_t>(s.b), 0);
+  DecVarlen dv;
+  int64_t max_splits = 0, max_chunk = 0;
+  const int64_t splits = plan_decode_varlen(s, cu_ctx, zeros.data(), varlen_target_ctas(), &dv,
+                                            &max_splits, &max_chunk);
+  if (splits < 0) return 0;
+  const size_t per = static_cast<size_t>(splits) * s.hq;
+  return align256(per * s.d * sizeof(float)) + align256(per * sizeof(float)) +
+         align256(static_cast<size_t>(s.b) * s.hkv * 4);
+}
 
 // Page-pool arguments: a tile (128 query-pass rows, 64 decode rows) must never
 // straddle two pages, and TMA coordinates of a page are 32-bit.
@@ -303,6 +328,66 @@ STAR_ATTN_API star_status_t star_attn_phase2_decode_fused(
   return star::cuda_status(star::launch_decode_partials(
       s, plan, q, k, v, k_ctx, v_ctx, c, cache_len, static_cast<float*>(workspace),
       star::lse_parts_of(workspace, s, plan, 1), &fm, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+STAR_ATTN_API size_t star_attn_decode_varlen_workspace_bytes(const star_attn_shape_t* shape,
+                                                             const int64_t* cu_ctx) {
+  Shape s;
+  if (star::resolve(shape, &s) != STAR_OK || !cu_ctx || s.b > star::kMaxVarSeqs) return 0;
+  if (!star::valid_offsets(cu_ctx, s.b, s.L)) return 0;
+  return star::varlen_decode_bytes(s, cu_ctx);
+}
+
+STAR_ATTN_API star_status_t star_attn_phase2_decode_varlen(
+    const star_attn_shape_t* shape, const int64_t* cu_ctx, const int64_t* cache_lens,
+    const void* q, const void* k, const void* v, const void* k_ctx, const void* v_ctx,
+    void* k_cache, void* v_cache, int64_t cache_capacity, const int32_t* page_table,
+    int32_t page_size, int32_t num_pages, int32_t max_pages, void* o, float* lse,
+    void* workspace, size_t workspace_bytes, star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (s.b > star::kMaxVarSeqs) return STAR_ERR_UNSUPPORTED;
+  if (!cu_ctx || !cache_lens || !star::valid_offsets(cu_ctx, s.b, s.L)) return STAR_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, k_ctx, v_ctx, k_cache, v_cache, o};
+  for (const void* p : ptrs)
+    if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned4(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
+  star::CacheRef c;
+  if (page_table) {
+    st = star::check_pages(page_size, num_pages, page_table, max_pages);
+    if (st != STAR_OK) return st;
+    c = star::paged_ref(k_cache, v_cache, page_size, num_pages, page_table, max_pages);
+  } else {
+    if (cache_capacity < 1) return STAR_ERR_INVALID_ARG;
+    c.k = k_cache;
+    c.v = v_cache;
+    c.cap = cache_capacity;
+  }
+  for (int i = 0; i < s.b; ++i) {
+    if (cache_lens[i] < 0 || cache_lens[i] > (int64_t{1} << 30)) return STAR_ERR_INVALID_ARG;
+    if (page_table ? cache_lens[i] / page_size + 1 > max_pages : cache_lens[i] + 1 > cache_capacity)
+      return STAR_ERR_CACHE_FULL;
+  }
+  star::DecVarlen dv;
+  int64_t max_splits = 0, max_chunk = 0;
+  const int64_t splits = star::plan_decode_varlen(s, cu_ctx, cache_lens, star::varlen_target_ctas(),
+                                                  &dv, &max_splits, &max_chunk);
+  if (splits < 0 || !star::decode_varlen_fused_fits(s, max_splits, max_chunk))
+    return STAR_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < star::varlen_decode_bytes(s, cu_ctx)) return STAR_ERR_WORKSPACE;
+  const size_t per = static_cast<size_t>(splits) * s.hq;
+  char* ws = static_cast<char*>(workspace);
+  float* o_parts = reinterpret_cast<float*>(ws);
+  float* lse_parts = reinterpret_cast<float*>(ws + star::align256(per * s.d * sizeof(float)));
+  star::FusedMerge fm;
+  fm.o = o;
+  fm.lse = lse;
+  fm.counters = reinterpret_cast<uint32_t*>(ws + star::align256(per * s.d * sizeof(float)) +
+                                            star::align256(per * sizeof(float)));
+  return star::cuda_status(star::launch_decode_varlen(s, dv, max_splits, max_chunk, q, k, v,
+                                                      k_ctx, v_ctx, c, o_parts, lse_parts, fm,
+                                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 STAR_ATTN_API star_status_t star_attn_phase2_query_paged(

@@ -86,6 +86,20 @@ struct VarSeqs {
   int32_t start[kMaxVarSeqs + 1];
 };
 
+// A varlen decode batch (kernel parameter): sequence i owns CTAs [cta0[i], cta0[i+1])
+// (its splits x Hkv), partial rows [split0[i], split0[i+1]) (one per split; the last
+// is its query-local cache), context tokens [ctx0[i], ctx0[i+1]) of the packed
+// context, spb[i] chunks per context block, and cache_len[i] cached rows.
+// n = 0: a uniform batch.
+struct DecVarlen {
+  int32_t n;
+  int32_t cta0[kMaxVarSeqs + 1];
+  int32_t split0[kMaxVarSeqs + 1];
+  int32_t ctx0[kMaxVarSeqs + 1];
+  int32_t spb[kMaxVarSeqs];
+  int32_t cache_len[kMaxVarSeqs];
+};
+
 // Device status word of the current device (address valid on that device).
 uint32_t* device_status_word();
 
@@ -118,6 +132,19 @@ cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const voi
                                    cudaStream_t st);
 // Whether the fused merge's weights and sums fit in the decode kernel's shared memory.
 bool decode_fused_fits(const Shape& s, const SplitPlan& p);
+// Varlen decode: split plan (s.b sequences, packed context offsets cu_ctx and cache
+// lengths, both host arrays) aiming at about target_ctas CTAs. Returns the total
+// split count (partial rows), or -1 if the grid would be too large.
+int64_t plan_decode_varlen(const Shape& s, const int64_t* cu_ctx, const int64_t* cache_lens,
+                           int64_t target_ctas, DecVarlen* dv, int64_t* max_splits,
+                           int64_t* max_chunk);
+bool decode_varlen_fused_fits(const Shape& s, int64_t max_splits, int64_t max_chunk);
+// One fused decode step over a varlen batch (always with the last-CTA merge).
+cudaError_t launch_decode_varlen(const Shape& s, const DecVarlen& dv, int64_t max_splits,
+                                 int64_t max_chunk, const void* q, const void* k_new,
+                                 const void* v_new, const void* kc, const void* vc,
+                                 const CacheRef& c, float* o_parts, float* lse_parts,
+                                 const FusedMerge& fm, cudaStream_t st);
 cudaError_t launch_phase1_sm100(const Shape& s, const void* q, const void* k, const void* v,
                                 void* o, float* lse, cudaStream_t st);
 // Phase 1 over a varlen batch: s.b sequences packed along tokens, s.L = total tokens,

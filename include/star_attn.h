@@ -193,6 +193,40 @@ STAR_ATTN_API star_status_t star_attn_phase2_decode_fused(
     star_stream_t stream);
 
 /*
+ * One decode step over a varlen batch (continuous batching): every sequence has its
+ * own context length and its own number of cached query-local rows. Same
+ * computation per sequence as star_attn_phase2_decode() with batch 1, in one
+ * launch, with the merge fused (last-CTA merge, as star_attn_phase2_decode_fused()).
+ *   shape->batch = sequences (at most 128); shape->ctx_len = total context tokens.
+ *   cu_ctx: HOST int64 [batch + 1] offsets of each sequence's context in the packed
+ *     k_ctx, v_ctx [total, Hkv, d] (cu_ctx[0] = 0, non-decreasing, last = total;
+ *     an empty context is allowed).
+ *   cache_lens: HOST int64 [batch], rows already cached per sequence; the new
+ *     token's KV is appended at row cache_lens[i] of sequence i.
+ *   q [batch, 1, Hq, d]; k, v [batch, 1, Hkv, d]; o [batch, 1, Hq, d]; lse [batch, Hq, 1] or NULL.
+ *   The query-local cache is either contiguous, k_cache/v_cache [batch, cache_capacity,
+ *     Hkv, d] (page_table NULL; rows past a sequence's cached ones may hold any
+ *     bytes), or a page pool as in star_attn_phase2_decode_paged() (page_table
+ *     [batch, max_pages], page_size, num_pages; cache_capacity ignored).
+ *   workspace: star_attn_decode_varlen_workspace_bytes(shape, cu_ctx) bytes, all zero
+ *     before its first use; every call leaves it reusable for the same cu_ctx.
+ * Errors: STAR_ERR_CACHE_FULL if a sequence has no room for its new row;
+ * STAR_ERR_UNSUPPORTED for more than 128 sequences, or a plan whose merge does not
+ * fit in shared memory (thousands of context blocks in one sequence).
+ * No counterpart on the pages (a serving-side batch of sequences at different
+ * lengths; the per-sequence computation is the Phase-2 decode step's).
+ */
+STAR_ATTN_API size_t star_attn_decode_varlen_workspace_bytes(const star_attn_shape_t* shape,
+                                                             const int64_t* cu_ctx);
+
+STAR_ATTN_API star_status_t star_attn_phase2_decode_varlen(
+    const star_attn_shape_t* shape, const int64_t* cu_ctx, const int64_t* cache_lens,
+    const void* q, const void* k, const void* v, const void* k_ctx, const void* v_ctx,
+    void* k_cache, void* v_cache, int64_t cache_capacity, const int32_t* page_table,
+    int32_t page_size, int32_t num_pages, int32_t max_pages, void* o, float* lse,
+    void* workspace, size_t workspace_bytes, star_stream_t stream);
+
+/*
  * Paged query-local cache (paperhub.cn page, the authors' response to Reviewer
  * dKGV, item 3 "Compatibility with Parallelism Methods and Serving Frameworks":
  * PagedAttention-style memory management applies within each host to its local

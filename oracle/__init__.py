@@ -37,4 +37,5 @@ from .star_oracle import (  # noqa: F401
     phase2_query,
     phase2_decode_head,
     phase2_decode,
+    phase2_decode_varlen,
 )

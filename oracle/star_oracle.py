@@ -279,3 +279,24 @@ def phase2_decode(q_t, k_t, v_t, k_ctx, v_ctx, k_cache, v_cache, cache_len: int,
     k_cache_new[:, cache_len] = np.asarray(k_t, F64)[:, 0]
     v_cache_new[:, cache_len] = np.asarray(v_t, F64)[:, 0]
     return o, lse, k_cache_new, v_cache_new
+
+
+def phase2_decode_varlen(q_t, k_t, v_t, k_ctx, v_ctx, cu_ctx: Sequence[int], k_cache, v_cache,
+                         cache_lens: Sequence[int], scale: float = None):
+    """One decode step over a varlen batch: sequence i has the context tokens
+    [cu_ctx[i], cu_ctx[i+1]) of the packed k_ctx, v_ctx [total, Hkv, d] and
+    cache_lens[i] cached rows of k_cache, v_cache [b, cap, Hkv, d]; q_t [b, 1, Hq, d],
+    k_t, v_t [b, 1, Hkv, d]. Each sequence is the decode step of its own slice.
+    Returns o [b, 1, Hq, d], lse [b, Hq, 1] and the caches with every new row appended."""
+    b, _, Hq, d = q_t.shape
+    o = np.zeros((b, 1, Hq, d), dtype=F64)
+    lse = np.zeros((b, Hq, 1), dtype=F64)
+    k_new = np.array(k_cache, dtype=F64, copy=True)
+    v_new = np.array(v_cache, dtype=F64, copy=True)
+    for i in range(b):
+        a, e = cu_ctx[i], cu_ctx[i + 1]
+        oi, li, ki, vi = phase2_decode(q_t[i:i + 1], k_t[i:i + 1], v_t[i:i + 1], k_ctx[None, a:e],
+                                       v_ctx[None, a:e], k_cache[i:i + 1], v_cache[i:i + 1],
+                                       cache_lens[i], scale)
+        o[i], lse[i], k_new[i], v_new[i] = oi[0], li[0], ki[0], vi[0]
+    return o, lse, k_new, v_new

@@ -287,12 +287,40 @@ def check_phase1_varlen_per_sequence(seed=9):
         np.testing.assert_allclose(lse[:, a:e], rl, atol=1e-12)
 
 
+def check_decode_varlen_is_global_per_sequence(seed=10):
+    """Varlen decode: sequence i's new token attends to exactly its own context,
+    its own cached rows and itself (torch SDPA over that concatenation), and its
+    KV lands at row cache_lens[i] of its own cache only."""
+    rng = np.random.default_rng(seed)
+    Hq, Hkv, d, cap = 4, 2, 8, 6
+    ctx_lens, cache_lens = [7, 0, 12], [2, 5, 0]
+    b = len(ctx_lens)
+    cu = [0] + list(np.cumsum(ctx_lens))
+    kc, vc = rand(rng, cu[-1], Hkv, d), rand(rng, cu[-1], Hkv, d)
+    kcache, vcache = rand(rng, b, cap, Hkv, d), rand(rng, b, cap, Hkv, d)
+    q, k, v = rand(rng, b, 1, Hq, d), rand(rng, b, 1, Hkv, d), rand(rng, b, 1, Hkv, d)
+    scale = 0.4
+    o, lse, kn, vn = oracle.phase2_decode_varlen(q, k, v, kc, vc, cu, kcache, vcache, cache_lens,
+                                                 scale)
+    for i in range(b):
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            keys = np.concatenate([kc[cu[i]:cu[i + 1], g], kcache[i, :cache_lens[i], g], k[i, :, g]])
+            vals = np.concatenate([vc[cu[i]:cu[i + 1], g], vcache[i, :cache_lens[i], g], v[i, :, g]])
+            ro, rl = sdpa_rows(q[i, :, h], keys, vals, scale)
+            np.testing.assert_allclose(o[i, 0, h], ro[0], atol=1e-12)
+            np.testing.assert_allclose(lse[i, h, 0], rl[0], atol=1e-12)
+        expect_k = kcache[i].copy()
+        expect_k[cache_lens[i]] = k[i, 0]
+        np.testing.assert_array_equal(kn[i], expect_k)
+
+
 ALL_CHECKS = [check_single_block_is_causal, check_two_blocks_is_full_causal,
               check_phase1_keysets_golden, check_first_and_last_row_of_block,
               check_block_independence, check_gqa_mapping, check_closed_forms,
               check_phase2_query_is_global, check_phase2_keysets_golden,
               check_merge_split_invariance, check_decode_matches_query_rows,
-              check_phase1_varlen_per_sequence]
+              check_phase1_varlen_per_sequence, check_decode_varlen_is_global_per_sequence]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda c: c.__name__)
@@ -358,8 +386,19 @@ def _mut_varlen_one_context(q, k, v, cu_seqlens, block_size, scale=None):
     return o[0], lse[0]
 
 
+_orig_decode_varlen = so.phase2_decode_varlen
+
+
+def _mut_decode_varlen_first_len(q_t, k_t, v_t, k_ctx, v_ctx, cu_ctx, k_cache, v_cache,
+                                 cache_lens, scale=None):
+    # every sequence given the first sequence's cache length
+    return _orig_decode_varlen(q_t, k_t, v_t, k_ctx, v_ctx, cu_ctx, k_cache, v_cache,
+                               [cache_lens[0]] * len(cache_lens), scale)
+
+
 MUTANTS = {
     "varlen_one_context": ("phase1_varlen", _mut_varlen_one_context),
+    "decode_varlen_first_len": ("phase2_decode_varlen", _mut_decode_varlen_first_len),
     "anchor_is_previous_block": ("phase1_visible", _mut_anchor_previous),
     "no_anchor": ("phase1_visible", _mut_no_anchor),
     "strict_causal": ("phase1_visible", _mut_strict_causal),

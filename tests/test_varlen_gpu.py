@@ -69,3 +69,73 @@ def test_phase1_varlen_long_sequences_equal_alone():
                                 oracle.default_scale(128), rows)
     check_rows(to_np(o[a + rows, 5]), ro, to_np(lse[5, a + rows]), rl, "varlen long")
     assert m.device_status() == 0
+
+
+DEC_CASES = [
+    # ctx lens, cache lens, Hq, Hkv, d, B, paged page size (0: contiguous)
+    ([3000, 0, 700, 9000], [5, 0, 17, 130], 8, 2, 128, 1024, 0),
+    ([3000, 0, 700, 9000], [5, 0, 127, 130], 8, 2, 128, 1024, 128),
+    ([513, 2048], [64, 3], 8, 1, 64, 512, 0),           # G = 8
+    ([40000, 100, 12000], [1, 2, 3], 32, 8, 128, 4096, 256),
+]
+
+
+@pytest.mark.parametrize("case", DEC_CASES, ids=lambda c: f"{len(c[0])}seq_g{c[2]//c[3]}_d{c[4]}_p{c[6]}")
+def test_decode_varlen_matches_oracle(case):
+    ctx_lens, lens0, hq, hkv, d, B, P = case
+    m = sa()
+    b = len(ctx_lens)
+    T = 3
+    g = torch.Generator(device="cpu").manual_seed(len(ctx_lens) * 7 + d)
+    rnd = lambda *shape: (torch.randn(*shape, generator=g) / d ** 0.5).to(torch.bfloat16).cuda()
+    cu = [0]
+    for n in ctx_lens:
+        cu.append(cu[-1] + n)
+    kc, vc = rnd(cu[-1], hkv, d), rnd(cu[-1], hkv, d)
+    cap = max(lens0) + T
+    k_rows, v_rows = rnd(b, cap, hkv, d), rnd(b, cap, hkv, d)  # rows [0, lens0[i]) are valid
+    if P:
+        max_pages = (cap + P - 1) // P
+        num_pages = b * max_pages + 2
+        gp = torch.Generator().manual_seed(3)
+        table = torch.randperm(num_pages, generator=gp)[: b * max_pages].view(b, max_pages)
+        table = table.to(torch.int32).cuda()
+        kp = torch.zeros((num_pages, P, hkv, d), dtype=torch.bfloat16, device="cuda")
+        vp = torch.zeros_like(kp)
+        for i in range(b):
+            for r in range(lens0[i]):
+                kp[int(table[i, r // P]), r % P] = k_rows[i, r]
+                vp[int(table[i, r // P]), r % P] = v_rows[i, r]
+        kcache, vcache = kp, vp
+    else:
+        table = None
+        kcache = torch.full((b, cap, hkv, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        vcache = torch.full_like(kcache, float("nan"))
+        for i in range(b):
+            kcache[i, :lens0[i]] = k_rows[i, :lens0[i]]
+            vcache[i, :lens0[i]] = v_rows[i, :lens0[i]]
+    ws = m.decode_varlen_workspace(b, hq, hkv, d, cu, B, "cuda")
+    k_ref = np.zeros((b, cap, hkv, d))
+    v_ref = np.zeros((b, cap, hkv, d))
+    for i in range(b):
+        k_ref[i, :lens0[i]] = to_np(k_rows[i, :lens0[i]])
+        v_ref[i, :lens0[i]] = to_np(v_rows[i, :lens0[i]])
+    for t in range(T):
+        lens = [n + t for n in lens0]
+        q, k, v = rnd(b, 1, hq, d), rnd(b, 1, hkv, d), rnd(b, 1, hkv, d)
+        o, lse = m.phase2_decode_varlen(q, k, v, kc, vc, cu, kcache, vcache, lens, B,
+                                        page_table=table, workspace=ws)
+        ro, rl, k_ref, v_ref = oracle.phase2_decode_varlen(
+            to_np(q), to_np(k), to_np(v), to_np(kc), to_np(vc), cu, k_ref, v_ref, lens)
+        check_rows(to_np(o), ro, to_np(lse), rl, f"decode varlen {case} t={t}")
+        # the counters (the workspace's last 256-byte-aligned segment) are back at zero
+        seg = (4 * b * hkv + 255) // 256 * 256
+        ctr = ws[ws.numel() - seg: ws.numel() - seg + 4 * b * hkv].view(torch.int32)
+        assert int(ctr.abs().sum()) == 0
+        for i in range(b):  # the new row landed in sequence i's cache only
+            if P:
+                row = kcache[int(table[i, lens[i] // P]), lens[i] % P]
+            else:
+                row = kcache[i, lens[i]]
+            assert torch.equal(row, k[i, 0])
+    assert m.device_status() == 0
