@@ -33,6 +33,7 @@ STATUS_NAMES = {0: "STAR_OK", 1: "STAR_ERR_INVALID_ARG", 2: "STAR_ERR_UNSUPPORTE
 
 # Every symbol the header declares; tests check that the library exports them all.
 EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase1_varlen",
+            "star_attn_rope", "star_attn_phase1_anchor_q",
             "star_attn_phase2_query",
             "star_attn_phase2_decode", "star_attn_phase2_decode_fused",
             "star_attn_phase2_decode_varlen", "star_attn_decode_varlen_workspace_bytes",
@@ -75,6 +76,8 @@ def lib() -> ctypes.CDLL:
         "star_attn_workspace_bytes": (SZ, [SP, I32, I64]),
         "star_attn_phase1": (I32, [SP, P, P, P, P, P, P]),
         "star_attn_phase1_varlen": (I32, [SP, ctypes.POINTER(I64), P, P, P, P, P, P]),
+        "star_attn_rope": (I32, [SP, ctypes.POINTER(ctypes.c_float), I64, P, P, P, P, P, P]),
+        "star_attn_phase1_anchor_q": (I32, [SP, P, P, P, P, P, P, P]),
         "star_attn_phase2_query": (I32, [SP, P, P, P, I64, P, P, P, P, I64, P, P, P, SZ, P]),
         "star_attn_phase2_decode": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P, SZ, P]),
         "star_attn_phase2_decode_fused": (I32, [SP, P, P, P, P, P, P, P, I64, I64, P, P, P, SZ,
@@ -157,6 +160,51 @@ def phase1(q, k, v, block_size: int, scale: Optional[float] = None, o=None, lse=
         lse = torch.empty((b, hq, L), dtype=torch.float32, device=q.device)
     _check(lib().star_attn_phase1(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                   _ptr(lse), _stream()), "star_attn_phase1")
+    return o, lse
+
+
+def rope_inv_freq(head_dim: int, base: float = 500000.0):
+    """Plain RoPE frequencies base^(-2f/d), f < d/2, as float32 values."""
+    import numpy as np
+    f = np.arange(head_dim // 2, dtype=np.float64)
+    return (base ** (-2.0 * f / head_dim)).astype(np.float32)
+
+
+def rope(q, k, inv_freq, pos0: int = 0, block_size: int = 1, want_anchor: bool = False,
+         inplace: bool = False):
+    """RoPE on q [b, L, Hq, d] and k [b, L, Hkv, d] at positions pos0 + t. Returns
+    (q_rot, k_rot, q_anchor or None); q_anchor is q rotated at the anchor-position
+    variant's positions for blocks of block_size tokens."""
+    _bf16(q, "q", 4)
+    _bf16(k, "k", 4)
+    b, L, hq, d = q.shape
+    freqs = [float(x) for x in inv_freq]
+    if len(freqs) != d // 2:
+        raise ValueError("inv_freq needs head_dim / 2 entries")
+    arr = (ctypes.c_float * len(freqs))(*freqs)
+    shape = make_shape(b, hq, k.shape[2], d, L, block_size)
+    qo = q if inplace else torch.empty_like(q)
+    ko = k if inplace else torch.empty_like(k)
+    qa = torch.empty_like(q) if want_anchor else None
+    _check(lib().star_attn_rope(ctypes.byref(shape), arr, int(pos0), _ptr(q), _ptr(k), _ptr(qo),
+                                _ptr(ko), _ptr(qa), _stream()), "star_attn_rope")
+    return qo, ko, qa
+
+
+def phase1_anchor_q(q, q_anchor, k, v, block_size: int, scale: Optional[float] = None,
+                    o=None, lse=None, want_lse: bool = True):
+    """Phase 1 whose anchor tiles are scored with q_anchor (anchor-position variant)."""
+    for t, n in ((q, "q"), (q_anchor, "q_anchor"), (k, "k"), (v, "v")):
+        _bf16(t, n, 4)
+    shape = _ctx_shape(q, k, block_size, scale)
+    b, L, hq, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((b, hq, L), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_phase1_anchor_q(ctypes.byref(shape), _ptr(q), _ptr(q_anchor), _ptr(k),
+                                           _ptr(v), _ptr(o), _ptr(lse), _stream()),
+           "star_attn_phase1_anchor_q")
     return o, lse
 
 

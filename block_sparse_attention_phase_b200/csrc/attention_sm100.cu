@@ -76,6 +76,7 @@ struct AttnArgs {
   // Phase 1
   int32_t n_blocks, mt;   // blocks; 128-row q-tiles per block
   int32_t n_anchor;       // 128-column tiles covering the anchor b_0
+  int32_t anchor_q;       // 1: the anchor tiles are scored with a second Q (map tk2)
   __nv_bfloat16* o;       // [b, L, Hq, d]
   float* lse;             // [b, Hq, L] or null
   // Phase-2 query
@@ -95,6 +96,7 @@ struct Bars {
   uint64_t p_full[2];  // per Q tile: P_q(j) written to TMEM
   uint64_t o_bar[2];   // per Q tile: the last O_q += P V complete
   uint64_t drain;
+  uint64_t q_free;     // the last anchor S MMAs are done: Q may be reloaded
   uint32_t tmem_base;
   int abort;
 };
@@ -313,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       mbar_init(&bars->o_bar[s], 1);
     }
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->q_free, 1);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -340,13 +343,25 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(mk);
       tma_prefetch_desc(mv);
-      mbar_arrive_expect_tx(&bars->q_full, 2 * kTileBytes);
+      // Anchor-position variant: the anchor tiles see Q rotated at the anchor
+      // positions (map tk2); after them, Q is reloaded from tq for the own block.
+      bool reload_q = false;
+      const CUtensorMap* mq = &tq;
+      if constexpr (M == Mode::kPhase1) {
+        reload_q = a.anchor_q && it.n_anchor > 0;
+        if (reload_q) mq = &tk2;
+      }
+      auto load_q = [&](const CUtensorMap* map) {
+        mbar_arrive_expect_tx(&bars->q_full, 2 * kTileBytes);
 #pragma unroll
-      for (int q = 0; q < 2; ++q)
+        for (int q = 0; q < 2; ++q)
 #pragma unroll
-        for (int c = 0; c < CH; ++c)
-          tma_load_4d(sq + q * kTileBytes + c * kChunkBytes, &tq, &bars->q_full, c * 64, it.qc1[q],
-                      it.qc2[q], it.bb);
+          for (int c = 0; c < CH; ++c)
+            tma_load_4d(sq + q * kTileBytes + c * kChunkBytes, map, &bars->q_full, c * 64,
+                        it.qc1[q], it.qc2[q], it.bb);
+      };
+      load_q(mq);
+      int q_loads = 1;
       int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j & 1;
@@ -379,10 +394,15 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         for (int c = 0; c < CH; ++c)
           tma_load_4d(sv + s * kTileBytes + c * kChunkBytes, mv, &bars->v_full[s], c * 64, it.kvh, kv0, c3);
         last_v[s] = j;
+        if (reload_q && j == it.n_anchor) {
+          if (!wait_or_abort(&bars->q_free, 0, bars, a.status)) break;
+          load_q(&tq);
+          q_loads = 2;
+        }
       }
       // Every copy this thread issued has landed before the CTA may exit (on the
       // normal path these phases completed long ago).
-      mbar_wait(&bars->q_full, 0, a.status);
+      mbar_wait(&bars->q_full, (q_loads - 1) & 1, a.status);
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
         if (last_k[s] >= 0) mbar_wait(&bars->k_full[s], (last_k[s] >> 1) & 1, a.status);
@@ -396,6 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       const uint32_t sk_addr = smem_u32(sk);
       const uint32_t sv_addr = smem_u32(sv);
       // S_q = Q_q K_j^T: A = Q, B = K, both K-major 128-byte swizzled (16 columns = 32 bytes a step).
+      bool reload_q = false;
+      if constexpr (M == Mode::kPhase1) reload_q = a.anchor_q && it.n_anchor > 0;
       auto issue_s = [&](int q, int j) {
         const uint32_t qa = sq_addr + q * kTileBytes;
         const uint32_t ka = sk_addr + (j & 1) * kTileBytes;
@@ -406,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
                     kIdescQK, kk > 0 ? 1u : 0u);
         }
         tc_commit(&bars->s_full[q]);
+        if (reload_q && q == 1 && j == it.n_anchor - 1) tc_commit(&bars->q_free);
       };
       // O_q += P_q V_j: P from TMEM (bf16 pairs over S_q's columns); V MN-major
       // (d contiguous): 16 kv rows a step, the next 64 columns of d one chunk (LBO)
@@ -437,6 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         if (!more) tc_commit(&bars->o_bar[0]);
         if (more) {
           ok = wait_or_abort(&bars->k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, bars, a.status);
+          // the first own-block tile needs the reloaded Q
+          if (ok && reload_q && j + 1 == it.n_anchor) ok = wait_or_abort(&bars->q_full, 1, bars, a.status);
           if (!ok) break;
           tc_fence_after();
           issue_s(0, j + 1);
@@ -685,6 +710,30 @@ cudaError_t launch_phase1_t(const Shape& s, const void* q, const void* k, const 
   return launch<D, Mode::kPhase1>(a, m, items, vs, st);
 }
 
+template <int D>
+cudaError_t launch_phase1_anchor_q_t(const Shape& s, const void* q, const void* qa, const void* k,
+                                     const void* v, void* o, float* lse, cudaStream_t st) {
+  alignas(64) CUtensorMap m[5];
+  if (!encode_tma_bf16_4d(&m[0], q, D, s.hq, s.L, s.L, s.b, 64, 1, 128, true) ||
+      !encode_tma_bf16_4d(&m[1], k, D, s.hkv, s.L, s.L, s.b, 64, 1, 128, true) ||
+      !encode_tma_bf16_4d(&m[2], v, D, s.hkv, s.L, s.L, s.b, 64, 1, 128, true) ||
+      !encode_tma_bf16_4d(&m[3], qa, D, s.hq, s.L, s.L, s.b, 64, 1, 128, true))
+    return cudaErrorInvalidValue;
+  m[4] = m[2];
+  AttnArgs a = base_args(s);
+  a.n_blocks = static_cast<int32_t>(s.n_blocks());
+  a.mt = static_cast<int32_t>((s.B + 127) / 128);
+  a.n_anchor = a.mt;
+  a.anchor_q = 1;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  const int64_t pairs_per_block = a.G >= 2 ? static_cast<int64_t>(a.mt) * (a.G / 2) : (a.mt + 1) / 2;
+  const int64_t items = static_cast<int64_t>(s.b) * s.hkv * a.n_blocks * pairs_per_block;
+  VarSeqs vs;
+  vs.n = 0;
+  return launch<D, Mode::kPhase1>(a, m, items, vs, st);
+}
+
 // Work items of one Phase-1 sequence of length L (blocks x q-tile pairs x kv-heads).
 int64_t phase1_items(int64_t L, int64_t B, int G, int hkv) {
   if (L <= 0) return 0;
@@ -772,6 +821,13 @@ cudaError_t launch_phase1_sm100(const Shape& s, const void* q, const void* k, co
                                 void* o, float* lse, cudaStream_t st) {
   if (s.d == 128) return launch_phase1_t<128>(s, q, k, v, o, lse, st);
   return launch_phase1_t<64>(s, q, k, v, o, lse, st);
+}
+
+cudaError_t launch_phase1_anchor_q(const Shape& s, const void* q, const void* q_anchor,
+                                   const void* k, const void* v, void* o, float* lse,
+                                   cudaStream_t st) {
+  if (s.d == 128) return launch_phase1_anchor_q_t<128>(s, q, q_anchor, k, v, o, lse, st);
+  return launch_phase1_anchor_q_t<64>(s, q, q_anchor, k, v, o, lse, st);
 }
 
 cudaError_t launch_phase1_varlen(const Shape& s, const int64_t* cu_seqlens, const void* q,

@@ -230,6 +230,39 @@ STAR_ATTN_API star_status_t star_attn_phase1(const star_attn_shape_t* shape, con
       star::launch_phase1_sm100(s, q, k, v, o, lse, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+STAR_ATTN_API star_status_t star_attn_rope(const star_attn_shape_t* shape,
+                                           const float* inv_freq, int64_t pos0, const void* q_in,
+                                           const void* k_in, void* q_out, void* k_out,
+                                           void* q_anchor, star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (!inv_freq || !q_in || !k_in || !q_out || !k_out || pos0 < 0) return STAR_ERR_INVALID_ARG;
+  const void* ptrs[] = {q_in, k_in, q_out, k_out};
+  for (const void* p : ptrs)
+    if (!star::aligned16(p)) return STAR_ERR_INVALID_ARG;
+  if (q_anchor && !star::aligned16(q_anchor)) return STAR_ERR_INVALID_ARG;
+  for (int f = 0; f < s.d / 2; ++f)
+    if (!(inv_freq[f] >= 0.f) || inv_freq[f] > 1e30f) return STAR_ERR_INVALID_ARG;
+  return star::cuda_status(star::launch_rope(s, inv_freq, pos0, q_in, k_in, q_out, k_out, q_anchor,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+STAR_ATTN_API star_status_t star_attn_phase1_anchor_q(const star_attn_shape_t* shape,
+                                                      const void* q, const void* q_anchor,
+                                                      const void* k, const void* v, void* o,
+                                                      float* lse, star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (!q || !q_anchor || !k || !v || !o) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned16(q) || !star::aligned16(q_anchor) || !star::aligned16(k) ||
+      !star::aligned16(v) || !star::aligned16(o) || !star::aligned4(lse))
+    return STAR_ERR_INVALID_ARG;
+  return star::cuda_status(star::launch_phase1_anchor_q(s, q, q_anchor, k, v, o, lse,
+                                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 STAR_ATTN_API star_status_t star_attn_phase1_varlen(const star_attn_shape_t* shape,
                                                     const int64_t* cu_seqlens, const void* q,
                                                     const void* k, const void* v, void* o,

@@ -156,6 +156,15 @@ cudaError_t launch_phase1_varlen(const Shape& s, const int64_t* cu_seqlens, cons
 cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q, int64_t lq,
                               const void* kc, const void* vc, const CacheRef& c, float* o_parts,
                               float* lse_parts, void* o, float* lse, cudaStream_t st);
+// RoPE on q [b, L, Hq, d] and k [b, L, Hkv, d] at positions pos0 + t (in place
+// allowed); q_anchor (or null) gets q rotated at the anchor-variant positions.
+cudaError_t launch_rope(const Shape& s, const float* inv_freq, int64_t pos0, const void* q_in,
+                        const void* k_in, void* q_out, void* k_out, void* q_anchor,
+                        cudaStream_t st);
+// Phase 1 whose anchor tiles are scored with q_anchor instead of q.
+cudaError_t launch_phase1_anchor_q(const Shape& s, const void* q, const void* q_anchor,
+                                   const void* k, const void* v, void* o, float* lse,
+                                   cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t wait_ns, cudaStream_t st);
 cudaError_t launch_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t st);
 

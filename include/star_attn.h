@@ -107,6 +107,38 @@ STAR_ATTN_API star_status_t star_attn_phase1(const star_attn_shape_t* shape, con
                                              star_stream_t stream);
 
 /*
+ * Rotary position embedding of a layer's projected q [batch, L, Hq, d] and
+ * k [batch, L, Hkv, d] (the model step before Phase 1 and Phase 2), at positions
+ * pos0 + t for token t (Phase 1: pos0 = 0; the query tokens: pos0 = L; decode step
+ * n: pos0 = L + Lq + n with L = 1 in the shape). Rotate-half pairs: frequency f <
+ * d/2 rotates (x[f], x[f + d/2]) by the angle position * inv_freq[f].
+ *   inv_freq: HOST float [d/2] (the model's frequencies, scaling included).
+ *   q_out, k_out may equal q_in, k_in (in place).
+ *   q_anchor (or NULL): q rotated at the positions of the anchor-position variant
+ *     of Phase 1 (rebuttal to x5MA, "Anchor Block Content and Position"): the
+ *     anchor tokens of block i >= 1 placed right before the block, at positions
+ *     (i-1)B .. iB-1. RoPE scores depend only on position differences, so this is
+ *     q of token t rotated at t - (i-1)B (block 0: at t); pass it to
+ *     star_attn_phase1_anchor_q(). Uses shape->block_size.
+ */
+STAR_ATTN_API star_status_t star_attn_rope(const star_attn_shape_t* shape,
+                                           const float* inv_freq, int64_t pos0, const void* q_in,
+                                           const void* k_in, void* q_out, void* k_out,
+                                           void* q_anchor, star_stream_t stream);
+
+/*
+ * Phase 1 with the anchor's position IDs moved next to each block: identical to
+ * star_attn_phase1() except that every block i >= 1 scores the anchor's keys with
+ * q_anchor (from star_attn_rope()) instead of q; its own block's keys use q.
+ * The kept K/V (the blocks' caches) are unchanged: the keys stay rotated at
+ * their own positions, as Phase 2 needs.
+ */
+STAR_ATTN_API star_status_t star_attn_phase1_anchor_q(const star_attn_shape_t* shape,
+                                                      const void* q, const void* q_anchor,
+                                                      const void* k, const void* v, void* o,
+                                                      float* lse, star_stream_t stream);
+
+/*
  * Phase 1 over a varlen batch: shape->batch sequences of different lengths,
  * packed back to back along the token axis; each sequence is its own context
  * with its own blocks and its own anchor (its first block), exactly as if it

@@ -38,4 +38,8 @@ from .star_oracle import (  # noqa: F401
     phase2_decode_head,
     phase2_decode,
     phase2_decode_varlen,
+    rope,
+    phase1_rope_head,
+    phase1_rope,
+    model_forward,
 )

@@ -300,3 +300,109 @@ def phase2_decode_varlen(q_t, k_t, v_t, k_ctx, v_ctx, cu_ctx: Sequence[int], k_c
                                        cache_lens[i], scale)
         o[i], lse[i], k_new[i], v_new[i] = oi[0], li[0], ki[0], vi[0]
     return o, lse, k_new, v_new
+
+
+def rope(x, positions: Sequence[int], inv_freq: Sequence[float]):
+    """Rotary position embedding in float64, rotate-half pairs: for x [..., L, H, d]
+    and token positions [L], the pair (x[f], x[f + d/2]) of a token at position p
+    is rotated by the angle p * inv_freq[f]."""
+    x = np.asarray(x, F64)
+    h = x.shape[-1] // 2
+    ang = np.asarray(positions, F64)[:, None] * np.asarray(inv_freq, F64)[None, :]  # [L, d/2]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    a, b = x[..., :h], x[..., h:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+def phase1_rope_head(q_raw, k_raw, v, block_size: int, scale: float, inv_freq,
+                     anchor_positions: str = "original"):
+    """Phase 1 for one head with RoPE applied inside each block's local attention
+    (rebuttal to x5MA, "Anchor Block Content and Position"). q_raw, k_raw [L, d] are
+    the un-rotated projections, v [L, d]. Block tokens keep their own positions;
+    the anchor (b_0's tokens) gets position j ("original") or (i-1)B + j
+    ("adjacent": right before block i) in block i's local context.
+    Returns o [L, d], lse [L]."""
+    L, d = q_raw.shape
+    B = block_size
+    o = np.zeros((L, d), dtype=F64)
+    lse = np.zeros(L, dtype=F64)
+    rot = lambda x, pos: rope(np.asarray(x, F64)[:, None, :], pos, inv_freq)[:, 0]
+    for start, end in block_plan(L, B):
+        i = start // B
+        own = np.arange(start, end)
+        q = rot(q_raw[start:end], own)
+        k_own = rot(k_raw[start:end], own)
+        causal = own[None, :] <= own[:, None]
+        if i == 0:
+            keys, vals, allowed = k_own, np.asarray(v[start:end], F64), causal
+        else:
+            apos = np.arange(B) if anchor_positions == "original" else (i - 1) * B + np.arange(B)
+            keys = np.concatenate([rot(k_raw[:B], apos), k_own])
+            vals = np.concatenate([np.asarray(v[:B], F64), np.asarray(v[start:end], F64)])
+            allowed = np.concatenate([np.ones((end - start, B), dtype=bool), causal], axis=1)
+        o[start:end], lse[start:end] = attend(q, keys, vals, scale, allowed)
+    return o, lse
+
+
+def phase1_rope(q_raw, k_raw, v, block_size: int, inv_freq, anchor_positions: str = "original",
+                scale: float = None):
+    """phase1_rope_head over whole tensors: q_raw [b, L, Hq, d], k_raw, v [b, L, Hkv, d].
+    Returns o [b, L, Hq, d] and lse [b, Hq, L]."""
+    b, L, Hq, d = q_raw.shape
+    Hkv = k_raw.shape[2]
+    scale = default_scale(d) if scale is None else scale
+    o = np.zeros((b, L, Hq, d), dtype=F64)
+    lse = np.zeros((b, Hq, L), dtype=F64)
+    for bi in range(b):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            o[bi, :, h], lse[bi, h] = phase1_rope_head(q_raw[bi, :, h], k_raw[bi, :, g], v[bi, :, g],
+                                                       block_size, scale, inv_freq, anchor_positions)
+    return o, lse
+
+
+def model_forward(x_ctx, x_qry, x_dec: Sequence, w_qkv: Sequence, w_o: Sequence, Hq: int, Hkv: int,
+                  d: int, block_size: int, inv_freq, anchor_positions: str = "original"):
+    """A stack of attention layers driven the Star Attention way, in float64: per
+    layer, q|k|v = x W_qkv, RoPE at the tokens' positions (context 0..L-1, query
+    L.., decode after them), Phase 1 over the context (phase1_rope: the anchor
+    positions as chosen), Phase 2 for the query tokens and then each decode token
+    (every layer keeps its rotated context K/V and its query-local cache), and
+    x += o W_o. x_ctx [b, L, hidden], x_qry [b, Lq, hidden], x_dec: list of
+    [b, 1, hidden]. Returns the hidden states after the last layer for the context,
+    the query and every decode token."""
+    b, L, _ = x_ctx.shape
+    Lq = x_qry.shape[1]
+    T = len(x_dec)
+    qd, kd = Hq * d, Hkv * d
+
+    def split(h, n):
+        h = np.asarray(h, F64)
+        return (h[..., :qd].reshape(b, n, Hq, d), h[..., qd:qd + kd].reshape(b, n, Hkv, d),
+                h[..., qd + kd:].reshape(b, n, Hkv, d))
+
+    xs = [np.asarray(x_ctx, F64), np.asarray(x_qry, F64)] + [np.asarray(t, F64) for t in x_dec]
+    for li in range(len(w_qkv)):
+        W, Wo = np.asarray(w_qkv[li], F64), np.asarray(w_o[li], F64)
+        q, k, v = split(xs[0] @ W, L)
+        o, _ = phase1_rope(q, k, v, block_size, inv_freq, anchor_positions)
+        k_ctx = rope(k, np.arange(L), inv_freq)
+        outs = [o]
+        qq, kq, vq = split(xs[1] @ W, Lq)
+        pos_q = L + np.arange(Lq)
+        qq, kq = rope(qq, pos_q, inv_freq), rope(kq, pos_q, inv_freq)
+        oq, _ = phase2_query(qq, kq, vq, k_ctx, v)
+        outs.append(oq)
+        cap = Lq + T
+        kc = np.zeros((b, cap, Hkv, d))
+        vc = np.zeros((b, cap, Hkv, d))
+        kc[:, :Lq], vc[:, :Lq] = kq, vq
+        for t in range(T):
+            qt, kt, vt = split(xs[2 + t] @ W, 1)
+            pos_t = [L + Lq + t]
+            qt, kt = rope(qt, pos_t, inv_freq), rope(kt, pos_t, inv_freq)
+            ot, _, kc, vc = phase2_decode(qt, kt, vt, k_ctx, v, kc, vc, Lq + t)
+            outs.append(ot)
+        xs = [x + oo.reshape(x.shape[0], x.shape[1], qd) @ Wo for x, oo in zip(xs, outs)]
+    return xs[0], xs[1], xs[2:]

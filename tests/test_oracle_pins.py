@@ -315,12 +315,86 @@ def check_decode_varlen_is_global_per_sequence(seed=10):
         np.testing.assert_array_equal(kn[i], expect_k)
 
 
+def check_rope_is_complex_rotation(seed=11):
+    """RoPE against its complex form: (x_f + i x_{f+d/2}) * exp(i p theta_f), plus
+    identity at position 0 and preserved norms."""
+    rng = np.random.default_rng(seed)
+    L, H, d = 9, 3, 16
+    x = rand(rng, 2, L, H, d)
+    pos = rng.integers(0, 100000, size=L)
+    inv = 10000.0 ** (-2 * np.arange(d // 2) / d)
+    y = oracle.rope(x, pos, inv)
+    z = (x[..., : d // 2] + 1j * x[..., d // 2:]) * np.exp(1j * pos[:, None, None] * inv)
+    np.testing.assert_allclose(y, np.concatenate([z.real, z.imag], axis=-1), atol=1e-9)
+    np.testing.assert_allclose(oracle.rope(x, np.zeros(L), inv), x, atol=0)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-12)
+
+
+def check_anchor_positions(seed=12):
+    """'original' anchor positions = Phase 1 on rotated q, k; 'adjacent' = plain
+    causal attention (SDPA) over [b_0 ; b_i] rotated at positions 0 .. 2B-1, since
+    RoPE scores depend only on position differences; both agree on blocks 0 and 1."""
+    rng = np.random.default_rng(seed)
+    B, L, d = 6, 22, 8
+    q, k, v = rand(rng, L, d), rand(rng, L, d), rand(rng, L, d)
+    inv = 500.0 ** (-2 * np.arange(d // 2) / d)
+    scale = 0.35
+    oo, lo = oracle.phase1_rope_head(q, k, v, B, scale, inv, "original")
+    qr = oracle.rope(q[:, None], np.arange(L), inv)[:, 0]
+    kr = oracle.rope(k[:, None], np.arange(L), inv)[:, 0]
+    ro, rl = oracle.phase1_head(qr, kr, v, B, scale)
+    np.testing.assert_allclose(oo, ro, atol=1e-12)
+    np.testing.assert_allclose(lo, rl, atol=1e-12)
+    oa, la = oracle.phase1_rope_head(q, k, v, B, scale, inv, "adjacent")
+    np.testing.assert_allclose(oa[:2 * B], oo[:2 * B], atol=1e-12)
+    for start, end in oracle.block_plan(L, B)[1:]:
+        seq = np.concatenate([np.arange(B), np.arange(start, end)])
+        qs = oracle.rope(q[seq][:, None], np.arange(len(seq)), inv)[:, 0]
+        ks = oracle.rope(k[seq][:, None], np.arange(len(seq)), inv)[:, 0]
+        n = len(seq)
+        so_, sl_ = sdpa_rows(qs, ks, v[seq], scale, np.tril(np.ones((n, n), dtype=bool)))
+        np.testing.assert_allclose(oa[start:end], so_[B:], atol=1e-9)
+        np.testing.assert_allclose(la[start:end], sl_[B:], atol=1e-9)
+    assert np.abs(oa[2 * B:] - oo[2 * B:]).max() > 1e-6  # the variant does change later blocks
+
+
+def check_model_decode_equals_query(seed=13):
+    """In the layer stack, T decode steps after Lq query tokens give the same hidden
+    states as Lq + T query tokens (a decoded token sees exactly what a query token
+    at its position sees), layer after layer; and 'original' anchors in the stack's
+    Phase 1 equal Phase 1 on the rotated q, k."""
+    rng = np.random.default_rng(seed)
+    b, L, hidden, Hq, Hkv, d, B, Lq, T = 1, 13, 16, 4, 2, 4, 5, 2, 3
+    w_qkv = [rand(rng, hidden, (Hq + 2 * Hkv) * d) / 4 for _ in range(2)]
+    w_o = [rand(rng, Hq * d, hidden) / 4 for _ in range(2)]
+    inv = 100.0 ** (-2 * np.arange(d // 2) / d)
+    xc, xq = rand(rng, b, L, hidden), rand(rng, b, Lq, hidden)
+    xd = [rand(rng, b, 1, hidden) for _ in range(T)]
+    yc, yq, yd = oracle.model_forward(xc, xq, xd, w_qkv, w_o, Hq, Hkv, d, B, inv)
+    yc2, yq2, _ = oracle.model_forward(xc, np.concatenate([xq] + xd, axis=1), [], w_qkv, w_o,
+                                       Hq, Hkv, d, B, inv)
+    np.testing.assert_allclose(yc, yc2, atol=1e-12)
+    np.testing.assert_allclose(yq, yq2[:, :Lq], atol=1e-12)
+    for t in range(T):
+        np.testing.assert_allclose(yd[t][:, 0], yq2[:, Lq + t], atol=1e-12)
+    # first layer's Phase 1 by hand: rotate, then plain Phase 1
+    h = np.asarray(xc) @ w_qkv[0]
+    q = h[..., :Hq * d].reshape(b, L, Hq, d)
+    k = h[..., Hq * d:(Hq + Hkv) * d].reshape(b, L, Hkv, d)
+    v = h[..., (Hq + Hkv) * d:].reshape(b, L, Hkv, d)
+    o, _ = oracle.phase1(oracle.rope(q, np.arange(L), inv), oracle.rope(k, np.arange(L), inv), v, B)
+    y1, _, _ = oracle.model_forward(xc, xq, [], w_qkv[:1], w_o[:1], Hq, Hkv, d, B, inv)
+    np.testing.assert_allclose(y1, xc + o.reshape(b, L, Hq * d) @ w_o[0], atol=1e-12)
+
+
 ALL_CHECKS = [check_single_block_is_causal, check_two_blocks_is_full_causal,
               check_phase1_keysets_golden, check_first_and_last_row_of_block,
               check_block_independence, check_gqa_mapping, check_closed_forms,
               check_phase2_query_is_global, check_phase2_keysets_golden,
               check_merge_split_invariance, check_decode_matches_query_rows,
-              check_phase1_varlen_per_sequence, check_decode_varlen_is_global_per_sequence]
+              check_phase1_varlen_per_sequence, check_decode_varlen_is_global_per_sequence,
+              check_rope_is_complex_rotation, check_anchor_positions,
+              check_model_decode_equals_query]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda c: c.__name__)
@@ -396,7 +470,16 @@ def _mut_decode_varlen_first_len(q_t, k_t, v_t, k_ctx, v_ctx, cu_ctx, k_cache, v
                                [cache_lens[0]] * len(cache_lens), scale)
 
 
+_orig_rope = so.rope
+
+
+def _mut_rope_sign(x, positions, inv_freq):
+    # rotation in the wrong direction
+    return _orig_rope(x, -np.asarray(positions), inv_freq)
+
+
 MUTANTS = {
+    "rope_wrong_direction": ("rope", _mut_rope_sign),
     "varlen_one_context": ("phase1_varlen", _mut_varlen_one_context),
     "decode_varlen_first_len": ("phase2_decode_varlen", _mut_decode_varlen_first_len),
     "anchor_is_previous_block": ("phase1_visible", _mut_anchor_previous),
