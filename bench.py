@@ -54,9 +54,9 @@ def load_peaks():
 # from an ncu capture, with the SHA-256 of the sources the kernel was built from;
 # a figure is reported only while those sources are unchanged.
 KERNEL_SOURCES = {
-    "phase1": ["attention_sm100.cu", "common.cuh"],
-    "decode": ["decode.cu", "common.cuh"],
-    "decode_separate": ["decode.cu", "merge.cu", "common.cuh"],
+    "phase1": ["attention_sm100.cu", "common.cuh", "star_internal.h"],
+    "decode": ["decode.cu", "common.cuh", "star_internal.h"],
+    "decode_separate": ["decode.cu", "merge.cu", "common.cuh", "star_internal.h"],
 }
 
 
@@ -69,15 +69,22 @@ def sources_sha256(kind: str) -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(kind: str, workload: str):
+def recorded_traffic(kind: str, w, algorithmic_bytes: float):
+    """DRAM bytes per launch for this workload: the ncu figure if it was captured on
+    this workload, else the captured workload's bytes per algorithmic byte times
+    this workload's algorithmic bytes (both kernels move each byte once, so their
+    traffic grows in proportion). None when the kernel's sources changed since."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            entry = json.load(f)[workload][kind]
+            entry = json.load(f)[kind]
     except Exception:
-        return None
+        return None, None
     if entry.get("sources_sha256") != sources_sha256(kind):
-        return None
-    return entry.get("dram_bytes_per_launch")
+        return None, "kernel sources changed since the capture"
+    if entry.get("workload") == w.name:
+        return entry["dram_bytes_per_launch"], f"ncu on {w.name}"
+    ratio = entry["dram_bytes_per_launch"] / entry["algorithmic_bytes_per_launch"]
+    return ratio * algorithmic_bytes, f"scaled from the ncu capture on {entry.get('workload')}"
 
 
 # ------------------------------------------------------------------ clocks
@@ -527,12 +534,15 @@ def main(argv=None):
     dec_cold_avg = statistics.mean(cold)
     dec_cold_gbs = statistics.mean(kv_bytes) / (dec_cold_avg / 1e3) / 1e9
 
+    p1_traffic, p1_tsrc = recorded_traffic("phase1", w, w.phase1_io_bytes())
+    dec_traffic, dec_tsrc = recorded_traffic("decode" if fused else "decode_separate", w,
+                                             statistics.mean(kv_bytes))
     rl_p1 = {"bound": "tensor", "kernel": "phase1", "achieved": p1_tflops,
              "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
              "frac": p1_tflops / peaks["bf16_tflops_sustained"],
              "frac_of_burst": p1_tflops / peaks["bf16_tflops"],
              "peak_kind": f"bf16 sustained ({peaks['source']})",
-             "traffic": recorded_traffic("phase1", w.name),
+             "traffic": p1_traffic, "traffic_source": p1_tsrc,
              "algorithmic_per_launch": flops, "avg_launch_ms": p1_avg}
     # Decode: per-step duration inside the timed region (partials + merge, consecutive
     # steps overlapping through programmatic launch); "cold" = one step timed alone
@@ -542,7 +552,7 @@ def main(argv=None):
     rl_dec = {"bound": "hbm", "kernel": dec_kernel, "achieved": dec_gbs,
               "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
               "peak_kind": f"HBM copy ({peaks['source']})",
-              "traffic": recorded_traffic("decode" if fused else "decode_separate", w.name),
+              "traffic": dec_traffic, "traffic_source": dec_tsrc,
               "algorithmic_per_launch": statistics.mean(kv_bytes), "avg_launch_ms": dec_avg,
               "cold_gbs": dec_cold_gbs, "cold_avg_launch_ms": dec_cold_avg,
               "cold_frac": dec_cold_gbs / peaks["hbm_gbs"]}

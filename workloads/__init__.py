@@ -77,6 +77,12 @@ class Workload:
                 pairs += n_i * B
         return 4.0 * self.head_dim * self.num_q_heads * self.batch * pairs
 
+    def phase1_io_bytes(self) -> int:
+        """Bytes Phase 1 must move at least once: Q, K, V read, O and the LSE written."""
+        tok = self.batch * self.ctx_len
+        return tok * self.head_dim * 2 * (2 * self.num_q_heads + 2 * self.num_kv_heads) + \
+            tok * self.num_q_heads * 4
+
     def decode_kv_bytes(self, step: int) -> int:
         """KV bytes a decode step must read once: context + query tokens + decoded
         tokens so far (including the one appended this step), K and V, bf16."""
