@@ -78,13 +78,19 @@ constexpr bool kIsVarlen = sizeof(VL) == sizeof(DecVarlen);
 struct Split {
   int bb, kvh, split, n_splits;
   bool is_cache;
-  int64_t k0, k1;         // key range: context tokens of the sequence, or cache rows
+  int32_t k0, k1;           // key range: context tokens of the sequence, or cache rows
   int32_t ctx_tok, ctx_c3;  // context-map coordinate offset (packed varlen) and outer coordinate
-  int64_t cache_len;
-  int64_t prow;           // partial row (in units of Hq rows) of this split
-  int64_t prow0, pstride; // partial row of the sequence's split 0; step between splits
-  int ctr;                // fused-merge counter of (sequence, kv-head)
+  int32_t cache_len;
 };
+
+// Partial row (in units of Hq rows) of split s of the CTA's sequence: [S, b] for a
+// uniform batch, the sequence's own run of rows for a varlen one.
+template <class VL>
+__device__ __forceinline__ int64_t part_row(const DecodeArgs& a, const VL& dv, const Split& w,
+                                            int s) {
+  if constexpr (kIsVarlen<VL>) return static_cast<int64_t>(dv.split0[w.bb]) + s;
+  else return static_cast<int64_t>(s) * a.b + w.bb;
+}
 
 // A uniform batch needs no table: its launches carry this instead of DecVarlen.
 struct NoVarlen {
@@ -101,13 +107,9 @@ __device__ __forceinline__ Split locate(const DecodeArgs& a, const VL& dv) {
     w.bb = blockIdx.y / a.hkv;
     w.kvh = blockIdx.y % a.hkv;
     w.n_splits = gridDim.x;
-    w.cache_len = a.cache_len;
+    w.cache_len = static_cast<int32_t>(a.cache_len);
     w.ctx_tok = 0;
     w.ctx_c3 = w.bb;
-    w.prow = static_cast<int64_t>(w.split) * a.b + w.bb;
-    w.prow0 = w.bb;
-    w.pstride = a.b;
-    w.ctr = blockIdx.y;
   } else {
     const int r0 = blockIdx.x;
     int lo = 0, hi = dv.n;
@@ -128,10 +130,6 @@ __device__ __forceinline__ Split locate(const DecodeArgs& a, const VL& dv) {
     w.cache_len = dv.cache_len[lo];
     w.ctx_tok = dv.ctx0[lo];
     w.ctx_c3 = 0;
-    w.prow = dv.split0[lo] + w.split;
-    w.prow0 = dv.split0[lo];
-    w.pstride = 1;
-    w.ctr = lo * a.hkv + w.kvh;
   }
   w.is_cache = w.split == n_ctx;
   if (!w.is_cache) {
@@ -139,8 +137,9 @@ __device__ __forceinline__ Split locate(const DecodeArgs& a, const VL& dv) {
     const int64_t sub = w.split % spb;
     const int64_t bstart = blk * B;
     const int64_t bend = min(L, bstart + B);
-    w.k0 = min(bend, bstart + sub * chunk);
-    w.k1 = min(bend, w.k0 + chunk);
+    const int64_t k0 = min(bend, bstart + sub * chunk);
+    w.k0 = static_cast<int32_t>(k0);
+    w.k1 = static_cast<int32_t>(min(bend, k0 + chunk));
   } else {
     w.k0 = 0;
     w.k1 = w.cache_len + 1;  // the cached rows and the new token, appended by the CTA
@@ -160,8 +159,9 @@ __device__ __forceinline__ Split locate(const DecodeArgs& a, const VL& dv) {
 // then the 4 warps take the splits in turn (warp w: splits w, w + 4, ...), each
 // lane owning float4 columns of the split's contiguous G x D partial block, with
 // several splits' loads in flight; the warps' sums meet in shared memory.
-template <int D, int G>
-__device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const Split& w, uint8_t* smem) {
+template <int D, int G, class VL>
+__device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const VL& dv, const Split& w,
+                                              uint8_t* smem) {
   __shared__ int s_last;
   __shared__ float s_red[kWarps][G];
   __shared__ float s_m[G], s_w[G];
@@ -169,7 +169,7 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const Split& 
   asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
   const int tid = threadIdx.x;  // 0 .. 127 (the consumer warps)
   if (tid == 0) {
-    uint32_t* ctr = a.counters + w.ctr;
+    uint32_t* ctr = a.counters + (static_cast<int64_t>(w.bb) * a.hkv + w.kvh);
     const uint32_t prev = atomicAdd(ctr, 1u);
     const int last = prev == static_cast<uint32_t>(w.n_splits - 1);
     if (last) atomicExch(ctr, 0u);  // every split of this launch has counted
@@ -182,8 +182,8 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const Split& 
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int S = w.n_splits;
-  const int64_t row0 = w.prow0 * a.hq + w.kvh * G;  // partial row: split 0, first head
-  const int64_t stride = w.pstride * a.hq;         // rows between splits
+  const int64_t row0 = part_row(a, dv, w, 0) * a.hq + w.kvh * G;  // split 0, first head
+  const int64_t stride = (part_row(a, dv, w, 1) - part_row(a, dv, w, 0)) * a.hq;  // between splits
   const int64_t orow0 = static_cast<int64_t>(w.bb) * a.hq + w.kvh * G;  // output row
   float* wts = reinterpret_cast<float*>(smem);                     // [S][G]
   float4* red = reinterpret_cast<float4*>(smem + fused_weights_bytes(S, G));  // [kWarps][G*D/4]
@@ -572,14 +572,14 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
         }
       }
       const int hq = kvh * G + h;
-      const int64_t row = w.prow;
+      const int64_t row = part_row(a, dv, w, w.split);
       a.o_parts[(row * a.hq + hq) * D + e] = lsum > 0.f ? acc / lsum : 0.f;
       if (e == 0) {
         a.lse_parts[row * a.hq + hq] =
             lsum > 0.f ? (M * sl2 + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
       }
     }
-    if (a.counters) merge_if_last<D, G>(a, w, base);
+    if (a.counters) merge_if_last<D, G>(a, dv, w, base);
   }
 }
 
