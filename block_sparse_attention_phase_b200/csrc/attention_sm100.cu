@@ -47,17 +47,27 @@
 namespace star {
 namespace {
 
-constexpr int kThreads = 384;
+// Threads per softmax row: 1 (a warpgroup per Q tile) or 2 (two warpgroups per Q
+// tile, each owning 64 of a row's 128 scores and d/2 of its output columns; the
+// two halves of a row trade their partial maxima through shared memory).
+#ifndef STAR_SOFTMAX_HALVES
+#define STAR_SOFTMAX_HALVES 1
+#endif
+constexpr int kHalves = STAR_SOFTMAX_HALVES;
+static_assert(kHalves == 1 || kHalves == 2, "one or two threads per softmax row");
+constexpr int kThreads = 128 * (1 + 2 * kHalves);
 constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle row each)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;          // lazy-rescale threshold (log2 units)
-// Register split: 384 threads launch with 168 registers each (64512); warpgroup 0
-// gives back down to 104, the two softmax warpgroups take 200: 128*104 + 256*200 = 64512
-// (the split with the least spilling in either region).
-constexpr int kLaunchRegs = 168;
-constexpr int kRegsLow = 104;
-constexpr int kRegsHigh = 200;
-static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
+// Register split. One thread per row: 384 threads launch with 168 registers
+// (64512); warpgroup 0 gives back down to 104, the two softmax warpgroups take 200.
+// Two per row: 640 threads launch with 96 (61440); warpgroup 0 drops to 56 and the
+// four softmax warpgroups take 104.
+constexpr int kLaunchRegs = kHalves == 1 ? 168 : 96;
+constexpr int kRegsLow = kHalves == 1 ? 104 : 56;
+constexpr int kRegsHigh = kHalves == 1 ? 200 : 104;
+static_assert(128 * kRegsLow + 256 * kHalves * kRegsHigh <= kThreads * kLaunchRegs, "register split");
+static_assert(kThreads * kLaunchRegs <= 65536, "register file");
 // Of every 8 pairs of scores, this many take the FMA-pipe exponential; the MUFU
 // (16 results per clock per SM) would otherwise pace the softmax at the same
 // rate as the tensor core's MMAs.
@@ -97,8 +107,11 @@ struct Bars {
   uint64_t o_bar[2];   // per Q tile: the last O_q += P V complete
   uint64_t drain;
   uint64_t q_free;     // the last anchor S MMAs are done: Q may be reloaded
+  uint64_t xchg[2][4]; // per Q tile and TMEM lane quarter: both halves posted a value
   uint32_t tmem_base;
   int abort;
+  float pmax[2][2][2][128];  // [tile][step parity][half][row] partial row maxima
+  float psum[2][2][128];     // [tile][half][row] partial row sums at the end
 };
 
 // What one CTA computes.
@@ -311,7 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], 128);
+      mbar_init(&bars->p_full[s], 128 * kHalves);
+#pragma unroll
+      for (int w4 = 0; w4 < 4; ++w4) mbar_init(&bars->xchg[s][w4], 64);
       mbar_init(&bars->o_bar[s], 1);
     }
     mbar_init(&bars->drain, 1);
@@ -484,12 +499,19 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
   } else {
     // ------------------------------------------------------------ softmax warpgroups
     setmaxnreg_inc<kRegsHigh>();
-    const int q = wg - 1;  // the Q tile this warpgroup owns
+    const int sw = wg - 1;
+    const int q = sw / kHalves;   // the Q tile this warpgroup works on
+    const int hf = sw % kHalves;  // which half of each row (with two threads per row)
+    constexpr int kCols = 128 / kHalves;  // scores per thread and tile
+    constexpr int kChunks = kCols / 32;
+    constexpr int kOCols = D / kHalves;   // output columns per thread
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    const uint32_t s_col = q * 128;
-    const uint32_t o_col = 256 + q * D;
+    const uint32_t s_col = q * 128 + hf * kCols;     // this thread's scores
+    const uint32_t p_col = q * 128 + hf * kCols / 2; // its bf16 pairs of P
+    const uint32_t o_col = 256 + q * D + hf * kOCols;
+    uint64_t* xbar = &bars->xchg[q][q4];
     // This tile's scalars (selected, so that Item stays in registers).
     int64_t row_tok;  // Phase 1: context position of this row; query: query-token index
     int head, rows_valid;
@@ -512,20 +534,22 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       ok = __all_sync(0xffffffffu, wait_or_abort(&bars->s_full[q], j & 1, bars, a.status));
       if (!ok) break;
       tc_fence_after();
-      const int limit = visible_prefix<M>(it, a, row_tok, j);
+      const int limit = visible_prefix<M>(it, a, row_tok, j) - hf * kCols;  // in this half
       // Most tiles are fully visible: mask only when some row of the warp needs it.
-      const bool masked = __any_sync(0xffffffffu, limit < 128);
-      // S in two halves: the max over the first 64 scores overlaps the TMEM read
-      // of the second 64. Row max with independent 3-input max chains.
-      uint32_t sr[4][32];
-      float mc[4];
+      const bool masked = __any_sync(0xffffffffu, limit < kCols);
+      // S in pieces of 32: the max over the first pieces overlaps the TMEM read of
+      // the later ones. Row max with independent 3-input max chains.
+      uint32_t sr[kChunks][32];
+      float mc[kChunks];
       tmem_ld32(lane_addr + s_col, sr[0]);
       tmem_ld32(lane_addr + s_col + 32, sr[1]);
       tmem_wait_ld();
-      tmem_ld32(lane_addr + s_col + 64, sr[2]);
-      tmem_ld32(lane_addr + s_col + 96, sr[3]);
+      if constexpr (kChunks == 4) {
+        tmem_ld32(lane_addr + s_col + 64, sr[2 % kChunks]);
+        tmem_ld32(lane_addr + s_col + 96, sr[3 % kChunks]);
+      }
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < kChunks / 2; ++half) {
         if (half == 1) tmem_wait_ld();
 #pragma unroll
         for (int c = 2 * half; c < 2 * half + 2; ++c) {
@@ -540,7 +564,18 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
             mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
         }
       }
-      const float mt = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
+      float mt = fmaxf(mc[0], mc[1]);
+      if constexpr (kChunks == 4) mt = fmaxf(mt, fmaxf(mc[2 % kChunks], mc[3 % kChunks]));
+      if constexpr (kHalves == 2) {
+        // Trade partial maxima with the other half of the row. Both halves have
+        // their scores in registers before either arrives, so P (which the halves
+        // write over S's first 64 columns) cannot overwrite unread scores.
+        bars->pmax[q][j & 1][hf][row] = mt;
+        mbar_arrive(xbar);
+        ok = __all_sync(0xffffffffu, wait_or_abort(xbar, j & 1, bars, a.status));
+        if (!ok) break;
+        mt = fmaxf(mt, bars->pmax[q][j & 1][hf ^ 1][row]);
+      }
       const bool need = (m_run == -INFINITY) || ((mt - m_run) * sl2 > kRescaleLog2);
       const float m_new = need ? mt : m_run;
       const float m_use = m_new == -INFINITY ? 0.f : m_new;  // a row with nothing visible yet
@@ -552,9 +587,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       const float2 nms = make_float2(-ms, -ms);
       float2 ps[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        // Chunk c (32 scores) -> 16 bf16 pairs, stored to TMEM columns [16c, 16c+16)
-        // at once (S is all in registers already), so few P words are ever live.
+      for (int c = 0; c < kChunks; ++c) {
+        // Chunk c (32 scores) -> 16 bf16 pairs, stored to TMEM at once (S is all
+        // in registers already), so few P words are ever live.
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -573,14 +608,14 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
           ps[(e >> 1) & 1] = fadd2(ps[(e >> 1) & 1], make_float2(p0, p1));
           pk[e / 2] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(lane_addr + s_col + c * 16, pk);
+        tmem_st16(lane_addr + p_col + c * 16, pk);
       }
       const float psum = (ps[0].x + ps[0].y) + (ps[1].x + ps[1].y);
       l_run = l_run * alpha + psum;
       // S_q(j) complete implies O_q += P_q(j-1) V complete: O may be rescaled now.
       if (j >= 1 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < kOCols / 32; ++c) {
           uint32_t ob[32];
           tmem_ld32(lane_addr + o_col + c * 32, ob);
           tmem_wait_ld();
@@ -593,6 +628,15 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       tc_fence_before();
       mbar_arrive(&bars->p_full[q]);
     }
+    if constexpr (kHalves == 2) {
+      // The row sum is the two halves' sums (same running max in both).
+      if (ok) {
+        bars->psum[q][hf][row] = l_run;
+        mbar_arrive(xbar);
+        ok = __all_sync(0xffffffffu, wait_or_abort(xbar, n_tiles & 1, bars, a.status));
+        if (ok) l_run += bars->psum[q][hf ^ 1][row];
+      }
+    }
     if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&bars->o_bar[q], 0, bars, a.status));
     tc_fence_after();
     if (ok) {
@@ -603,9 +647,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         const int64_t t = row_tok;
         const bool valid = row < rows_valid;
         // uniform: row bb * L + t of [b, L, Hq, d]; varlen: row tok_base + t of [total, Hq, d]
-        __nv_bfloat16* dst = a.o + ((static_cast<int64_t>(it.bb) * a.L + it.tok_base + t) * a.hq + head) * D;
+        __nv_bfloat16* dst = a.o + ((static_cast<int64_t>(it.bb) * a.L + it.tok_base + t) * a.hq + head) * D +
+                             hf * kOCols;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < kOCols / 32; ++c) {
           uint32_t ob[32];
           tmem_ld32(lane_addr + o_col + c * 32, ob);
           tmem_wait_ld();
@@ -620,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
               d4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
           }
         }
-        if (a.lse && valid)
+        if (a.lse && valid && hf == 0)
           a.lse[(static_cast<int64_t>(it.bb) * a.hq + head) * a.L + it.tok_base + t] =
               lse2 * 0.69314718055994531f;
       } else {
@@ -628,9 +673,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         const int hq = head;
         const bool valid = tok < a.lq;
         const int64_t prow = static_cast<int64_t>(it.split) * a.b + it.bb;
-        float* dst = a.o_parts + ((prow * a.lq + tok) * a.hq + hq) * D;
+        float* dst = a.o_parts + ((prow * a.lq + tok) * a.hq + hq) * D + hf * kOCols;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < kOCols / 32; ++c) {
           uint32_t ob[32];
           tmem_ld32(lane_addr + o_col + c * 32, ob);
           tmem_wait_ld();
@@ -642,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
                                   __uint_as_float(ob[4 * u + 2]) * inv, __uint_as_float(ob[4 * u + 3]) * inv);
           }
         }
-        if (valid) a.lse_parts[(prow * a.hq + hq) * a.lq + tok] = lse2 * 0.69314718055994531f;
+        if (valid && hf == 0) a.lse_parts[(prow * a.hq + hq) * a.lq + tok] = lse2 * 0.69314718055994531f;
       }
     }
   }

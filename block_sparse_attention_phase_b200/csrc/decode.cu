@@ -210,7 +210,7 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const VL& dv,
   if (tid < G) {
     float mm = s_red[0][tid];
 #pragma unroll
-    for (int w = 1; w < kWarps; ++w) mm = fmaxf(mm, s_red[w][tid]);
+    for (int wi = 1; wi < kWarps; ++wi) mm = fmaxf(mm, s_red[wi][tid]);
     s_m[tid] = mm;
   }
   asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
@@ -269,7 +269,7 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const VL& dv,
   if (tid < G) {
     float W = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) W += s_red[w][tid];
+    for (int wi = 0; wi < kWarps; ++wi) W += s_red[wi][tid];
     s_w[tid] = W;
     if (a.lse) a.lse[orow0 + tid] = W > 0.f ? s_m[tid] + logf(W) : -INFINITY;
   }
@@ -277,8 +277,8 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const VL& dv,
   for (int f = tid; f < F; f += kWarps * 32) {
     float4 x = red[f];
 #pragma unroll
-    for (int w = 1; w < kWarps; ++w) {
-      const float4 y = red[w * F + f];
+    for (int wi = 1; wi < kWarps; ++wi) {
+      const float4 y = red[wi * F + f];
       x.x += y.x;
       x.y += y.y;
       x.z += y.z;
@@ -561,14 +561,14 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
       const int e = idx % D;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, cm[w * G + h]);
+      for (int wi = 0; wi < kWarps; ++wi) M = fmaxf(M, cm[wi * G + h]);
       float lsum = 0.f, acc = 0.f;
       if (M != -INFINITY) {
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-          const float sc = ex2_approx((cm[w * G + h] - M) * sl2);
-          lsum += cl[w * G + h] * sc;
-          acc += cacc[(w * G + h) * D + e] * sc;
+        for (int wi = 0; wi < kWarps; ++wi) {
+          const float sc = ex2_approx((cm[wi * G + h] - M) * sl2);
+          lsum += cl[wi * G + h] * sc;
+          acc += cacc[(wi * G + h) * D + e] * sc;
         }
       }
       const int hq = kvh * G + h;
