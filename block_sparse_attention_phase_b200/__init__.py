@@ -37,6 +37,7 @@ EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase1_v
             "star_attn_phase2_query",
             "star_attn_phase2_decode", "star_attn_phase2_decode_fused",
             "star_attn_phase2_decode_varlen", "star_attn_decode_varlen_workspace_bytes",
+            "star_attn_phase2_query_varlen", "star_attn_query_varlen_workspace_bytes",
             "star_attn_phase2_query_paged",
             "star_attn_phase2_decode_paged", "star_attn_phase2_decode_noalloc",
             "star_attn_lse_merge", "star_attn_simple_phase1",
@@ -86,6 +87,11 @@ def lib() -> ctypes.CDLL:
                                                   P, P, P, P, P, P, P, I64, P, I32, I32, I32,
                                                   P, P, P, SZ, P]),
         "star_attn_decode_varlen_workspace_bytes": (SZ, [SP, ctypes.POINTER(I64)]),
+        "star_attn_phase2_query_varlen": (I32, [SP, ctypes.POINTER(I64), ctypes.POINTER(I64),
+                                                 P, P, P, P, P, P, P, I64, P, I32, I32, I32,
+                                                 P, P, P, SZ, P]),
+        "star_attn_query_varlen_workspace_bytes": (SZ, [SP, ctypes.POINTER(I64),
+                                                        ctypes.POINTER(I64)]),
         "star_attn_phase2_query_paged": (I32, [SP, P, P, P, I64, P, P, P, P, I32, I32, P, I32,
                                                 P, P, P, SZ, P]),
         "star_attn_phase2_decode_paged": (I32, [SP, P, P, P, P, P, P, P, I32, I32, P, I32, I64,
@@ -372,6 +378,48 @@ def phase2_decode_fused(q, k, v, k_ctx, v_ctx, k_cache, v_cache, cache_len: int,
         ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_cache),
         _ptr(v_cache), int(cache_len), k_cache.shape[1], _ptr(o), _ptr(lse), _ptr(workspace),
         workspace.numel(), _stream()), "star_attn_phase2_decode_fused")
+    return o, lse
+
+
+def phase2_query_varlen(q, k, v, k_ctx, v_ctx, cu_ctx, cu_q, k_cache, v_cache,
+                        block_size: int, page_table=None, scale: Optional[float] = None,
+                        o=None, lse=None, workspace=None):
+    """Phase-2 query pass for sequences with their own context and query lengths:
+    q [total_q, Hq, d], k/v [total_q, Hkv, d] packed with host offsets cu_q [b + 1];
+    contexts k_ctx/v_ctx [total_ctx, Hkv, d] with cu_ctx [b + 1]; caches [b, cap, Hkv, d]
+    (or page pools with page_table [b, max_pages]). Returns (o [total_q, Hq, d],
+    lse [Hq, total_q])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (k_ctx, "k_ctx"), (v_ctx, "v_ctx")):
+        _bf16(t, n, 3)
+    cc, cvals = _cu_array(cu_ctx)
+    cq, qvals = _cu_array(cu_q)
+    b = len(cvals) - 1
+    if len(qvals) != b + 1:
+        raise ValueError("cu_ctx and cu_q need the same number of sequences")
+    total_q, hq, d = q.shape
+    shape = make_shape(b, hq, k_ctx.shape[1], d, cvals[-1], block_size, scale)
+    if workspace is None:
+        need = int(lib().star_attn_query_varlen_workspace_bytes(ctypes.byref(shape), cc, cq))
+        if need == 0:
+            raise ValueError("unsupported shape or offsets")
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if page_table is not None:
+        page_size, num_pages, max_pages = _page_pool(k_cache, v_cache, page_table)
+        cap = 0
+    else:
+        _bf16(k_cache, "k_cache", 4)
+        _bf16(v_cache, "v_cache", 4)
+        page_size = num_pages = max_pages = 0
+        cap = k_cache.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((hq, total_q), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_phase2_query_varlen(
+        ctypes.byref(shape), cc, cq, _ptr(q), _ptr(k), _ptr(v), _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(k_cache), _ptr(v_cache), cap, _ptr(page_table), page_size, num_pages, max_pages,
+        _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(), _stream()),
+        "star_attn_phase2_query_varlen")
     return o, lse
 
 

@@ -128,6 +128,10 @@ struct Item {
   int split, tok0[2];
   bool cache;
   int64_t k0, k1;
+  int32_t lq;          // this sequence's query tokens
+  int32_t q_c3;        // outer Q coordinate: the sequence, or 0 for packed queries
+  int32_t ctx_tok, ctx_c3;  // context coordinates: packed offset and outer coordinate
+  int64_t rbase;       // partial token-row of (this split, token 0)
 };
 
 template <Mode M>
@@ -198,32 +202,68 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, const VarSeqs& vs
       it.qc2[q] = static_cast<int32_t>(it.tok_base + it.t0[q]);
     }
   } else {
-    const int npair = (a.n_qt + 1) / 2;
+    int n_qt = a.n_qt, n_splits = a.n_splits, n_ctx = a.n_ctx, spb = a.spb;
+    int64_t chunk = a.chunk;
+    it.lq = static_cast<int32_t>(a.lq);
+    int32_t qbase = 0;
+    int lo = 0;
+    if (vs.n > 0) {
+      // Varlen batch: the sequence that owns this item, then its own split plan
+      // (packed queries and context; per-sequence caches).
+      int hi = vs.n;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (vs.item0[mid] <= r) lo = mid; else hi = mid;
+      }
+      r -= vs.item0[lo];
+      it.lq = vs.start[lo + 1] - vs.start[lo];
+      qbase = vs.start[lo];
+      it.L = vs.ctx0[lo + 1] - vs.ctx0[lo];
+      it.B = min(a.B, it.L);
+      spb = vs.spb[lo];
+      n_ctx = it.L > 0 ? static_cast<int>((it.L + it.B - 1) / it.B) * spb : 0;
+      n_splits = n_ctx + 1;
+      chunk = it.L > 0 ? (it.B + spb - 1) / spb : 1;
+      n_qt = (it.lq * a.G + 127) / 128;
+    }
+    const int npair = (n_qt + 1) / 2;
     const int qp = static_cast<int>(r % npair);
     r /= npair;
-    it.split = static_cast<int>(r % a.n_splits);
-    r /= a.n_splits;
+    it.split = static_cast<int>(r % n_splits);
+    r /= n_splits;
     it.kvh = static_cast<int>(r % a.hkv);
-    it.bb = static_cast<int>(r / a.hkv);
+    if (vs.n > 0) {
+      it.bb = lo;
+      it.q_c3 = 0;
+      it.ctx_tok = vs.ctx0[lo];
+      it.ctx_c3 = 0;
+      it.rbase = static_cast<int64_t>(vs.rbase[lo]) + static_cast<int64_t>(it.split) * it.lq;
+    } else {
+      it.bb = static_cast<int>(r / a.hkv);
+      it.q_c3 = it.bb;
+      it.ctx_tok = 0;
+      it.ctx_c3 = it.bb;
+      it.rbase = (static_cast<int64_t>(it.split) * a.b + it.bb) * it.lq;
+    }
     it.tok0[0] = 2 * qp * (128 / a.G);
     it.tok0[1] = it.tok0[0] + 128 / a.G;  // may lie past Lq: zero rows, never stored
-    it.cache = it.split == a.n_ctx;
+    it.cache = it.split == n_ctx;
     if (!it.cache) {
-      const int64_t blk = it.split / a.spb;
-      const int64_t sub = it.split % a.spb;
-      const int64_t bs = blk * a.B;
-      const int64_t be = min(a.L, bs + a.B);
-      it.k0 = min(be, bs + sub * a.chunk);
-      it.k1 = min(be, it.k0 + a.chunk);
+      const int64_t blk = it.split / spb;
+      const int64_t sub = it.split % spb;
+      const int64_t bs = blk * it.B;
+      const int64_t be = min(it.L, bs + it.B);
+      it.k0 = min(be, bs + sub * chunk);
+      it.k1 = min(be, it.k0 + chunk);
     } else {
       it.k0 = 0;
-      it.k1 = a.lq;
+      it.k1 = it.lq;
     }
     it.n_tiles = static_cast<int>((it.k1 - it.k0 + 127) / 128);
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       it.qc1[q] = it.kvh * a.G;
-      it.qc2[q] = it.tok0[q];
+      it.qc2[q] = qbase + it.tok0[q];
     }
   }
   return it;
@@ -300,11 +340,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       for (int idx = threadIdx.x; idx < 256 * D; idx += kThreads) {
         const int row = idx / D, e = idx % D;
         const int tok = it.tok0[row >> 7] + (row & 127) / a.G;
-        if (tok >= a.lq) continue;
+        if (tok >= it.lq) continue;
         const int hq = it.kvh * a.G + (row & 127) % a.G;
-        const int64_t prow = static_cast<int64_t>(it.split) * a.b + it.bb;
-        a.o_parts[((prow * a.lq + tok) * a.hq + hq) * D + e] = 0.f;
-        if (e == 0) a.lse_parts[(prow * a.hq + hq) * a.lq + tok] = -INFINITY;
+        a.o_parts[((it.rbase + tok) * a.hq + hq) * D + e] = 0.f;
+        if (e == 0) a.lse_parts[it.rbase * a.hq + static_cast<int64_t>(hq) * it.lq + tok] = -INFINITY;
       }
     }
     return;  // before any barrier or TMEM allocation
@@ -373,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
 #pragma unroll
           for (int c = 0; c < CH; ++c)
             tma_load_4d(sq + q * kTileBytes + c * kChunkBytes, map, &bars->q_full, c * 64,
-                        it.qc1[q], it.qc2[q], it.bb);
+                        it.qc1[q], it.qc2[q], M == Mode::kQuery ? it.q_c3 : it.bb);
       };
       load_q(mq);
       int q_loads = 1;
@@ -392,7 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         // this 128-row tile (page sizes are multiples of 128).
         int32_t c3 = it.bb;
         if constexpr (M == Mode::kQuery) {
-          if (it.cache && a.page_table) {
+          if (!it.cache) {
+            kv0 += it.ctx_tok;
+            c3 = it.ctx_c3;
+          } else if (a.page_table) {
             c3 = a.page_table[static_cast<int64_t>(it.bb) * a.max_pages + kv0 / a.page_size];
             kv0 %= a.page_size;
           }
@@ -671,9 +713,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       } else {
         const int tok = static_cast<int>(row_tok);
         const int hq = head;
-        const bool valid = tok < a.lq;
-        const int64_t prow = static_cast<int64_t>(it.split) * a.b + it.bb;
-        float* dst = a.o_parts + ((prow * a.lq + tok) * a.hq + hq) * D + hf * kOCols;
+        const bool valid = tok < it.lq;
+        float* dst = a.o_parts + ((it.rbase + tok) * a.hq + hq) * D + hf * kOCols;
 #pragma unroll
         for (int c = 0; c < kOCols / 32; ++c) {
           uint32_t ob[32];
@@ -687,7 +728,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
                                   __uint_as_float(ob[4 * u + 2]) * inv, __uint_as_float(ob[4 * u + 3]) * inv);
           }
         }
-        if (valid && hf == 0) a.lse_parts[(prow * a.hq + hq) * a.lq + tok] = lse2 * 0.69314718055994531f;
+        if (valid && hf == 0)
+          a.lse_parts[it.rbase * a.hq + static_cast<int64_t>(hq) * it.lq + tok] = lse2 * 0.69314718055994531f;
       }
     }
   }
@@ -858,9 +900,92 @@ cudaError_t launch_query_t(const Shape& s, const SplitPlan& p, const void* q, in
   return launch<D, Mode::kQuery>(a, m, items, vs, st);
 }
 
+template <int D>
+cudaError_t launch_query_varlen_t(const Shape& s, const VarSeqs& vs, const void* q,
+                                  const void* kc, const void* vc, const CacheRef& c,
+                                  float* o_parts, float* lse_parts, cudaStream_t st) {
+  const int G = s.group();
+  const uint64_t total_q = static_cast<uint64_t>(vs.start[vs.n]);
+  const uint64_t total_ctx = static_cast<uint64_t>(vs.ctx0[vs.n]);
+  alignas(64) CUtensorMap m[5];
+  bool ok = encode_tma_bf16_4d(&m[0], q, D, s.hq, total_q, total_q, 1, 64, G, 128 / G, true) &&
+            encode_tma_bf16_4d(&m[1], kc, D, s.hkv, total_ctx, total_ctx, 1, 64, 1, 128, true) &&
+            encode_tma_bf16_4d(&m[2], vc, D, s.hkv, total_ctx, total_ctx, 1, 64, 1, 128, true);
+  if (c.paged()) {
+    ok = ok &&
+         encode_tma_bf16_4d(&m[3], c.k, D, s.hkv, c.page_size, c.page_size, c.num_pages, 64, 1, 128, true) &&
+         encode_tma_bf16_4d(&m[4], c.v, D, s.hkv, c.page_size, c.page_size, c.num_pages, 64, 1, 128, true);
+  } else {
+    // every row of a sequence's cache is in bounds; the varlen cache write zeroed
+    // the rows past its query rows up to the end of their 128-row tile
+    ok = ok && encode_tma_bf16_4d(&m[3], c.k, D, s.hkv, c.cap, c.cap, s.b, 64, 1, 128, true) &&
+         encode_tma_bf16_4d(&m[4], c.v, D, s.hkv, c.cap, c.cap, s.b, 64, 1, 128, true);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  AttnArgs a = base_args(s);
+  a.page_table = c.page_table;
+  a.page_size = c.page_size;
+  a.max_pages = c.max_pages;
+  a.o_parts = o_parts;
+  a.lse_parts = lse_parts;
+  return launch<D, Mode::kQuery>(a, m, vs.item0[vs.n], vs, st);
+}
+
 }  // namespace
 
 int64_t query_tiles(const Shape& s, int64_t lq) { return (lq * s.group() + 127) / 128; }
+
+int64_t plan_query_varlen(const Shape& s, const int64_t* cu_ctx, const int64_t* cu_q,
+                          int64_t target_ctas, VarSeqs* vs) {
+  // One chunk size for the batch, chosen so that all items (q-tile pairs x splits
+  // x kv-heads) come to about target_ctas.
+  int64_t work = 0, cache_items = 0;
+  for (int i = 0; i < s.b; ++i) {
+    const int64_t pairs = ((cu_q[i + 1] - cu_q[i]) * s.group() + 255) / 256;
+    work += pairs * (cu_ctx[i + 1] - cu_ctx[i]) * s.hkv;
+    cache_items += pairs * s.hkv;
+  }
+  const int64_t ctx_items = target_ctas - cache_items;
+  int64_t C = ctx_items > 0 ? (work + ctx_items - 1) / ctx_items : work;
+  if (C < 128) C = 128;
+  vs->n = s.b;
+  int64_t items = 0, rows = 0;
+  for (int i = 0; i < s.b; ++i) {
+    const int64_t L = cu_ctx[i + 1] - cu_ctx[i];
+    const int64_t lq = cu_q[i + 1] - cu_q[i];
+    int64_t spb = 1, n_ctx = 0;
+    if (L > 0) {
+      const int64_t B = s.B < L ? s.B : L;
+      spb = (B + C - 1) / C;
+      n_ctx = (L + B - 1) / B * spb;
+    }
+    const int64_t ns = n_ctx + 1;
+    const int64_t pairs = (lq * s.group() + 255) / 256;
+    vs->item0[i] = static_cast<int32_t>(items);
+    vs->start[i] = static_cast<int32_t>(cu_q[i]);
+    vs->ctx0[i] = static_cast<int32_t>(cu_ctx[i]);
+    vs->rbase[i] = static_cast<int32_t>(rows);
+    vs->spb[i] = static_cast<int32_t>(spb);
+    items += pairs * ns * s.hkv;
+    rows += ns * lq;
+    if (items > 0x7fffffffLL || rows > 0x7fffffffLL) return -1;
+  }
+  vs->item0[s.b] = static_cast<int32_t>(items);
+  vs->start[s.b] = static_cast<int32_t>(cu_q[s.b]);
+  vs->ctx0[s.b] = static_cast<int32_t>(cu_ctx[s.b]);
+  vs->rbase[s.b] = static_cast<int32_t>(rows);
+  return rows;
+}
+
+cudaError_t launch_query_varlen(const Shape& s, const VarSeqs& vs, const void* q,
+                                const void* kc, const void* vc, const CacheRef& c,
+                                float* o_parts, float* lse_parts, void* o, float* lse,
+                                cudaStream_t st) {
+  cudaError_t e = s.d == 128 ? launch_query_varlen_t<128>(s, vs, q, kc, vc, c, o_parts, lse_parts, st)
+                             : launch_query_varlen_t<64>(s, vs, q, kc, vc, c, o_parts, lse_parts, st);
+  if (e != cudaSuccess) return e;
+  return launch_merge_varlen(o_parts, lse_parts, vs, s.B, s.hq, s.d, o, lse, st);
+}
 
 cudaError_t launch_phase1_sm100(const Shape& s, const void* q, const void* k, const void* v,
                                 void* o, float* lse, cudaStream_t st) {

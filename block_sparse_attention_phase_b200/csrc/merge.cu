@@ -22,25 +22,54 @@ namespace {
 
 constexpr int kWarps = 8;
 
-template <int D>
+// Varlen query pass: one row per (packed query token, head); the token's sequence
+// (binary search in vs.start) gives its split count and partial rows: split s of
+// sequence i holds token-rows rbase[i] + s * lq_i .. (o: [rows, H, D]; lse: H x lq_i
+// per split). Outputs are packed: o [total, H, D], lse [H, total].
+template <int D, bool kVarlen>
 __global__ void __launch_bounds__(kWarps * 32) merge_kernel(
     const float* __restrict__ o_parts, const float* __restrict__ lse_parts, int32_t S, int32_t b,
-    int64_t T, int32_t H, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+    int64_t T, int32_t H, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
+    const __grid_constant__ VarSeqs vs, int64_t block_size) {
   constexpr int E = D / 32;
   __shared__ float red[kWarps];
   __shared__ float acc_s[kWarps][D];
   __shared__ float wsum_s[kWarps];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int64_t row = blockIdx.x;  // (bb, t, h) with h fastest
+  const int64_t row = blockIdx.x;  // (bb, t, h) with h fastest; varlen: (packed token, h)
   const int h = static_cast<int>(row % H);
-  const int64_t t = (row / H) % T;
-  const int bb = static_cast<int>(row / (static_cast<int64_t>(H) * T));
-  // lse_parts[s][bb][h][t]; o_parts[s][bb][t][h][:]
-  const int64_t lse_stride = static_cast<int64_t>(b) * H * T;
-  const int64_t lse_off = (static_cast<int64_t>(bb) * H + h) * T + t;
-  const int64_t o_stride = static_cast<int64_t>(b) * T * H * D;
-  const int64_t o_off = ((static_cast<int64_t>(bb) * T + t) * H + h) * D + lane * E;
+  int64_t lse_stride, lse_off, o_stride, o_off, out_o, out_lse;
+  if constexpr (kVarlen) {
+    const int64_t tg = row / H;
+    int lo = 0, hi = vs.n;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (vs.start[mid] <= tg) lo = mid; else hi = mid;
+    }
+    const int64_t lq = vs.start[lo + 1] - vs.start[lo];
+    const int64_t t = tg - vs.start[lo];
+    const int64_t L = vs.ctx0[lo + 1] - vs.ctx0[lo];
+    const int64_t B = block_size < L ? block_size : L;
+    S = static_cast<int32_t>((L > 0 ? (L + B - 1) / B * vs.spb[lo] : 0) + 1);
+    const int64_t r0 = vs.rbase[lo];
+    lse_stride = lq * H;
+    lse_off = r0 * H + static_cast<int64_t>(h) * lq + t;
+    o_stride = lq * H * D;
+    o_off = ((r0 + t) * H + h) * D + lane * E;
+    out_o = (tg * H + h) * D + lane * E;
+    out_lse = static_cast<int64_t>(h) * T + tg;  // T = total packed tokens
+  } else {
+    const int64_t t = (row / H) % T;
+    const int bb = static_cast<int>(row / (static_cast<int64_t>(H) * T));
+    // lse_parts[s][bb][h][t]; o_parts[s][bb][t][h][:]
+    lse_stride = static_cast<int64_t>(b) * H * T;
+    lse_off = (static_cast<int64_t>(bb) * H + h) * T + t;
+    o_stride = static_cast<int64_t>(b) * T * H * D;
+    o_off = ((static_cast<int64_t>(bb) * T + t) * H + h) * D + lane * E;
+    out_o = o_off;
+    out_lse = lse_off;
+  }
 
   // Launched programmatically: wait until the kernel that wrote the partials has
   // finished, then let the next kernel in the stream start being scheduled (the
@@ -87,7 +116,7 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) Wt += wsum_s[w];
     const float inv = Wt > 0.f ? 1.f / Wt : 0.f;
-    __nv_bfloat16* dst = o + ((static_cast<int64_t>(bb) * T + t) * H + h) * D + lane * E;
+    __nv_bfloat16* dst = o + out_o;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       float x = 0.f;
@@ -95,7 +124,7 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(
       for (int w = 0; w < kWarps; ++w) x += acc_s[w][lane * E + e];
       dst[e] = __float2bfloat16_rn(x * inv);
     }
-    if (lse && lane == 0) lse[lse_off] = Wt > 0.f ? M + logf(Wt) : -INFINITY;
+    if (lse && lane == 0) lse[out_lse] = Wt > 0.f ? M + logf(Wt) : -INFINITY;
   }
 }
 
@@ -109,11 +138,34 @@ cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int32_t n
   if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(rows));
   auto* oo = static_cast<__nv_bfloat16*>(o);
+  VarSeqs vs;
+  vs.n = 0;
   const cudaError_t e =
-      d == 128 ? launch_programmatic(merge_kernel<128>, grid, dim3(kWarps * 32), 0, st, o_parts,
-                                     lse_parts, n_splits, b, tokens, heads, oo, lse)
-               : launch_programmatic(merge_kernel<64>, grid, dim3(kWarps * 32), 0, st, o_parts,
-                                     lse_parts, n_splits, b, tokens, heads, oo, lse);
+      d == 128 ? launch_programmatic(merge_kernel<128, false>, grid, dim3(kWarps * 32), 0, st,
+                                     o_parts, lse_parts, n_splits, b, tokens, heads, oo, lse, vs,
+                                     int64_t{0})
+               : launch_programmatic(merge_kernel<64, false>, grid, dim3(kWarps * 32), 0, st,
+                                     o_parts, lse_parts, n_splits, b, tokens, heads, oo, lse, vs,
+                                     int64_t{0});
+  if (e != cudaSuccess) return e;
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge_varlen(const float* o_parts, const float* lse_parts, const VarSeqs& vs,
+                                int64_t block_size, int32_t heads, int32_t d, void* o, float* lse,
+                                cudaStream_t st) {
+  const int64_t total = vs.start[vs.n];
+  const int64_t rows = total * heads;
+  if (rows == 0) return cudaSuccess;
+  if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(rows));
+  auto* oo = static_cast<__nv_bfloat16*>(o);
+  const cudaError_t e =
+      d == 128 ? launch_programmatic(merge_kernel<128, true>, grid, dim3(kWarps * 32), 0, st,
+                                     o_parts, lse_parts, 0, 1, total, heads, oo, lse, vs, block_size)
+               : launch_programmatic(merge_kernel<64, true>, grid, dim3(kWarps * 32), 0, st,
+                                     o_parts, lse_parts, 0, 1, total, heads, oo, lse, vs, block_size);
   if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();

@@ -158,7 +158,91 @@ __global__ void cache_write_kernel(const uint4* __restrict__ k, const uint4* __r
   }
 }
 
+// Varlen cache write: sequence i's rows [0, e0[i+1] - e0[i]) of its cache (its
+// query rows, then zeros up to the end of the tile or page) come from packed rows
+// q0[i] .. of k, v [total, Hkv, d]; e0 is the prefix of those row counts.
+struct CacheRows {
+  int32_t n;
+  int32_t q0[kMaxVarSeqs + 1];
+  int32_t e0[kMaxVarSeqs + 1];
+};
+
+__global__ void cache_write_varlen_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                          int32_t hkv, int32_t d, uint4* __restrict__ kc,
+                                          uint4* __restrict__ vc, int64_t cap,
+                                          const int32_t* __restrict__ table, int32_t P,
+                                          int32_t max_pages, int32_t num_pages, uint32_t* status,
+                                          const __grid_constant__ CacheRows cr) {
+  const int64_t per_row = static_cast<int64_t>(hkv) * d / 8;
+  const int64_t total = static_cast<int64_t>(cr.e0[cr.n]) * per_row;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t e = i % per_row;
+    const int64_t gr = i / per_row;
+    int lo = 0, hi = cr.n;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (cr.e0[mid] <= gr) lo = mid; else hi = mid;
+    }
+    const int64_t r = gr - cr.e0[lo];
+    const int64_t rows = cr.q0[lo + 1] - cr.q0[lo];
+    int64_t drow = static_cast<int64_t>(lo) * cap + r;
+    if (table) {
+      const int64_t page = table[static_cast<int64_t>(lo) * max_pages + r / P];
+      if (page < 0 || page >= num_pages) {
+        atomicOr(status, kBoundsFlag);
+        continue;
+      }
+      drow = page * P + r % P;
+    }
+    const int64_t dst = drow * per_row + e;
+    if (r < rows) {
+      const int64_t src = (cr.q0[lo] + r) * per_row + e;
+      kc[dst] = k[src];
+      vc[dst] = v[src];
+    } else {
+      kc[dst] = make_uint4(0u, 0u, 0u, 0u);
+      vc[dst] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_cache_write_varlen(const Shape& s, const int64_t* cu_q, const void* k,
+                                      const void* v, const CacheRef& c, cudaStream_t st) {
+  CacheRows cr;
+  cr.n = s.b;
+  int64_t ext_total = 0;
+  for (int i = 0; i < s.b; ++i) {
+    cr.q0[i] = static_cast<int32_t>(cu_q[i]);
+    cr.e0[i] = static_cast<int32_t>(ext_total);
+    const int64_t rows = cu_q[i + 1] - cu_q[i];
+    // zero-fill to the end of the page (paged) or of the 128-row tile (contiguous,
+    // within the capacity), so the query pass's cache tiles read zeros past the rows
+    int64_t ext = rows;
+    if (c.paged()) {
+      ext = (rows + c.page_size - 1) / c.page_size * c.page_size;
+    } else {
+      ext = (rows + 127) / 128 * 128;
+      if (ext > c.cap) ext = c.cap;
+    }
+    ext_total += ext;
+  }
+  cr.q0[s.b] = static_cast<int32_t>(cu_q[s.b]);
+  cr.e0[s.b] = static_cast<int32_t>(ext_total);
+  const int64_t total = ext_total * s.hkv * s.d / 8;
+  if (total == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks64 = (total + threads - 1) / threads;
+  const unsigned blocks = static_cast<unsigned>(blocks64 < 4096 ? blocks64 : 4096);
+  cache_write_varlen_kernel<<<blocks, threads, 0, st>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), s.hkv, s.d,
+      static_cast<uint4*>(c.k), static_cast<uint4*>(c.v), c.cap, c.page_table, c.page_size,
+      c.max_pages, c.num_pages, device_status_word(), cr);
+  count_launch();
+  return cudaGetLastError();
+}
 
 cudaError_t launch_simple_phase1(const Shape& s, const void* q, const void* k, const void* v,
                                  void* o, float* lse, cudaStream_t st) {

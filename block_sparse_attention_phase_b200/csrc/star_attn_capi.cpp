@@ -423,6 +423,70 @@ STAR_ATTN_API star_status_t star_attn_phase2_decode_varlen(
                                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
+STAR_ATTN_API size_t star_attn_query_varlen_workspace_bytes(const star_attn_shape_t* shape,
+                                                            const int64_t* cu_ctx,
+                                                            const int64_t* cu_q) {
+  Shape s;
+  if (star::resolve(shape, &s) != STAR_OK || !cu_ctx || !cu_q || s.b > star::kMaxVarSeqs) return 0;
+  if (!star::valid_offsets(cu_ctx, s.b, s.L) || !star::valid_offsets(cu_q, s.b, cu_q[s.b])) return 0;
+  star::VarSeqs vs;
+  const int64_t rows = star::plan_query_varlen(s, cu_ctx, cu_q, star::varlen_target_ctas(), &vs);
+  if (rows < 0) return 0;
+  const size_t per = static_cast<size_t>(rows) * s.hq;
+  return star::align256(per * s.d * sizeof(float)) + star::align256(per * sizeof(float));
+}
+
+STAR_ATTN_API star_status_t star_attn_phase2_query_varlen(
+    const star_attn_shape_t* shape, const int64_t* cu_ctx, const int64_t* cu_q, const void* q,
+    const void* k, const void* v, const void* k_ctx, const void* v_ctx, void* k_cache,
+    void* v_cache, int64_t cache_capacity, const int32_t* page_table, int32_t page_size,
+    int32_t num_pages, int32_t max_pages, void* o, float* lse, void* workspace,
+    size_t workspace_bytes, star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  if (s.b > star::kMaxVarSeqs) return STAR_ERR_UNSUPPORTED;
+  if (!cu_ctx || !cu_q || !star::valid_offsets(cu_ctx, s.b, s.L) ||
+      !star::valid_offsets(cu_q, s.b, cu_q[s.b]))
+    return STAR_ERR_INVALID_ARG;
+  if (cu_q[s.b] > (int64_t{1} << 31) - 1) return STAR_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, k_ctx, v_ctx, k_cache, v_cache, o};
+  for (const void* p : ptrs)
+    if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned4(lse) || !star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
+  star::CacheRef c;
+  if (page_table) {
+    st = star::check_pages(page_size, num_pages, page_table, max_pages);
+    if (st != STAR_OK) return st;
+    c = star::paged_ref(k_cache, v_cache, page_size, num_pages, page_table, max_pages);
+  } else {
+    if (cache_capacity < 1) return STAR_ERR_INVALID_ARG;
+    c.k = k_cache;
+    c.v = v_cache;
+    c.cap = cache_capacity;
+  }
+  for (int i = 0; i < s.b; ++i) {
+    const int64_t lq = cu_q[i + 1] - cu_q[i];
+    if (page_table ? (lq + page_size - 1) / page_size > max_pages : lq > cache_capacity)
+      return STAR_ERR_CACHE_FULL;
+  }
+  star::VarSeqs vs;
+  const int64_t rows = star::plan_query_varlen(s, cu_ctx, cu_q, star::varlen_target_ctas(), &vs);
+  if (rows < 0) return STAR_ERR_UNSUPPORTED;
+  const size_t per = static_cast<size_t>(rows) * s.hq;
+  if (!workspace || workspace_bytes < star::align256(per * s.d * sizeof(float)) +
+                                          star::align256(per * sizeof(float)))
+    return STAR_ERR_WORKSPACE;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = star::launch_cache_write_varlen(s, cu_q, k, v, c, cs);
+  if (e != cudaSuccess) return STAR_ERR_CUDA;
+  float* o_parts = static_cast<float*>(workspace);
+  float* lse_parts = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                              star::align256(per * s.d * sizeof(float)));
+  return star::cuda_status(
+      star::launch_query_varlen(s, vs, q, k_ctx, v_ctx, c, o_parts, lse_parts, o, lse, cs));
+}
+
 STAR_ATTN_API star_status_t star_attn_phase2_query_paged(
     const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
     int64_t query_len, const void* k_ctx, const void* v_ctx, void* k_pages, void* v_pages,

@@ -79,11 +79,18 @@ struct CacheRef {
 // A varlen batch as the kernels see it (passed by value as a kernel parameter):
 // sequence i owns work items [item0[i], item0[i+1]) and tokens
 // [start[i], start[i+1]) of the packed tensors. n = 0: a uniform batch.
+// The Phase-2 query pass of a varlen batch also uses: ctx0 (first context token of
+// each sequence in the packed context), rbase (first partial token-row of each
+// sequence: its splits' partials are [S_i, lq_i] token rows from there) and spb
+// (chunks per context block).
 constexpr int kMaxVarSeqs = 128;
 struct VarSeqs {
   int32_t n;
   int32_t item0[kMaxVarSeqs + 1];
   int32_t start[kMaxVarSeqs + 1];
+  int32_t ctx0[kMaxVarSeqs + 1];
+  int32_t rbase[kMaxVarSeqs + 1];
+  int32_t spb[kMaxVarSeqs];
 };
 
 // A varlen decode batch (kernel parameter): sequence i owns CTAs [cta0[i], cta0[i+1])
@@ -165,6 +172,21 @@ cudaError_t launch_rope(const Shape& s, const float* inv_freq, int64_t pos0, con
 cudaError_t launch_phase1_anchor_q(const Shape& s, const void* q, const void* q_anchor,
                                    const void* k, const void* v, void* o, float* lse,
                                    cudaStream_t st);
+// Phase-2 query pass over a varlen batch: split plan (host offsets cu_ctx, cu_q),
+// returning the partial token-rows needed (-1: too large) and filling vs.
+int64_t plan_query_varlen(const Shape& s, const int64_t* cu_ctx, const int64_t* cu_q,
+                          int64_t target_ctas, VarSeqs* vs);
+cudaError_t launch_cache_write_varlen(const Shape& s, const int64_t* cu_q, const void* k,
+                                      const void* v, const CacheRef& c, cudaStream_t st);
+// Partials (after the cache write) and the varlen merge into o [total_q, Hq, d],
+// lse [Hq, total_q].
+cudaError_t launch_query_varlen(const Shape& s, const VarSeqs& vs, const void* q,
+                                const void* kc, const void* vc, const CacheRef& c,
+                                float* o_parts, float* lse_parts, void* o, float* lse,
+                                cudaStream_t st);
+cudaError_t launch_merge_varlen(const float* o_parts, const float* lse_parts, const VarSeqs& vs,
+                                int64_t block_size, int32_t heads, int32_t d, void* o, float* lse,
+                                cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t wait_ns, cudaStream_t st);
 cudaError_t launch_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t st);
 

@@ -225,6 +225,36 @@ STAR_ATTN_API star_status_t star_attn_phase2_decode_fused(
     star_stream_t stream);
 
 /*
+ * The Phase-2 query pass over a varlen batch: every sequence has its own context
+ * length and its own number of query tokens. Same computation per sequence as
+ * star_attn_phase2_query() with batch 1, in one cache write, one partial launch and
+ * one merge launch.
+ *   shape->batch = sequences (at most 128); shape->ctx_len = total context tokens.
+ *   cu_ctx: HOST int64 [batch + 1] offsets of the packed context k_ctx, v_ctx
+ *     [total_ctx, Hkv, d]; cu_q: HOST int64 [batch + 1] offsets of the packed query
+ *     tokens q [total_q, Hq, d], k, v [total_q, Hkv, d] (both: first 0, non-decreasing).
+ *   Cache: contiguous k_cache/v_cache [batch, cache_capacity, Hkv, d] (page_table
+ *     NULL) or a page pool (page_table [batch, max_pages], page_size, num_pages), as
+ *     in star_attn_phase2_decode_varlen(). Rows [0, lq_i) of sequence i's cache get
+ *     its query tokens' KV; the rows after them up to the end of their 128-row tile
+ *     (contiguous, within the capacity) or page (paged) are written with zeros.
+ *   o [total_q, Hq, d] bf16; lse [Hq, total_q] or NULL.
+ *   workspace: star_attn_query_varlen_workspace_bytes(shape, cu_ctx, cu_q) bytes.
+ * Errors: STAR_ERR_CACHE_FULL if a sequence's query tokens do not fit its cache;
+ * STAR_ERR_UNSUPPORTED for more than 128 sequences.
+ */
+STAR_ATTN_API size_t star_attn_query_varlen_workspace_bytes(const star_attn_shape_t* shape,
+                                                            const int64_t* cu_ctx,
+                                                            const int64_t* cu_q);
+
+STAR_ATTN_API star_status_t star_attn_phase2_query_varlen(
+    const star_attn_shape_t* shape, const int64_t* cu_ctx, const int64_t* cu_q, const void* q,
+    const void* k, const void* v, const void* k_ctx, const void* v_ctx, void* k_cache,
+    void* v_cache, int64_t cache_capacity, const int32_t* page_table, int32_t page_size,
+    int32_t num_pages, int32_t max_pages, void* o, float* lse, void* workspace,
+    size_t workspace_bytes, star_stream_t stream);
+
+/*
  * One decode step over a varlen batch (continuous batching): every sequence has its
  * own context length and its own number of cached query-local rows. Same
  * computation per sequence as star_attn_phase2_decode() with batch 1, in one

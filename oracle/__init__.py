@@ -35,6 +35,7 @@ from .star_oracle import (  # noqa: F401
     phase2_query_head,
     phase2_query_head_blockwise,
     phase2_query,
+    phase2_query_varlen,
     phase2_decode_head,
     phase2_decode,
     phase2_decode_varlen,

@@ -281,6 +281,28 @@ def phase2_decode(q_t, k_t, v_t, k_ctx, v_ctx, k_cache, v_cache, cache_len: int,
     return o, lse, k_cache_new, v_cache_new
 
 
+def phase2_query_varlen(q_qry, k_qry, v_qry, k_ctx, v_ctx, cu_ctx: Sequence[int],
+                        cu_q: Sequence[int], scale: float = None):
+    """Phase-2 query tokens over a varlen batch: sequence i has context tokens
+    [cu_ctx[i], cu_ctx[i+1]) of k_ctx, v_ctx [total_ctx, Hkv, d] and query tokens
+    [cu_q[i], cu_q[i+1]) of q_qry [total_q, Hq, d], k_qry, v_qry [total_q, Hkv, d];
+    each sequence is the batch-1 query pass of its own slices.
+    Returns o [total_q, Hq, d] and lse [Hq, total_q]."""
+    total_q, Hq, d = q_qry.shape
+    o = np.zeros((total_q, Hq, d), dtype=F64)
+    lse = np.zeros((Hq, total_q), dtype=F64)
+    for i in range(len(cu_q) - 1):
+        a, e = cu_q[i], cu_q[i + 1]
+        c0, c1 = cu_ctx[i], cu_ctx[i + 1]
+        if e == a:
+            continue
+        oi, li = phase2_query(q_qry[None, a:e], k_qry[None, a:e], v_qry[None, a:e],
+                              k_ctx[None, c0:c1], v_ctx[None, c0:c1], scale)
+        o[a:e] = oi[0]
+        lse[:, a:e] = li[0]
+    return o, lse
+
+
 def phase2_decode_varlen(q_t, k_t, v_t, k_ctx, v_ctx, cu_ctx: Sequence[int], k_cache, v_cache,
                          cache_lens: Sequence[int], scale: float = None):
     """One decode step over a varlen batch: sequence i has the context tokens

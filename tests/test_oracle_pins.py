@@ -387,6 +387,34 @@ def check_model_decode_equals_query(seed=13):
     np.testing.assert_allclose(y1, xc + o.reshape(b, L, Hq * d) @ w_o[0], atol=1e-12)
 
 
+def check_query_varlen_is_global_per_sequence(seed=14):
+    """Varlen query pass: query token j of sequence i sees exactly its own context
+    and its own query tokens 0..j (torch SDPA with that mask)."""
+    rng = np.random.default_rng(seed)
+    Hq, Hkv, d = 4, 2, 8
+    ctx_lens, q_lens = [9, 0, 14], [3, 2, 0]
+    cu_c = [0] + list(np.cumsum(ctx_lens))
+    cu_q = [0] + list(np.cumsum(q_lens))
+    kc, vc = rand(rng, cu_c[-1], Hkv, d), rand(rng, cu_c[-1], Hkv, d)
+    q, k, v = rand(rng, cu_q[-1], Hq, d), rand(rng, cu_q[-1], Hkv, d), rand(rng, cu_q[-1], Hkv, d)
+    scale = 0.45
+    o, lse = oracle.phase2_query_varlen(q, k, v, kc, vc, cu_c, cu_q, scale)
+    for i in range(3):
+        a, e, c0, c1 = cu_q[i], cu_q[i + 1], cu_c[i], cu_c[i + 1]
+        n = e - a
+        if n == 0:
+            continue
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            keys = np.concatenate([kc[c0:c1, g], k[a:e, g]])
+            vals = np.concatenate([vc[c0:c1, g], v[a:e, g]])
+            mask = np.concatenate([np.ones((n, c1 - c0), dtype=bool),
+                                   np.tril(np.ones((n, n), dtype=bool))], axis=1)
+            ro, rl = sdpa_rows(q[a:e, h], keys, vals, scale, mask)
+            np.testing.assert_allclose(o[a:e, h], ro, atol=1e-12)
+            np.testing.assert_allclose(lse[h, a:e], rl, atol=1e-12)
+
+
 ALL_CHECKS = [check_single_block_is_causal, check_two_blocks_is_full_causal,
               check_phase1_keysets_golden, check_first_and_last_row_of_block,
               check_block_independence, check_gqa_mapping, check_closed_forms,
@@ -394,7 +422,7 @@ ALL_CHECKS = [check_single_block_is_causal, check_two_blocks_is_full_causal,
               check_merge_split_invariance, check_decode_matches_query_rows,
               check_phase1_varlen_per_sequence, check_decode_varlen_is_global_per_sequence,
               check_rope_is_complex_rotation, check_anchor_positions,
-              check_model_decode_equals_query]
+              check_model_decode_equals_query, check_query_varlen_is_global_per_sequence]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda c: c.__name__)

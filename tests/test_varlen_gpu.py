@@ -139,3 +139,68 @@ def test_decode_varlen_matches_oracle(case):
                 row = kcache[i, lens[i]]
             assert torch.equal(row, k[i, 0])
     assert m.device_status() == 0
+
+
+QRY_CASES = [
+    # ctx lens, query lens, Hq, Hkv, d, B, page size (0: contiguous)
+    ([3000, 0, 700, 9000], [5, 3, 0, 130], 8, 2, 128, 1024, 0),
+    ([3000, 700, 9000], [200, 1, 64], 8, 2, 128, 1024, 256),
+    ([513, 2048], [40, 17], 8, 1, 64, 512, 0),          # G = 8
+]
+
+
+@pytest.mark.parametrize("case", QRY_CASES, ids=lambda c: f"{len(c[0])}seq_g{c[2]//c[3]}_d{c[4]}_p{c[6]}")
+def test_query_varlen_then_decode(case):
+    """Varlen query pass against the oracle (NaN-filled caches), then a varlen decode
+    step on the caches it wrote, against the oracle again."""
+    ctx_lens, q_lens, hq, hkv, d, B, P = case
+    m = sa()
+    b = len(ctx_lens)
+    g = torch.Generator(device="cpu").manual_seed(sum(ctx_lens) + d)
+    rnd = lambda *shape: (torch.randn(*shape, generator=g) / d ** 0.5).to(torch.bfloat16).cuda()
+    cu_c, cu_q = [0], [0]
+    for n in ctx_lens:
+        cu_c.append(cu_c[-1] + n)
+    for n in q_lens:
+        cu_q.append(cu_q[-1] + n)
+    kc, vc = rnd(cu_c[-1], hkv, d), rnd(cu_c[-1], hkv, d)
+    q, k, v = rnd(cu_q[-1], hq, d), rnd(cu_q[-1], hkv, d), rnd(cu_q[-1], hkv, d)
+    cap = max(q_lens) + 2
+    if P:
+        max_pages = (cap + P - 1) // P
+        num_pages = b * max_pages + 1
+        table = torch.randperm(num_pages, generator=torch.Generator().manual_seed(1))[: b * max_pages]
+        table = table.view(b, max_pages).to(torch.int32).cuda()
+        kcache = torch.full((num_pages, P, hkv, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    else:
+        table = None
+        kcache = torch.full((b, cap, hkv, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vcache = torch.full_like(kcache, float("nan"))
+    o, lse = m.phase2_query_varlen(q, k, v, kc, vc, cu_c, cu_q, kcache, vcache, B, page_table=table)
+    ro, rl = oracle.phase2_query_varlen(to_np(q), to_np(k), to_np(v), to_np(kc), to_np(vc), cu_c, cu_q)
+    check_rows(to_np(o), ro, to_np(lse), rl, f"query varlen {case}")
+    # each sequence alone through the uniform entry point agrees
+    for i in range(b):
+        a, e = cu_q[i], cu_q[i + 1]
+        if e == a or cu_c[i + 1] == cu_c[i]:
+            continue
+        kci = torch.zeros((1, cap, hkv, d), dtype=torch.bfloat16, device="cuda")
+        vci = torch.zeros_like(kci)
+        oi, li = m.phase2_query(q[None, a:e].contiguous(), k[None, a:e].contiguous(),
+                                v[None, a:e].contiguous(), kc[None, cu_c[i]:cu_c[i + 1]].contiguous(),
+                                vc[None, cu_c[i]:cu_c[i + 1]].contiguous(), kci, vci, B)
+        check_rows(to_np(o[a:e]), to_np(oi[0]).astype(np.float64), to_np(lse[:, a:e]),
+                   to_np(li[0]).astype(np.float64), f"query varlen vs alone {i}")
+    # then one decode step per sequence on the caches the query pass wrote
+    qd, kd, vd = rnd(b, 1, hq, d), rnd(b, 1, hkv, d), rnd(b, 1, hkv, d)
+    od, ld = m.phase2_decode_varlen(qd, kd, vd, kc, vc, cu_c, kcache, vcache, q_lens, B,
+                                    page_table=table)
+    k_ref = np.zeros((b, cap, hkv, d))
+    v_ref = np.zeros((b, cap, hkv, d))
+    for i in range(b):
+        k_ref[i, :q_lens[i]] = to_np(k[cu_q[i]:cu_q[i + 1]])
+        v_ref[i, :q_lens[i]] = to_np(v[cu_q[i]:cu_q[i + 1]])
+    rod, rld, _, _ = oracle.phase2_decode_varlen(to_np(qd), to_np(kd), to_np(vd), to_np(kc),
+                                                 to_np(vc), cu_c, k_ref, v_ref, q_lens)
+    check_rows(to_np(od), rod, to_np(ld), rld, f"decode after query varlen {case}")
+    assert m.device_status() == 0
