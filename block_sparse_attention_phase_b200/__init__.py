@@ -38,6 +38,7 @@ EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase1_v
             "star_attn_phase2_decode", "star_attn_phase2_decode_fused",
             "star_attn_phase2_decode_varlen", "star_attn_decode_varlen_workspace_bytes",
             "star_attn_phase2_query_varlen", "star_attn_query_varlen_workspace_bytes",
+            "star_attn_phase2_partial",
             "star_attn_phase2_query_paged",
             "star_attn_phase2_decode_paged", "star_attn_phase2_decode_noalloc",
             "star_attn_lse_merge", "star_attn_simple_phase1",
@@ -87,6 +88,8 @@ def lib() -> ctypes.CDLL:
                                                   P, P, P, P, P, P, P, I64, P, I32, I32, I32,
                                                   P, P, P, SZ, P]),
         "star_attn_decode_varlen_workspace_bytes": (SZ, [SP, ctypes.POINTER(I64)]),
+        "star_attn_phase2_partial": (I32, [SP, P, P, P, I64, P, P, P, P, I64, I64, P, P, P, SZ,
+                                           P]),
         "star_attn_phase2_query_varlen": (I32, [SP, ctypes.POINTER(I64), ctypes.POINTER(I64),
                                                  P, P, P, P, P, P, P, I64, P, I32, I32, I32,
                                                  P, P, P, SZ, P]),
@@ -421,6 +424,42 @@ def phase2_query_varlen(q, k, v, k_ctx, v_ctx, cu_ctx, cu_q, k_cache, v_cache,
         _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(), _stream()),
         "star_attn_phase2_query_varlen")
     return o, lse
+
+
+def phase2_partial(q, block_size: int, k_ctx=None, v_ctx=None, k=None, v=None, k_cache=None,
+                   v_cache=None, cache_len: int = 0, scale: Optional[float] = None,
+                   workspace=None):
+    """One host's share of Phase 2 in the multi-host form: attention of the rows of
+    q [b, rows, Hq, d] over this host's context (k_ctx/v_ctx [b, L, Hkv, d], all
+    visible) and, on the query host, its query-local cache (k_cache/v_cache with the
+    rows' own k/v: one row = a decode step appended at cache_len, several rows = the
+    query tokens written to rows [0, rows)). Returns (o32 [b, rows, Hq, d] fp32,
+    lse [b, Hq, rows]) for star_attn_lse_merge across hosts."""
+    _bf16(q, "q", 4)
+    b, rows, hq, d = q.shape
+    if k_ctx is None and k_cache is None:
+        raise ValueError("a host needs context keys, a cache, or both")
+    if k_ctx is not None:
+        _bf16(k_ctx, "k_ctx", 4)
+        _bf16(v_ctx, "v_ctx", 4)
+        hkv, L = k_ctx.shape[2], k_ctx.shape[1]
+    else:
+        hkv, L = k_cache.shape[2], 1
+    if k_cache is not None:
+        for t, n in ((k, "k"), (v, "v"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+            _bf16(t, n, 4)
+    shape = make_shape(b, hq, hkv, d, L, block_size, scale)
+    if workspace is None:
+        workspace = _ws(shape, STAR_PHASE2_DECODE if rows == 1 else STAR_PHASE2_QUERY, rows,
+                        q.device, None)
+    o32 = torch.empty((b, rows, hq, d), dtype=torch.float32, device=q.device)
+    lse = torch.empty((b, hq, rows), dtype=torch.float32, device=q.device)
+    cap = 0 if k_cache is None else k_cache.shape[1]
+    _check(lib().star_attn_phase2_partial(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), rows, _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(k_cache), _ptr(v_cache), int(cache_len), cap, _ptr(o32), _ptr(lse), _ptr(workspace),
+        workspace.numel(), _stream()), "star_attn_phase2_partial")
+    return o32, lse
 
 
 def decode_varlen_workspace(batch, num_q_heads, num_kv_heads, head_dim, cu_ctx, block_size,

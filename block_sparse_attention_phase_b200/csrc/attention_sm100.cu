@@ -1009,11 +1009,12 @@ cudaError_t launch_phase1_varlen(const Shape& s, const int64_t* cu_seqlens, cons
 
 cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q, int64_t lq,
                               const void* kc, const void* vc, const CacheRef& c, float* o_parts,
-                              float* lse_parts, void* o, float* lse, cudaStream_t st) {
+                              float* lse_parts, void* o, float* lse, cudaStream_t st,
+                              bool o_fp32) {
   cudaError_t e = s.d == 128 ? launch_query_t<128>(s, p, q, lq, kc, vc, c, o_parts, lse_parts, st)
                              : launch_query_t<64>(s, p, q, lq, kc, vc, c, o_parts, lse_parts, st);
   if (e != cudaSuccess) return e;
-  return launch_merge(o_parts, lse_parts, p.n_splits, s.b, lq, s.hq, s.d, o, lse, st);
+  return launch_merge(o_parts, lse_parts, p.n_splits, s.b, lq, s.hq, s.d, o, lse, st, o_fp32);
 }
 
 }  // namespace star

@@ -26,10 +26,10 @@ constexpr int kWarps = 8;
 // (binary search in vs.start) gives its split count and partial rows: split s of
 // sequence i holds token-rows rbase[i] + s * lq_i .. (o: [rows, H, D]; lse: H x lq_i
 // per split). Outputs are packed: o [total, H, D], lse [H, total].
-template <int D, bool kVarlen>
+template <int D, bool kVarlen, class OutT>
 __global__ void __launch_bounds__(kWarps * 32) merge_kernel(
     const float* __restrict__ o_parts, const float* __restrict__ lse_parts, int32_t S, int32_t b,
-    int64_t T, int32_t H, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
+    int64_t T, int32_t H, OutT* __restrict__ o, float* __restrict__ lse,
     const __grid_constant__ VarSeqs vs, int64_t block_size) {
   constexpr int E = D / 32;
   __shared__ float red[kWarps];
@@ -116,13 +116,14 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) Wt += wsum_s[w];
     const float inv = Wt > 0.f ? 1.f / Wt : 0.f;
-    __nv_bfloat16* dst = o + out_o;
+    OutT* dst = o + out_o;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       float x = 0.f;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) x += acc_s[w][lane * E + e];
-      dst[e] = __float2bfloat16_rn(x * inv);
+      if constexpr (sizeof(OutT) == 4) dst[e] = x * inv;
+      else dst[e] = __float2bfloat16_rn(x * inv);
     }
     if (lse && lane == 0) lse[out_lse] = Wt > 0.f ? M + logf(Wt) : -INFINITY;
   }
@@ -132,21 +133,30 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(
 
 cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int32_t n_splits,
                          int32_t b, int64_t tokens, int32_t heads, int32_t d, void* o,
-                         float* lse, cudaStream_t st) {
+                         float* lse, cudaStream_t st, bool o_fp32) {
   const int64_t rows = static_cast<int64_t>(b) * tokens * heads;
   if (rows == 0) return cudaSuccess;
   if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(rows));
   auto* oo = static_cast<__nv_bfloat16*>(o);
+  auto* of = static_cast<float*>(o);
   VarSeqs vs;
   vs.n = 0;
-  const cudaError_t e =
-      d == 128 ? launch_programmatic(merge_kernel<128, false>, grid, dim3(kWarps * 32), 0, st,
-                                     o_parts, lse_parts, n_splits, b, tokens, heads, oo, lse, vs,
-                                     int64_t{0})
-               : launch_programmatic(merge_kernel<64, false>, grid, dim3(kWarps * 32), 0, st,
-                                     o_parts, lse_parts, n_splits, b, tokens, heads, oo, lse, vs,
-                                     int64_t{0});
+  const dim3 blk(kWarps * 32);
+  const int64_t none = 0;
+  cudaError_t e;
+  if (o_fp32)
+    e = d == 128 ? launch_programmatic(merge_kernel<128, false, float>, grid, blk, 0, st, o_parts,
+                                       lse_parts, n_splits, b, tokens, heads, of, lse, vs, none)
+                 : launch_programmatic(merge_kernel<64, false, float>, grid, blk, 0, st, o_parts,
+                                       lse_parts, n_splits, b, tokens, heads, of, lse, vs, none);
+  else
+    e = d == 128 ? launch_programmatic(merge_kernel<128, false, __nv_bfloat16>, grid, blk, 0, st,
+                                       o_parts, lse_parts, n_splits, b, tokens, heads, oo, lse, vs,
+                                       none)
+                 : launch_programmatic(merge_kernel<64, false, __nv_bfloat16>, grid, blk, 0, st,
+                                       o_parts, lse_parts, n_splits, b, tokens, heads, oo, lse, vs,
+                                       none);
   if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();
@@ -162,10 +172,10 @@ cudaError_t launch_merge_varlen(const float* o_parts, const float* lse_parts, co
   const dim3 grid(static_cast<unsigned>(rows));
   auto* oo = static_cast<__nv_bfloat16*>(o);
   const cudaError_t e =
-      d == 128 ? launch_programmatic(merge_kernel<128, true>, grid, dim3(kWarps * 32), 0, st,
-                                     o_parts, lse_parts, 0, 1, total, heads, oo, lse, vs, block_size)
-               : launch_programmatic(merge_kernel<64, true>, grid, dim3(kWarps * 32), 0, st,
-                                     o_parts, lse_parts, 0, 1, total, heads, oo, lse, vs, block_size);
+      d == 128 ? launch_programmatic(merge_kernel<128, true, __nv_bfloat16>, grid, dim3(kWarps * 32), 0,
+                                     st, o_parts, lse_parts, 0, 1, total, heads, oo, lse, vs, block_size)
+               : launch_programmatic(merge_kernel<64, true, __nv_bfloat16>, grid, dim3(kWarps * 32), 0,
+                                     st, o_parts, lse_parts, 0, 1, total, heads, oo, lse, vs, block_size);
   if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();

@@ -487,6 +487,68 @@ STAR_ATTN_API star_status_t star_attn_phase2_query_varlen(
       star::launch_query_varlen(s, vs, q, k_ctx, v_ctx, c, o_parts, lse_parts, o, lse, cs));
 }
 
+STAR_ATTN_API star_status_t star_attn_phase2_partial(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v, int64_t rows,
+    const void* k_ctx, const void* v_ctx, void* k_cache, void* v_cache, int64_t cache_len,
+    int64_t cache_capacity, float* o32, float* lse, void* workspace, size_t workspace_bytes,
+    star_stream_t stream) {
+  const bool has_ctx = k_ctx != nullptr;
+  const bool has_cache = k_cache != nullptr;
+  if (!shape || (!has_ctx && !has_cache) || rows < 1) return STAR_ERR_INVALID_ARG;
+  star_attn_shape_t sh = *shape;
+  if (!has_ctx) sh.ctx_len = 1;  // no context keys on this rank (the plan gets none)
+  Shape s;
+  star_status_t st = star::resolve(&sh, &s);
+  if (st != STAR_OK) return st;
+  if (!q || !o32 || !lse || !star::aligned16(q) || !star::aligned16(o32) || !star::aligned4(lse))
+    return STAR_ERR_INVALID_ARG;
+  if (has_ctx && (!v_ctx || !star::aligned16(k_ctx) || !star::aligned16(v_ctx)))
+    return STAR_ERR_INVALID_ARG;
+  if (has_cache) {
+    const void* ptrs[] = {k, v, k_cache, v_cache};
+    for (const void* p : ptrs)
+      if (!p || !star::aligned16(p)) return STAR_ERR_INVALID_ARG;
+    if (cache_capacity < 1 || cache_len < 0) return STAR_ERR_INVALID_ARG;
+    if (rows == 1 ? cache_len + 1 > cache_capacity : rows > cache_capacity) return STAR_ERR_CACHE_FULL;
+  }
+  if (!star::aligned16(workspace)) return STAR_ERR_INVALID_ARG;
+  star::SplitPlan plan = rows == 1 ? star::decode_plan(s) : star::query_plan(s, rows);
+  if (!has_ctx) {
+    plan.spb = 1;
+    plan.chunk = 1;
+    plan.n_ctx = 0;
+    plan.n_splits = 1;
+  } else if (!has_cache) {
+    plan.n_splits = plan.n_ctx;
+  }
+  const size_t need = star::partial_bytes(s, plan, rows);
+  if (!workspace || workspace_bytes < need) return STAR_ERR_WORKSPACE;
+  // Stand-ins for an absent context or cache: valid buffers whose maps no split uses.
+  star::CacheRef c;
+  c.k = has_cache ? k_cache : const_cast<void*>(k_ctx);
+  c.v = has_cache ? v_cache : const_cast<void*>(v_ctx);
+  c.cap = has_cache ? cache_capacity : s.L;
+  const void* kc = has_ctx ? k_ctx : k_cache;
+  const void* vc = has_ctx ? v_ctx : v_cache;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  float* o_parts = static_cast<float*>(workspace);
+  float* lse_parts = star::lse_parts_of(workspace, s, plan, rows);
+  cudaError_t e;
+  if (rows == 1) {
+    e = star::launch_decode_partials(s, plan, q, has_cache ? k : q, has_cache ? v : q, kc, vc, c,
+                                     has_cache ? cache_len : 0, o_parts, lse_parts, nullptr, cs);
+    if (e != cudaSuccess) return STAR_ERR_CUDA;
+    e = star::launch_merge(o_parts, lse_parts, plan.n_splits, s.b, 1, s.hq, s.d, o32, lse, cs, true);
+  } else {
+    if (has_cache) {
+      e = star::launch_cache_write(s, k, v, rows, c, cs);
+      if (e != cudaSuccess) return STAR_ERR_CUDA;
+    }
+    e = star::launch_query_path(s, plan, q, rows, kc, vc, c, o_parts, lse_parts, o32, lse, cs, true);
+  }
+  return star::cuda_status(e);
+}
+
 STAR_ATTN_API star_status_t star_attn_phase2_query_paged(
     const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
     int64_t query_len, const void* k_ctx, const void* v_ctx, void* k_pages, void* v_pages,

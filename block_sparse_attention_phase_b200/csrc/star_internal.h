@@ -117,9 +117,10 @@ cudaError_t launch_simple_phase2(const Shape& s, const void* q, int64_t rows, co
                                  const void* vc, const void* kk, const void* vk, int64_t cap,
                                  int64_t vis_base, int causal, void* o, float* lse,
                                  cudaStream_t st);
+// o: bf16 [b, tokens, heads, d], or fp32 with o_fp32.
 cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int32_t n_splits,
                          int32_t b, int64_t tokens, int32_t heads, int32_t d, void* o,
-                         float* lse, cudaStream_t st);
+                         float* lse, cudaStream_t st, bool o_fp32 = false);
 // Cache rows [0, rows) <- k, v [b, rows, Hkv, d]; for a paged cache, also zero
 // the rest of the page holding row rows-1.
 cudaError_t launch_cache_write(const Shape& s, const void* k, const void* v, int64_t rows,
@@ -162,7 +163,8 @@ cudaError_t launch_phase1_varlen(const Shape& s, const int64_t* cu_seqlens, cons
 // Phase-2 query tokens after their KV is in the cache: partials + merge into o/lse.
 cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q, int64_t lq,
                               const void* kc, const void* vc, const CacheRef& c, float* o_parts,
-                              float* lse_parts, void* o, float* lse, cudaStream_t st);
+                              float* lse_parts, void* o, float* lse, cudaStream_t st,
+                              bool o_fp32 = false);
 // RoPE on q [b, L, Hq, d] and k [b, L, Hkv, d] at positions pos0 + t (in place
 // allowed); q_anchor (or null) gets q rotated at the anchor-variant positions.
 cudaError_t launch_rope(const Shape& s, const float* inv_freq, int64_t pos0, const void* q_in,

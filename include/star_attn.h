@@ -225,6 +225,31 @@ STAR_ATTN_API star_status_t star_attn_phase2_decode_fused(
     star_stream_t stream);
 
 /*
+ * One host's share of Phase 2 in the pages' multi-host form (hotaipapers.com page,
+ * Phase 2 paragraph: the query goes to every host, each attends with its own keys
+ * and sends back one vector and one scalar per query row; the query host also
+ * holds the query-local cache). Computes, for `rows` query rows q [batch, rows, Hq, d],
+ * softmax attention over this host's keys only and returns it ready for
+ * star_attn_lse_merge() across hosts:
+ *   o32 [batch, rows, Hq, d] fp32 (normalised over these keys), lse [batch, Hq, rows].
+ * Keys: the context k_ctx, v_ctx [batch, shape->ctx_len, Hkv, d], all visible (NULL:
+ * this host holds no context; shape->ctx_len is then ignored), and, on the query
+ * host, the query-local cache k_cache, v_cache [batch, cache_capacity, Hkv, d] (NULL
+ * elsewhere) with k, v [batch, rows, Hkv, d] the rows' own KV:
+ *   rows == 1: a decode step, appended at cache_len, seeing cache rows 0..cache_len;
+ *   rows > 1: the query tokens, written to cache rows [0, rows), row j seeing 0..j.
+ *   workspace: star_attn_workspace_bytes(shape, rows == 1 ? STAR_PHASE2_DECODE :
+ *     STAR_PHASE2_QUERY, rows) bytes (nothing needs to be zero).
+ * Errors: STAR_ERR_INVALID_ARG if neither keys nor cache are given; CACHE_FULL as
+ * for the single-host calls.
+ */
+STAR_ATTN_API star_status_t star_attn_phase2_partial(
+    const star_attn_shape_t* shape, const void* q, const void* k, const void* v, int64_t rows,
+    const void* k_ctx, const void* v_ctx, void* k_cache, void* v_cache, int64_t cache_len,
+    int64_t cache_capacity, float* o32, float* lse, void* workspace, size_t workspace_bytes,
+    star_stream_t stream);
+
+/*
  * The Phase-2 query pass over a varlen batch: every sequence has its own context
  * length and its own number of query tokens. Same computation per sequence as
  * star_attn_phase2_query() with batch 1, in one cache write, one partial launch and

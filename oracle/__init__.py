@@ -39,6 +39,7 @@ from .star_oracle import (  # noqa: F401
     phase2_decode_head,
     phase2_decode,
     phase2_decode_varlen,
+    phase2_partial,
     rope,
     phase1_rope_head,
     phase1_rope,

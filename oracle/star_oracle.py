@@ -428,3 +428,48 @@ def model_forward(x_ctx, x_qry, x_dec: Sequence, w_qkv: Sequence, w_o: Sequence,
             outs.append(ot)
         xs = [x + oo.reshape(x.shape[0], x.shape[1], qd) @ Wo for x, oo in zip(xs, outs)]
     return xs[0], xs[1], xs[2:]
+
+
+def phase2_partial(q, k_ctx, v_ctx, k_new, v_new, k_cache, v_cache, cache_len: int,
+                   scale: float = None):
+    """One host's share of Phase 2 (hotaipapers.com page, Phase 2 paragraph: each host
+    attends with its own keys and returns one vector and one scalar per query row).
+    Rows of q [b, rows, Hq, d] attend to this host's context keys k_ctx, v_ctx
+    [b, L, Hkv, d] (all visible; None: no context) and, on the query host, to its
+    query-local cache k_cache, v_cache [b, cap, Hkv, d] (None elsewhere): one row is a
+    decode step whose k_new, v_new go to row cache_len and which sees rows
+    0..cache_len; several rows are the query tokens, written to rows [0, rows), row j
+    seeing rows 0..j. Returns o [b, rows, Hq, d], lse [b, Hq, rows] and the updated
+    caches (None without a cache)."""
+    q = np.asarray(q, F64)
+    b, rows, Hq, d = q.shape
+    Hkv = (k_ctx if k_ctx is not None else k_cache).shape[2]
+    scale = default_scale(d) if scale is None else scale
+    kc = vc = None
+    if k_cache is not None:
+        kc = np.array(k_cache, dtype=F64, copy=True)
+        vc = np.array(v_cache, dtype=F64, copy=True)
+        start = cache_len if rows == 1 else 0
+        kc[:, start:start + rows] = np.asarray(k_new, F64)
+        vc[:, start:start + rows] = np.asarray(v_new, F64)
+    o = np.zeros((b, rows, Hq, d), dtype=F64)
+    lse = np.zeros((b, Hq, rows), dtype=F64)
+    for bi in range(b):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            keys, vals, masks = [], [], []
+            if k_ctx is not None:
+                n = k_ctx.shape[1]
+                keys.append(np.asarray(k_ctx[bi, :, g], F64))
+                vals.append(np.asarray(v_ctx[bi, :, g], F64))
+                masks.append(np.ones((rows, n), dtype=bool))
+            if kc is not None:
+                last = np.full(rows, cache_len) if rows == 1 else np.arange(rows)
+                n = int(last.max()) + 1
+                keys.append(kc[bi, :n, g])
+                vals.append(vc[bi, :n, g])
+                masks.append(np.arange(n)[None, :] <= last[:, None])
+            o[bi, :, h], lse[bi, h] = attend(q[bi, :, h], np.concatenate(keys),
+                                             np.concatenate(vals), scale,
+                                             np.concatenate(masks, axis=1))
+    return o, lse, kc, vc

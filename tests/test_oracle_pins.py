@@ -415,6 +415,46 @@ def check_query_varlen_is_global_per_sequence(seed=14):
             np.testing.assert_allclose(lse[h, a:e], rl, atol=1e-12)
 
 
+def check_host_partials_merge_to_global(seed=15):
+    """The multi-host form of Phase 2: the context cut into per-host runs, each host's
+    partial over its own keys (the last one also over the query-local cache), merged
+    with the LSE combine, equals the single-host query pass and decode step."""
+    rng = np.random.default_rng(seed)
+    b, L, Lq, Hq, Hkv, d, cap = 2, 23, 3, 4, 2, 8, 6
+    kc, vc = rand(rng, b, L, Hkv, d), rand(rng, b, L, Hkv, d)
+    q, k, v = rand(rng, b, Lq, Hq, d), rand(rng, b, Lq, Hkv, d), rand(rng, b, Lq, Hkv, d)
+    cuts = [0, 5, 6, 17, L]
+    ref_o, ref_l = oracle.phase2_query(q, k, v, kc, vc)
+    parts = []
+    kcache = vcache = None
+    for i, (a, e) in enumerate(zip(cuts[:-1], cuts[1:])):
+        host = i == len(cuts) - 2
+        o, l, k2, v2 = oracle.phase2_partial(
+            q, kc[:, a:e], vc[:, a:e], k if host else None, v if host else None,
+            np.zeros((b, cap, Hkv, d)) if host else None, np.zeros((b, cap, Hkv, d)) if host else None, 0)
+        if host:
+            kcache, vcache = k2, v2
+        parts.append((o, l))
+    mo, ml = oracle.lse_merge(np.stack([p[0].transpose(0, 2, 1, 3) for p in parts]),
+                              np.stack([p[1] for p in parts]))
+    np.testing.assert_allclose(mo.transpose(0, 2, 1, 3), ref_o, atol=1e-12)
+    np.testing.assert_allclose(ml, ref_l, atol=1e-12)
+    # a decode step on top: the new row appended at row Lq of the host's cache
+    qd, kd, vd = rand(rng, b, 1, Hq, d), rand(rng, b, 1, Hkv, d), rand(rng, b, 1, Hkv, d)
+    rdo, rdl, _, _ = oracle.phase2_decode(qd, kd, vd, kc, vc, kcache, vcache, Lq)
+    parts = []
+    for i, (a, e) in enumerate(zip(cuts[:-1], cuts[1:])):
+        host = i == len(cuts) - 2
+        o, l, _, _ = oracle.phase2_partial(qd, kc[:, a:e], vc[:, a:e], kd if host else None,
+                                           vd if host else None, kcache if host else None,
+                                           vcache if host else None, Lq)
+        parts.append((o, l))
+    mo, ml = oracle.lse_merge(np.stack([p[0].transpose(0, 2, 1, 3) for p in parts]),
+                              np.stack([p[1] for p in parts]))
+    np.testing.assert_allclose(mo.transpose(0, 2, 1, 3), rdo, atol=1e-12)
+    np.testing.assert_allclose(ml, rdl, atol=1e-12)
+
+
 ALL_CHECKS = [check_single_block_is_causal, check_two_blocks_is_full_causal,
               check_phase1_keysets_golden, check_first_and_last_row_of_block,
               check_block_independence, check_gqa_mapping, check_closed_forms,
@@ -422,7 +462,8 @@ ALL_CHECKS = [check_single_block_is_causal, check_two_blocks_is_full_causal,
               check_merge_split_invariance, check_decode_matches_query_rows,
               check_phase1_varlen_per_sequence, check_decode_varlen_is_global_per_sequence,
               check_rope_is_complex_rotation, check_anchor_positions,
-              check_model_decode_equals_query, check_query_varlen_is_global_per_sequence]
+              check_model_decode_equals_query, check_query_varlen_is_global_per_sequence,
+              check_host_partials_merge_to_global]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda c: c.__name__)
