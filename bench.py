@@ -627,10 +627,14 @@ def main(argv=None):
                        "decode_merge": args.decode_merge,
                        "l2": "256 MiB write before every step; every decode step reads "
                              f"{w.decode_kv_bytes(0) / 1e6:.1f} MB of KV"},
-            "phase1": {"ms": p1_avg, "tok_s": tokens / (p1_avg / 1e3), "tflops": p1_tflops,
+            "phase1": {"ms": p1_avg, "ms_median": statistics.median(p1_list),
+                       "tok_s": tokens / (p1_avg / 1e3), "tflops": p1_tflops,
                        "frac_sustained": rl_p1["frac"], "frac_burst": rl_p1["frac_of_burst"]},
-            "query": {"ms": statistics.mean(q_list)},
-            "decode": {"ms_per_token_in_step": dec_avg, "gbs_in_step": dec_gbs,
+            "query": {"ms": statistics.mean(q_list), "ms_median": statistics.median(q_list)},
+            "decode": {"ms_per_token_in_step": dec_avg,
+                       "ms_per_token_in_step_median": statistics.median(dec_all),
+                       "ms_per_token_cold_median": statistics.median(cold),
+                       "gbs_in_step": dec_gbs,
                        "frac_hbm_in_step": dec_gbs / peaks["hbm_gbs"],
                        "ms_per_token_cold": dec_cold_avg, "gbs_cold": dec_cold_gbs,
                        "frac_hbm_cold": dec_cold_gbs / peaks["hbm_gbs"]},
