@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], 128 * kHalves);
+      mbar_init(&bars->p_full[s], 4 * kHalves);  // one arrival per softmax warp
 #pragma unroll
       for (int w4 = 0; w4 < 4; ++w4) mbar_init(&bars->xchg[s][w4], 64);
       mbar_init(&bars->o_bar[s], 1);
@@ -666,9 +666,12 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
           tmem_st32(lane_addr + o_col + c * 32, ob);
         }
       }
+      // Every lane's P (and O rescale) stores are complete; one lane per warp tells
+      // the MMA thread (32x fewer arrivals on the barrier than one per thread).
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[q]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[q]);
     }
     if constexpr (kHalves == 2) {
       // The row sum is the two halves' sums (same running max in both).
