@@ -235,3 +235,23 @@ def test_full_size_workload(name):
     del o, lse
     _phase2_sampled(w, x, heads, steps=[0, 1, w.decode_steps - 1])
     assert m.device_status() == 0
+
+
+@pytest.mark.parametrize("boost", [20.0, 60.0])
+def test_phase1_score_jumps_in_later_tiles(boost):
+    """A key whose score towers over everything seen before it, in a late tile of
+    its block: a moderate jump (the running max's raise is applied at the next tile)
+    and a huge one (the tile is recomputed with its own max). Rows that see the key
+    must put nearly all weight on it; all rows match the oracle."""
+    m = sa()
+    b, hq, hkv, d, L, B = 1, 2, 1, 128, 1536, 768
+    w, x = make(b, hq, hkv, d, L, B, 1, 1, seed=12)
+    q, k, v = x["q_ctx"].clone(), x["k_ctx"].clone(), x["v_ctx"].clone()
+    key = 768 + 500  # block 1, its fourth 128-key tile
+    for h in range(hq):
+        q[0, key + 10:, h] = q[0, key + 10:, h] * 0 + 1.0 / d ** 0.5
+    k[0, key, 0] = boost * torch.ones(d, dtype=torch.bfloat16, device="cuda")  # logit = boost
+    o, lse = m.phase1(q, k, v, B)
+    ro, rl = oracle.phase1(to_np(q), to_np(k), to_np(v), B)
+    check_rows(to_np(o), ro, to_np(lse), rl, f"score jump x{boost}")
+    assert m.device_status() == 0
