@@ -48,6 +48,7 @@ struct DecodeArgs {
   __nv_bfloat16* o;    // [b, 1, Hq, D]
   float* lse;          // [b, Hq, 1]
   uint32_t* counters;  // [b * Hkv], zero between calls
+  int32_t merge_batch; // splits the fused merge stages in shared memory per pass (>= 1)
 };
 
 constexpr int kTile = 64;      // tokens per TMA tile
@@ -66,9 +67,35 @@ STAR_HD constexpr size_t ring_bytes(int d, int stages) {
 STAR_HD constexpr size_t fused_weights_bytes(int64_t n_splits, int g) {
   return (static_cast<size_t>(n_splits) * g * 4 + 15) & ~size_t(15);
 }
-STAR_HD constexpr size_t fused_merge_bytes(int64_t n_splits, int g, int d) {
-  return fused_weights_bytes(n_splits, g) + size_t{kWarps} * g * d * 4;
+// The fused merge stages the LSE weights and then the splits' partial blocks (G x d
+// fp32 each) in the CTA's shared memory, reusing the ring. The region may grow past
+// the ring up to a cap that keeps the same number of CTAs per SM (three with 2
+// stages, two with 3 stages); splits that do not fit are staged in several passes.
+STAR_HD constexpr size_t merge_cap_bytes(int stages) {
+  return stages <= 2 ? size_t{72} * 1024 : size_t{108} * 1024;
 }
+STAR_HD constexpr size_t split_block_bytes(int g, int d) { return static_cast<size_t>(g) * d * 4; }
+STAR_HD constexpr size_t merge_region_bytes(int64_t n_splits, int g, int d, int stages) {
+  const size_t ring = ring_bytes(d, stages);
+  const size_t need = fused_weights_bytes(n_splits, g) + static_cast<size_t>(n_splits) * split_block_bytes(g, d);
+  const size_t want = need < merge_cap_bytes(stages) ? need : merge_cap_bytes(stages);
+  return want > ring ? want : ring;
+}
+// The fused merge needs room for the weights and at least one split's block.
+STAR_HD constexpr bool fused_merge_fits(int64_t n_splits, int g, int d, int stages) {
+  return fused_weights_bytes(n_splits, g) + split_block_bytes(g, d) <=
+         merge_region_bytes(n_splits, g, d, stages);
+}
+// Splits staged per pass of the fused merge (at least 1 when it fits).
+STAR_HD constexpr int64_t merge_batch_splits(int64_t n_splits, int g, int d, int stages) {
+  const int64_t nb = static_cast<int64_t>(
+      (merge_region_bytes(n_splits, g, d, stages) - fused_weights_bytes(n_splits, g)) /
+      split_block_bytes(g, d));
+  return nb < n_splits ? nb : n_splits;
+}
+// A uniform batch takes the two-kernel path (partials, then the merge kernel) when
+// its fused merge would need more passes than this.
+constexpr int64_t kMaxFusedPasses = 4;
 
 template <class VL>
 constexpr bool kIsVarlen = sizeof(VL) == sizeof(DecVarlen);
@@ -154,142 +181,139 @@ __device__ __forceinline__ Split locate(const DecodeArgs& a, const VL& dv) {
 // o = sum exp(lse_s - M) o_s / W, lse = M + ln W) for its G heads. It also puts
 // the counter back to zero for the next call.
 //
-// The combine is bound by L2 latency, so it is spread wide: the S x G split
-// LSEs are staged in shared memory in one pass and turned into weights there;
-// then the 4 warps take the splits in turn (warp w: splits w, w + 4, ...), each
-// lane owning float4 columns of the split's contiguous G x D partial block, with
-// several splits' loads in flight; the warps' sums meet in shared memory.
+// The combine is bound by L2 latency, so it takes as few round trips as possible:
+// one gpu-scope fence and one atomic per CTA (the grid-barrier pattern: the CTA's
+// stores, a CTA barrier, then one thread's fence and count); in the last CTA the
+// splits' partial blocks are copied into shared memory with asynchronous 16-byte
+// copies, issued before the LSEs are read so that both are in flight together.
+// Each thread then owns float4 columns of the G x d output and sums over the
+// staged splits from shared memory.
 template <int D, int G, class VL>
 __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const VL& dv, const Split& w,
                                               uint8_t* smem) {
+  constexpr int kThreads = kWarps * 32;
+  constexpr int F = G * D / 4;  // float4 columns of one split's G x D block
   __shared__ int s_last;
-  __shared__ float s_red[kWarps][G];
   __shared__ float s_m[G], s_w[G];
-  __threadfence();  // this thread's partial stores, before the count
-  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
   const int tid = threadIdx.x;  // 0 .. 127 (the consumer warps)
+  asm volatile("bar.sync 1, %0;" ::"r"(kThreads) : "memory");  // every partial store issued
   if (tid == 0) {
+    __threadfence();  // orders the CTA's partial stores (ordered before it by the barrier)
     uint32_t* ctr = a.counters + (static_cast<int64_t>(w.bb) * a.hkv + w.kvh);
     const uint32_t prev = atomicAdd(ctr, 1u);
     const int last = prev == static_cast<uint32_t>(w.n_splits - 1);
-    if (last) atomicExch(ctr, 0u);  // every split of this launch has counted
+    if (last) {
+      atomicExch(ctr, 0u);  // every split of this launch has counted
+      __threadfence();      // the other splits' partials are visible from here on
+    }
     s_last = last;
   }
-  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"r"(kThreads) : "memory");
   if (!s_last) return;
-  __threadfence();
 
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int S = w.n_splits;
+  const int nb = a.merge_batch;
   const int64_t row0 = part_row(a, dv, w, 0) * a.hq + w.kvh * G;  // split 0, first head
   const int64_t stride = (part_row(a, dv, w, 1) - part_row(a, dv, w, 0)) * a.hq;  // between splits
   const int64_t orow0 = static_cast<int64_t>(w.bb) * a.hq + w.kvh * G;  // output row
-  float* wts = reinterpret_cast<float*>(smem);                     // [S][G]
-  float4* red = reinterpret_cast<float4*>(smem + fused_weights_bytes(S, G));  // [kWarps][G*D/4]
+  float* wts = reinterpret_cast<float*>(smem);                                  // [S][G]
+  float4* parts = reinterpret_cast<float4*>(smem + fused_weights_bytes(S, G));  // [nb][F]
+  const uint32_t parts_s = smem_u32(parts);
 
-  // 1. the LSEs -> shared memory; per-head maximum
-  float m[G];
+  // Copies of splits sp0 .. sp0 + nb - 1 into the staging area (L2 only: the
+  // partials were written by other SMs).
+  auto stage = [&](int sp0) {
+    const int cnt = min(nb, S - sp0) * F;
+    for (int i = tid; i < cnt; i += kThreads) {
+      const float* src = a.o_parts + (row0 + static_cast<int64_t>(sp0 + i / F) * stride) * D + 4 * (i % F);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(parts_s + 16u * i), "l"(src)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  // 1. the LSEs -> shared memory (the first 4 per thread are loaded before the
+  //    staging copies are issued, so that they do not queue behind them); per head
+  //    (warp h % 4, lanes over the splits) the maximum M, the weights exp(lse_s - M)
+  //    in place and their sum W
+  auto lse_at = [&](int i) {
+    return __ldcg(a.lse_parts + row0 + static_cast<int64_t>(i / G) * stride + i % G);
+  };
+  float first[4];
 #pragma unroll
-  for (int h = 0; h < G; ++h) m[h] = -INFINITY;
-  for (int i = tid; i < S * G; i += kWarps * 32) {
-    const int sp = i / G, h = i % G;
-    const float l = __ldcg(a.lse_parts + row0 + sp * stride + h);
-    wts[i] = l;
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh)
-      if (hh == h) m[hh] = fmaxf(m[hh], l);
+  for (int k = 0; k < 4; ++k) {
+    const int i = tid + kThreads * k;
+    first[k] = i < S * G ? lse_at(i) : 0.f;
   }
+  stage(0);
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], off));
-    if (lane == 0) s_red[warp][h] = m[h];
+  for (int k = 0; k < 4; ++k) {
+    const int i = tid + kThreads * k;
+    if (i < S * G) wts[i] = first[k];
   }
-  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
-  if (tid < G) {
-    float mm = s_red[0][tid];
+  for (int i = tid + 4 * kThreads; i < S * G; i += kThreads) wts[i] = lse_at(i);
+  asm volatile("bar.sync 1, %0;" ::"r"(kThreads) : "memory");
+  for (int h = warp; h < G; h += kWarps) {
+    float m = -INFINITY;
+    for (int sp = lane; sp < S; sp += 32) m = fmaxf(m, wts[sp * G + h]);
 #pragma unroll
-    for (int wi = 1; wi < kWarps; ++wi) mm = fmaxf(mm, s_red[wi][tid]);
-    s_m[tid] = mm;
+    for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float sum = 0.f;
+    for (int sp = lane; sp < S; sp += 32) {
+      const float wv = m == -INFINITY ? 0.f : expf(wts[sp * G + h] - m);  // 0: empty split or head
+      wts[sp * G + h] = wv;
+      sum += wv;
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane == 0) {
+      s_m[h] = m;
+      s_w[h] = sum;
+    }
   }
-  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
 
-  // 2. weights exp(lse_s - M) in place (0 for an empty split or an all-empty head); sums
-  float wsum[G];
+  // 2. weighted sums of the staged partial blocks
+  constexpr int KPT = (F + kThreads - 1) / kThreads;  // float4 columns per thread
+  float4 acc[KPT];
 #pragma unroll
-  for (int h = 0; h < G; ++h) wsum[h] = 0.f;
-  for (int i = tid; i < S * G; i += kWarps * 32) {
-    const int h = i % G;
-    const float M = s_m[h];
-    const float wv = M == -INFINITY ? 0.f : expf(wts[i] - M);
-    wts[i] = wv;
+  for (int k = 0; k < KPT; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int sp0 = 0; sp0 < S; sp0 += nb) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"r"(kThreads) : "memory");  // staged blocks and weights ready
+    const int cnt = min(nb, S - sp0);
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh)
-      if (hh == h) wsum[hh] += wv;
-  }
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) wsum[h] += __shfl_xor_sync(0xffffffffu, wsum[h], off);
-  }
-  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");  // s_red reads above are done
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-    if (lane == 0) s_red[warp][h] = wsum[h];
-
-  // 3. weighted sums of the partial outputs
-  constexpr int F = G * D / 4;          // float4 columns of one split's G x D block
-  constexpr int KPL = (F + 31) / 32;    // per lane
-  float4 acc[KPL];
-#pragma unroll
-  for (int k = 0; k < KPL; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int sp = warp; sp < S; sp += kWarps) {
-    const float4* src = reinterpret_cast<const float4*>(a.o_parts + (row0 + sp * stride) * D);
-#pragma unroll
-    for (int k = 0; k < KPL; ++k) {
-      const int f = lane + 32 * k;
-      if (F % 32 == 0 || f < F) {
-        const float wv = wts[sp * G + f / (D / 4)];
-        const float4 x = __ldcg(src + f);
-        acc[k].x += wv * x.x;
-        acc[k].y += wv * x.y;
-        acc[k].z += wv * x.z;
-        acc[k].w += wv * x.w;
+    for (int k = 0; k < KPT; ++k) {
+      const int f = tid + kThreads * k;
+      if (F % kThreads == 0 || f < F) {
+        const int h = f / (D / 4);
+        for (int j = 0; j < cnt; ++j) {
+          const float wv = wts[(sp0 + j) * G + h];
+          const float4 x = parts[j * F + f];
+          acc[k].x += wv * x.x;
+          acc[k].y += wv * x.y;
+          acc[k].z += wv * x.z;
+          acc[k].w += wv * x.w;
+        }
       }
     }
-  }
-#pragma unroll
-  for (int k = 0; k < KPL; ++k) {
-    const int f = lane + 32 * k;
-    if (F % 32 == 0 || f < F) red[warp * F + f] = acc[k];
-  }
-  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
-  if (tid < G) {
-    float W = 0.f;
-#pragma unroll
-    for (int wi = 0; wi < kWarps; ++wi) W += s_red[wi][tid];
-    s_w[tid] = W;
-    if (a.lse) a.lse[orow0 + tid] = W > 0.f ? s_m[tid] + logf(W) : -INFINITY;
-  }
-  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
-  for (int f = tid; f < F; f += kWarps * 32) {
-    float4 x = red[f];
-#pragma unroll
-    for (int wi = 1; wi < kWarps; ++wi) {
-      const float4 y = red[wi * F + f];
-      x.x += y.x;
-      x.y += y.y;
-      x.z += y.z;
-      x.w += y.w;
+    if (sp0 + nb < S) {
+      asm volatile("bar.sync 1, %0;" ::"r"(kThreads) : "memory");  // staging area free again
+      stage(sp0 + nb);
     }
-    const float W = s_w[f / (D / 4)];
-    const float inv = W > 0.f ? 1.f / W : 0.f;
-    uint2 packed;
-    packed.x = pack_bf16x2(x.x * inv, x.y * inv);
-    packed.y = pack_bf16x2(x.z * inv, x.w * inv);
-    *reinterpret_cast<uint2*>(a.o + orow0 * D + 4 * f) = packed;  // G heads are contiguous
+  }
+  if (tid < G && a.lse) a.lse[orow0 + tid] = s_w[tid] > 0.f ? s_m[tid] + logf(s_w[tid]) : -INFINITY;
+#pragma unroll
+  for (int k = 0; k < KPT; ++k) {
+    const int f = tid + kThreads * k;
+    if (F % kThreads == 0 || f < F) {
+      const float W = s_w[f / (D / 4)];
+      const float inv = W > 0.f ? 1.f / W : 0.f;
+      uint2 packed;
+      packed.x = pack_bf16x2(acc[k].x * inv, acc[k].y * inv);
+      packed.y = pack_bf16x2(acc[k].z * inv, acc[k].w * inv);
+      *reinterpret_cast<uint2*>(a.o + orow0 * D + 4 * f) = packed;  // G heads are contiguous
+    }
   }
 }
 
@@ -308,11 +332,18 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
                                              ~uintptr_t(1023));
   uint8_t* kbuf = base;                          // [kStages][kTileBytes]
   uint8_t* vbuf = base + kStages * kTileBytes;   // [kStages][kTileBytes]
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + 2 * kStages * kTileBytes);
-  uint64_t* empty = full + kStages;
+  // The barriers live outside the dynamic region, which the fused merge reuses whole.
+  __shared__ alignas(8) uint64_t full[kStages];
+  __shared__ alignas(8) uint64_t empty[kStages];
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (warp == kWarps && lane == 0) {  // descriptor fetches overlap the prologue
+    tma_prefetch_desc(&mk_ctx);
+    tma_prefetch_desc(&mv_ctx);
+    tma_prefetch_desc(&mk_cache);
+    tma_prefetch_desc(&mv_cache);
+  }
   const Split w = locate(a, dv);
   const int bb = w.bb;
   const int kvh = w.kvh;
@@ -555,30 +586,48 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
       }
     }
     asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
-    pdl_wait();  // the previous kernel (which may still read the workspace) has finished
-    for (int idx = threadIdx.x; idx < G * D; idx += kWarps * 32) {
-      const int h = idx / D;
-      const int e = idx % D;
+    // Per head: the CTA's maximum over the warps, each warp's weight exp2(m_w - M)
+    // divided by the CTA's sum, and the CTA's LSE; then every thread writes float4
+    // columns of the G x D partial as the weighted sum of the warps' accumulators.
+    __shared__ float s_sc[kWarps][G];
+    __shared__ float s_plse[G];
+    if (threadIdx.x < G) {
+      const int h = threadIdx.x;
       float M = -INFINITY;
 #pragma unroll
       for (int wi = 0; wi < kWarps; ++wi) M = fmaxf(M, cm[wi * G + h]);
-      float lsum = 0.f, acc = 0.f;
-      if (M != -INFINITY) {
+      float sc[kWarps];
+      float lsum = 0.f;
 #pragma unroll
-        for (int wi = 0; wi < kWarps; ++wi) {
-          const float sc = ex2_approx((cm[wi * G + h] - M) * sl2);
-          lsum += cl[wi * G + h] * sc;
-          acc += cacc[(wi * G + h) * D + e] * sc;
-        }
+      for (int wi = 0; wi < kWarps; ++wi) {
+        sc[wi] = M == -INFINITY ? 0.f : ex2_approx((cm[wi * G + h] - M) * sl2);
+        lsum += cl[wi * G + h] * sc[wi];
       }
-      const int hq = kvh * G + h;
-      const int64_t row = part_row(a, dv, w, w.split);
-      a.o_parts[(row * a.hq + hq) * D + e] = lsum > 0.f ? acc / lsum : 0.f;
-      if (e == 0) {
-        a.lse_parts[row * a.hq + hq] =
-            lsum > 0.f ? (M * sl2 + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
-      }
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll
+      for (int wi = 0; wi < kWarps; ++wi) s_sc[wi][h] = sc[wi] * inv;
+      s_plse[h] = lsum > 0.f ? (M * sl2 + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
     }
+    asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
+    pdl_wait();  // the previous kernel (which may still read the workspace) has finished
+    const int64_t prow = part_row(a, dv, w, w.split) * a.hq + kvh * G;  // first head's row
+    const float4* cacc4 = reinterpret_cast<const float4*>(cacc);
+    float4* dst = reinterpret_cast<float4*>(a.o_parts + prow * D);
+    for (int f = threadIdx.x; f < G * D / 4; f += kWarps * 32) {
+      const int h = f / (D / 4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int wi = 0; wi < kWarps; ++wi) {
+        const float4 x = cacc4[wi * (G * D / 4) + f];
+        const float sc = s_sc[wi][h];
+        acc.x += sc * x.x;
+        acc.y += sc * x.y;
+        acc.z += sc * x.z;
+        acc.w += sc * x.w;
+      }
+      dst[f] = acc;
+    }
+    if (threadIdx.x < G) a.lse_parts[prow + threadIdx.x] = s_plse[threadIdx.x];
     if (a.counters) merge_if_last<D, G>(a, dv, w, base);
   }
 }
@@ -605,14 +654,19 @@ cudaError_t launch_decode_t(const Shape& s, const DecodeArgs& a, const VL& dv, d
          encode_tma_bf16_4d(&m[3], a.v_cache, D, s.hkv, cache_rows, a.cap, s.b, 64, 1, kTile, true);
   }
   if (!ok) return cudaErrorInvalidValue;
-  if (a.counters && fused_merge_bytes(max_splits, G, D) > ring_bytes(D, kStages))
-    return cudaErrorInvalidValue;
-  const size_t smem = ring_bytes(D, kStages) + 2 * kStages * sizeof(uint64_t) + 1024;
+  size_t region = ring_bytes(D, kStages);
+  DecodeArgs args = a;
+  if (a.counters) {
+    if (!fused_merge_fits(max_splits, G, D, kStages)) return cudaErrorInvalidValue;
+    region = merge_region_bytes(max_splits, G, D, kStages);
+    args.merge_batch = static_cast<int32_t>(merge_batch_splits(max_splits, G, D, kStages));
+  }
+  const size_t smem = region + 1024;  // + alignment of the region to 1024 bytes
   auto kern = decode_partials_kernel<D, G, kStages, VL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  e = launch_programmatic(kern, grid, dim3((kWarps + 1) * 32), smem, st, m[0], m[1], m[2], m[3], a,
+  e = launch_programmatic(kern, grid, dim3((kWarps + 1) * 32), smem, st, m[0], m[1], m[2], m[3], args,
                           dv);
   if (e != cudaSuccess) return e;
   count_launch();
@@ -671,7 +725,9 @@ cudaError_t dispatch(const Shape& s, const DecodeArgs& a, const VL& dv, dim3 gri
 }  // namespace
 
 bool decode_fused_fits(const Shape& s, const SplitPlan& p) {
-  return fused_merge_bytes(p.n_splits, s.group(), s.d) <= ring_bytes(s.d, decode_stages(p.chunk));
+  const int st = decode_stages(p.chunk);
+  return fused_merge_fits(p.n_splits, s.group(), s.d, st) &&
+         merge_batch_splits(p.n_splits, s.group(), s.d, st) * kMaxFusedPasses >= p.n_splits;
 }
 
 cudaError_t launch_decode_partials(const Shape& s, const SplitPlan& p, const void* q,
@@ -739,7 +795,7 @@ cudaError_t launch_decode_varlen(const Shape& s, const DecVarlen& dv, int64_t ma
 }
 
 bool decode_varlen_fused_fits(const Shape& s, int64_t max_splits, int64_t max_chunk) {
-  return fused_merge_bytes(max_splits, s.group(), s.d) <= ring_bytes(s.d, decode_stages(max_chunk));
+  return fused_merge_fits(max_splits, s.group(), s.d, decode_stages(max_chunk));
 }
 
 }  // namespace star

@@ -36,6 +36,7 @@ CASES = [
     (1, 2, 1, 64, 40, 1, 2, 2),          # 40 one-token blocks: 41 splits of one key
     (1, 8, 8, 128, 20000, 2500, 9, 3),   # G = 1, many splits per block
     (2, 64, 8, 128, 9000, 4096, 4, 2),   # G = 8, ragged last block
+    (1, 64, 8, 128, 8192, 1024, 4, 2),   # G = 8, 33 splits: the merge stages them in 2 passes
     (1, 8, 1, 64, 2000, 1, 2, 2),        # 2001 splits: too many to fuse, runs unfused
 ]
 
