@@ -76,6 +76,7 @@ DEC_CASES = [
     ([3000, 0, 700, 9000], [5, 0, 17, 130], 8, 2, 128, 1024, 0),
     ([3000, 0, 700, 9000], [5, 0, 127, 130], 8, 2, 128, 1024, 128),
     ([513, 2048], [64, 3], 8, 1, 64, 512, 0),           # G = 8
+    ([4096, 2048], [3, 5], 8, 1, 128, 512, 0),          # G = 8, d 128: 65 splits, merge in 4 passes
     ([40000, 100, 12000], [1, 2, 3], 32, 8, 128, 4096, 256),
 ]
 
