@@ -214,9 +214,10 @@ STAR_ATTN_API star_status_t star_attn_phase2_decode(
  *     (query pass, unfused decode) has written must be zeroed again first.
  *   The result equals star_attn_phase2_decode()'s to fp32 rounding of the merge
  *     (summation order differs); it is deterministic.
- *   Shapes with so many splits that the merge's weights do not fit in the kernel's
- *     shared memory (thousands of context blocks) run as partials + merge kernel,
- *     with the same results and without touching the counters.
+ *   Shapes with so many splits that the merge would need more than four passes over
+ *     the kernel's shared memory (hundreds of splits per sequence and kv-head, e.g.
+ *     block sizes of a few tokens) run as partials + merge kernel, with the same
+ *     results and without touching the counters.
  */
 STAR_ATTN_API star_status_t star_attn_phase2_decode_fused(
     const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
