@@ -477,20 +477,20 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       // address field cannot carry out: shared addresses stay below 256 KB). The
       // thread shares its SMSP with two busy softmax warps, so every instruction it
       // saves between MMAs shortens the hand-off.
-      const uint64_t qd0 = make_sdesc(sq_addr, 16, 1024), qd1 = make_sdesc(sq_addr + kTileBytes, 16, 1024);
-      const uint64_t kd0 = make_sdesc(sk_addr, 16, 1024), kd1 = make_sdesc(sk_addr + kTileBytes, 16, 1024);
-      const uint64_t vd0 = make_sdesc(sv_addr, kChunkBytes, 1024);
-      const uint64_t vd1 = make_sdesc(sv_addr + kTileBytes, kChunkBytes, 1024);
+      constexpr uint32_t kDescHi = sdesc_hi(1024);
+      const uint32_t qd0 = sdesc_lo(sq_addr, 16), qd1 = sdesc_lo(sq_addr + kTileBytes, 16);
+      const uint32_t kd0 = sdesc_lo(sk_addr, 16), kd1 = sdesc_lo(sk_addr + kTileBytes, 16);
+      const uint32_t vd0 = sdesc_lo(sv_addr, kChunkBytes), vd1 = sdesc_lo(sv_addr + kTileBytes, kChunkBytes);
       // S_q = Q_q K_j^T: A = Q, B = K, both K-major 128-byte swizzled (16 columns = 32 bytes a step).
       bool reload_q = false;
       if constexpr (M == Mode::kPhase1) reload_q = a.anchor_q && it.n_anchor > 0;
       auto issue_s = [&](int q, int j) {
-        const uint64_t qd = q ? qd1 : qd0;
-        const uint64_t kd = (j & 1) ? kd1 : kd0;
+        const uint32_t qd = q ? qd1 : qd0;
+        const uint32_t kd = (j & 1) ? kd1 : kd0;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off16 = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
-          tc_mma_ss(tmem + q * 128, qd + off16, kd + off16, kIdescQK, kk > 0 ? 1u : 0u);
+          const uint32_t off16 = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
+          tc_mma_ss_lo(tmem + q * 128, qd + off16, kd + off16, kDescHi, kIdescQK, kk > 0 ? 1u : 0u);
         }
         tc_commit(&bars->s_full[q]);
         if (reload_q && q == 1 && j == it.n_anchor - 1) tc_commit(&bars->q_free);
@@ -499,11 +499,11 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       // (d contiguous): 16 kv rows a step, the next 64 columns of d one chunk (LBO)
       // away, the next 8 kv rows 1024 B (SBO) away.
       auto issue_pv = [&](int q, int j) {
-        const uint64_t vd = (j & 1) ? vd1 : vd0;
+        const uint32_t vd = (j & 1) ? vd1 : vd0;
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          tc_mma_ts(tmem + 256 + q * D, tmem + q * 128 + kk * 8, vd + static_cast<uint64_t>(kk * (2048 >> 4)),
-                    kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts_lo(tmem + 256 + q * D, tmem + q * 128 + kk * 8, vd + kk * (2048 >> 4), kDescHi,
+                       kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
       };
       bool ok = wait_or_abort(&bars->q_full, 0, bars, a.status) &&
                 wait_or_abort(&bars->k_full[0], 0, bars, a.status);
