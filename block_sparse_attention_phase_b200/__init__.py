@@ -43,7 +43,8 @@ EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase1_v
             "star_attn_phase2_decode_paged", "star_attn_phase2_decode_noalloc",
             "star_attn_lse_merge", "star_attn_simple_phase1",
             "star_attn_simple_phase2", "star_attn_get_device_status",
-            "star_attn_selftest_wait_timeout", "star_attn_selftest_exp2", "star_attn_launch_count",
+            "star_attn_selftest_wait_timeout", "star_attn_selftest_exp2", "star_attn_selftest_read",
+            "star_attn_launch_count",
             "star_attn_status_string", "star_attn_version"]
 
 
@@ -106,6 +107,7 @@ def lib() -> ctypes.CDLL:
         "star_attn_get_device_status": (I32, [P]),
         "star_attn_selftest_wait_timeout": (I32, [ctypes.c_uint64, P]),
         "star_attn_selftest_exp2": (I32, [P, P, I64, P]),
+        "star_attn_selftest_read": (I32, [P, SZ, P, I32, P]),
         "star_attn_launch_count": (ctypes.c_uint64, []),
         "star_attn_status_string": (ctypes.c_char_p, [I32]),
         "star_attn_version": (ctypes.c_char_p, []),
@@ -572,6 +574,17 @@ def selftest_exp2(x: torch.Tensor) -> torch.Tensor:
     _check(lib().star_attn_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream()),
            "star_attn_selftest_exp2")
     return y
+
+
+def selftest_read(buf: torch.Tensor, sink: torch.Tensor, ctas: int) -> None:
+    """Stream every byte of the CUDA tensor `buf` once (read-only bandwidth probe);
+    `sink` is an int32 CUDA tensor of at least `ctas` elements."""
+    if not buf.is_cuda or not buf.is_contiguous():
+        raise TypeError("buf must be a contiguous CUDA tensor")
+    if sink.dtype != torch.int32 or sink.numel() < ctas or not sink.is_cuda:
+        raise TypeError("sink must be an int32 CUDA tensor with ctas elements")
+    _check(lib().star_attn_selftest_read(_ptr(buf), buf.numel() * buf.element_size(), _ptr(sink),
+                                         int(ctas), _stream()), "star_attn_selftest_read")
 
 
 def launch_count() -> int:

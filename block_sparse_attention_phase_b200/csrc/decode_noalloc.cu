@@ -32,6 +32,11 @@
 #include "star_internal.h"
 
 namespace star {
+
+// The shape checks every entry point applies (STAR_OK, STAR_ERR_INVALID_ARG or
+// STAR_ERR_UNSUPPORTED), from the C-ABI layer.
+star_status_t check_shape(const star_attn_shape_t* shape);
+
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t{4} << 20;
@@ -63,8 +68,11 @@ extern "C" STAR_ATTN_API star_status_t star_attn_phase2_decode_noalloc(
     const star_attn_shape_t* shape, const void* q, const void* k, const void* v,
     const void* k_ctx, const void* v_ctx, void* k_cache, void* v_cache, int64_t cache_len,
     int64_t cache_capacity, void* o, float* lse, star_stream_t stream) {
+  // An invalid or unsupported shape gets the same status as from star_attn_phase2_decode().
+  const star_status_t shape_status = star::check_shape(shape);
+  if (shape_status != STAR_OK) return shape_status;
   const size_t need = star_attn_workspace_bytes(shape, STAR_PHASE2_DECODE, 1);
-  if (need == 0) return STAR_ERR_INVALID_ARG;  // the shape itself is invalid or unsupported
+  if (need == 0) return STAR_ERR_INVALID_ARG;
   if (need > star::kNoAllocScratchBytes) return STAR_ERR_WORKSPACE;
   if (cache_len < 0 || cache_capacity < 1) return STAR_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, k_ctx, v_ctx, k_cache, v_cache, o};

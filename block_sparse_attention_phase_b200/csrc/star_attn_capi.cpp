@@ -14,12 +14,34 @@
 namespace star {
 namespace {
 
-constexpr int kSMs = 148;              // B200
 #ifndef STAR_DECODE_CTAS_PER_SM
 #define STAR_DECODE_CTAS_PER_SM 2
 #endif
 constexpr int kDecodeCtasPerSM = STAR_DECODE_CTAS_PER_SM;
 constexpr int64_t kMinChunk = 64;      // one TMA tile of keys
+
+// Streaming multiprocessors of the current device, read once per device; 148 (a
+// B200) when no device can be queried, e.g. for workspace sizing on a host
+// without a GPU.
+constexpr int kMaxDevices = 64;
+constexpr int kDefaultSMs = 148;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();  // a failed query must not linger as the next call's error
+    return kDefaultSMs;
+  }
+  int n = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return kDefaultSMs;
+  }
+  g_sm_count[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 // LSE outputs are written one float at a time: 4-byte alignment is enough.
@@ -78,7 +100,7 @@ bool valid_offsets(const int64_t* cu, int n, int64_t total) {
   return true;
 }
 
-int64_t varlen_target_ctas() { return int64_t{kSMs} * kDecodeCtasPerSM; }
+int64_t varlen_target_ctas() { return int64_t{sm_count()} * kDecodeCtasPerSM; }
 
 // Varlen decode workspace = [o_parts][lse_parts][counters: b * Hkv uint32], each
 // 256-B aligned; partial rows = the plan's splits.
@@ -162,13 +184,18 @@ std::atomic<uint64_t> g_launches{0};
 
 void count_launch(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
-SplitPlan decode_plan(const Shape& s) { return make_plan(s, int64_t{kSMs} * kDecodeCtasPerSM); }
+star_status_t check_shape(const star_attn_shape_t* shape) {
+  Shape s;
+  return resolve(shape, &s);
+}
+
+SplitPlan decode_plan(const Shape& s) { return make_plan(s, int64_t{sm_count()} * kDecodeCtasPerSM); }
 
 SplitPlan query_plan(const Shape& s, int64_t lq) {
   // One tensor-core CTA per SM, each taking two q-tiles; aim at about two waves
   // over (splits x pairs of q-tiles).
   const int64_t pairs = (query_tiles(s, lq) + 1) / 2;
-  return make_plan(s, 2 * int64_t{kSMs} / pairs);
+  return make_plan(s, 2 * int64_t{sm_count()} / pairs);
 }
 
 size_t partial_bytes(const Shape& s, const SplitPlan& p, int64_t rows) {
@@ -659,6 +686,17 @@ STAR_ATTN_API star_status_t star_attn_selftest_exp2(const float* x, float* y, in
   if (n < 0 || (n > 0 && (!x || !y))) return STAR_ERR_INVALID_ARG;
   return star::cuda_status(
       star::launch_selftest_exp2(x, y, n, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+STAR_ATTN_API star_status_t star_attn_selftest_read(const void* src, size_t bytes,
+                                                    uint32_t* sink, int32_t ctas,
+                                                    star_stream_t stream) {
+  if (!src || !sink || bytes == 0 || bytes % 16 != 0 || ctas < 1 || ctas > (1 << 20))
+    return STAR_ERR_INVALID_ARG;
+  if (!star::aligned16(src) || !star::aligned4(sink)) return STAR_ERR_INVALID_ARG;
+  if (bytes > (size_t{1} << 40)) return STAR_ERR_INVALID_ARG;
+  return star::cuda_status(star::launch_selftest_read(src, static_cast<int64_t>(bytes), sink, ctas,
+                                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 STAR_ATTN_API star_status_t star_attn_selftest_wait_timeout(uint64_t wait_ns,

@@ -191,6 +191,8 @@ cudaError_t launch_merge_varlen(const float* o_parts, const float* lse_parts, co
                                 cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t wait_ns, cudaStream_t st);
 cudaError_t launch_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t st);
+cudaError_t launch_selftest_read(const void* src, int64_t bytes, uint32_t* sink, int32_t ctas,
+                                 cudaStream_t st);
 
 // TMA descriptor encoding (host). Returns false if the driver entry point is
 // unavailable or the encode call rejects the arguments.

@@ -50,7 +50,51 @@ __global__ void selftest_exp2_kernel(const float* x, float* y, int64_t n) {
   }
 }
 
+// Reads every 16-byte word of src once (streaming loads that bypass L1) and
+// writes one XOR per CTA to sink, so that no load can be optimised away. A
+// measure of how fast this GPU streams bytes out of HBM when nothing is written
+// back: the ceiling for a kernel that only reads, such as the decode step.
+__global__ void __launch_bounds__(512) selftest_read_kernel(const uint4* src, int64_t n16,
+                                                            uint32_t* sink) {
+  constexpr int kUnroll = 4;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  uint32_t acc = 0;
+  for (; i + (kUnroll - 1) * stride < n16; i += kUnroll * stride) {
+    uint4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(v[u].x), "=r"(v[u].y), "=r"(v[u].z), "=r"(v[u].w)
+                   : "l"(src + i + u * stride));
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) acc ^= v[u].x ^ v[u].y ^ v[u].z ^ v[u].w;
+  }
+  for (; i < n16; i += stride) {
+    const uint4 v = src[i];
+    acc ^= v.x ^ v.y ^ v.z ^ v.w;
+  }
+  for (int o = 16; o >= 1; o >>= 1) acc ^= __shfl_xor_sync(0xffffffffu, acc, o);
+  __shared__ uint32_t warp_acc[16];
+  if ((threadIdx.x & 31) == 0) warp_acc[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t x = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) x ^= warp_acc[w];
+    sink[blockIdx.x] = x;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_selftest_read(const void* src, int64_t bytes, uint32_t* sink, int32_t ctas,
+                                 cudaStream_t st) {
+  if (bytes <= 0 || ctas <= 0) return cudaSuccess;
+  selftest_read_kernel<<<static_cast<unsigned>(ctas), 512, 0, st>>>(
+      static_cast<const uint4*>(src), bytes / 16, sink);
+  count_launch();
+  return cudaGetLastError();
+}
 
 cudaError_t launch_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;

@@ -427,6 +427,22 @@ STAR_ATTN_API star_status_t star_attn_selftest_exp2(const float* x, float* y, in
                                                     star_stream_t stream);
 
 /*
+ * Read-only streaming probe: reads every byte of `src` once (16-byte streaming
+ * loads that bypass L1), spread over `ctas` blocks of 512 threads, and writes one
+ * 32-bit XOR of the bytes each block read to sink[block] so that no load can be
+ * dropped. Timing it over a buffer much larger than L2 gives the rate at which
+ * this GPU reads HBM when nothing is written back, the ceiling of a read-only
+ * kernel such as the decode step (a copy-based bandwidth figure counts a read
+ * and a write per byte). Measurement infrastructure; no counterpart on the Star
+ * Attention pages.
+ * src: device, 16-byte aligned; bytes: a positive multiple of 16 (<= 2^40);
+ * sink: device array of `ctas` uint32 (4-byte aligned); ctas in [1, 2^20].
+ * Returns STAR_ERR_INVALID_ARG (nothing launched) otherwise.
+ */
+STAR_ATTN_API star_status_t star_attn_selftest_read(const void* src, size_t bytes, uint32_t* sink,
+                                                    int32_t ctas, star_stream_t stream);
+
+/*
  * Number of kernels this library has launched in this process (all devices).
  * A host-side counter for accounting, incremented at every successful launch.
  */

@@ -58,3 +58,63 @@ def test_noalloc_rejects_shapes_beyond_its_array():
     st = sa.lib().star_attn_phase2_decode_noalloc(ctypes.byref(shape), F, F, F, F, F, F, F, 0, 8,
                                                   F, None, None)
     assert st == 3  # STAR_ERR_WORKSPACE, nothing launched
+
+
+def test_noalloc_reports_unsupported_shapes_like_the_workspace_call():
+    import block_sparse_attention_phase_b200 as sa
+    # Shapes the library does not implement get STAR_ERR_UNSUPPORTED from both entry
+    # points (checked before any pointer is looked at, so nothing is launched).
+    F = ctypes.c_void_p(1 << 20)
+    for shape in (sa.make_shape(1, 4, 2, 96, 4096, 1024),    # head_dim 96
+                  sa.make_shape(1, 6, 2, 128, 4096, 1024)):  # GQA group of 3
+        st_ws = sa.lib().star_attn_phase2_decode(ctypes.byref(shape), F, F, F, F, F, F, F, 0, 8,
+                                                 F, None, F, 1 << 20, None)
+        st = sa.lib().star_attn_phase2_decode_noalloc(ctypes.byref(shape), F, F, F, F, F, F, F,
+                                                      0, 8, F, None, None)
+        assert st_ws == 2 and st == 2, (st_ws, st)  # STAR_ERR_UNSUPPORTED
+    bad = sa.make_shape(1, 4, 3, 128, 4096, 1024)  # Hq not a multiple of Hkv
+    st = sa.lib().star_attn_phase2_decode_noalloc(ctypes.byref(bad), F, F, F, F, F, F, F, 0, 8,
+                                                  F, None, None)
+    assert st == 1  # STAR_ERR_INVALID_ARG
+
+
+def test_noalloc_shape_that_just_fits_its_array():
+    """The largest block count whose partials still fit the 4 MiB array runs and
+    matches the workspace call (so the array's tail is in use); one block more is
+    refused with STAR_ERR_WORKSPACE."""
+    import block_sparse_attention_phase_b200 as sa
+    b, hq, hkv, d, B = 2, 32, 8, 128, 256
+    limit = 4 << 20
+    n = 1
+    while sa.workspace_bytes(sa.make_shape(b, hq, hkv, d, (n + 1) * B, B),
+                             sa.STAR_PHASE2_DECODE) <= limit:
+        n += 1
+    L = n * B
+    shape = sa.make_shape(b, hq, hkv, d, L, B)
+    need = sa.workspace_bytes(shape, sa.STAR_PHASE2_DECODE)
+    assert limit - 64 * 1024 < need <= limit, need
+    w = workloads.Workload("noalloc-edge", b, hq, hkv, d, L, B, 3, 1, 0, 5)
+    x = workloads.make_inputs(w, device="cuda")
+    cap = 8
+    kc_a = torch.zeros((b, cap, hkv, d), dtype=torch.bfloat16, device="cuda")
+    vc_a = torch.zeros_like(kc_a)
+    sa.phase2_query(x["q_qry"], x["k_qry"], x["v_qry"], x["k_ctx"], x["v_ctx"], kc_a, vc_a, B)
+    kc_b, vc_b = kc_a.clone(), vc_a.clone()
+    o_ref, l_ref = sa.phase2_decode(x["q_dec"][0], x["k_dec"][0], x["v_dec"][0], x["k_ctx"],
+                                    x["v_ctx"], kc_a, vc_a, 3, B)
+    o = torch.empty_like(o_ref)
+    lse = torch.empty_like(l_ref)
+    st = _call_noalloc(sa, shape, x["q_dec"][0], x["k_dec"][0], x["v_dec"][0], x["k_ctx"],
+                       x["v_ctx"], kc_b, vc_b, 3, o, lse)
+    assert st == 0, sa.STATUS_NAMES.get(st, st)
+    torch.cuda.synchronize()
+    check_rows(to_np(o), to_np(o_ref), to_np(lse), to_np(l_ref), "noalloc at the array's limit")
+    # same kernels, same split plan: the two calls agree exactly
+    assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
+    assert torch.equal(kc_a, kc_b) and torch.equal(vc_a, vc_b)
+    over = sa.make_shape(b, hq, hkv, d, L + B, B)
+    assert sa.workspace_bytes(over, sa.STAR_PHASE2_DECODE) > limit
+    st = _call_noalloc(sa, over, x["q_dec"][0], x["k_dec"][0], x["v_dec"][0], x["k_ctx"],
+                       x["v_ctx"], kc_b, vc_b, 3, o, lse)
+    assert st == 3  # STAR_ERR_WORKSPACE, nothing launched
+    assert sa.device_status() == 0
