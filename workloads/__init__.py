@@ -83,6 +83,24 @@ class Workload:
         return tok * self.head_dim * 2 * (2 * self.num_q_heads + 2 * self.num_kv_heads) + \
             tok * self.num_q_heads * 4
 
+    def query_flops(self) -> float:
+        """Algorithmic FLOPs of the Phase-2 query pass: query token j attends to all
+        L context keys and to query tokens 0..j (QK^T and PV multiply-adds x2)."""
+        lq = self.query_len
+        pairs = lq * self.ctx_len + lq * (lq + 1) // 2
+        return 4.0 * self.head_dim * self.num_q_heads * self.batch * pairs
+
+    def query_io_bytes(self) -> int:
+        """Bytes the query pass must move at least once: the context K/V read, the
+        query tokens' Q read, their K/V read and written into the cache, O and the
+        LSE written."""
+        b, lq, d = self.batch, self.query_len, self.head_dim
+        ctx = b * self.ctx_len * self.num_kv_heads * d * 2 * 2
+        q = b * lq * self.num_q_heads * d * 2
+        kv = b * lq * self.num_kv_heads * d * 2 * 2 * 2
+        out = b * lq * self.num_q_heads * (d * 2 + 4)
+        return ctx + q + kv + out
+
     def decode_kv_bytes(self, step: int) -> int:
         """KV bytes a decode step must read once: context + query tokens + decoded
         tokens so far (including the one appended this step), K and V, bf16."""
@@ -219,6 +237,32 @@ def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None,
                     out[qkey][p.batch, p.q_token, p.q_head] = qt.to(device)
             if "k_ctx" in out:
                 out["k_ctx"][p.batch, p.k_token, p.kv_head] = kt.to(device)
+    return out
+
+
+def make_head_slices(w: Workload, rows, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """The one-head slices a bounded CPU timing sample needs, drawn on the host
+    with the workload's distribution (N(0,1)/sqrt(d), rounded to bf16) from the
+    same per-tensor seeds, without materialising the whole batch x heads tensors:
+      q_ctx [L, d] (zero except at `rows`), k_ctx / v_ctx [L, d] (one kv-head),
+      q_qry / k_qry / v_qry [Lq, d], q_dec / k_dec / v_dec [d] (the first step),
+    as float32 arrays holding bf16 values. Planted pairs are left out (they do not
+    change how much work the oracle does). The values are not those of the GPU
+    arm's tensors (a host generator and a device generator draw different
+    streams); only shapes and distribution match."""
+    seed = w.seed if seed is None else seed
+    d, L = w.head_dim, w.ctx_len
+    rows = np.asarray(rows, dtype=np.int64)
+    f = lambda t: t.float().numpy()  # noqa: E731
+    q = np.zeros((L, d), dtype=np.float32)
+    q[rows] = f(_randn_bf16((len(rows), d), seed, "q_ctx", d, "cpu"))
+    out = {"q_ctx": q,
+           "k_ctx": f(_randn_bf16((L, d), seed, "k_ctx", d, "cpu")),
+           "v_ctx": f(_randn_bf16((L, d), seed, "v_ctx", d, "cpu"))}
+    for name in ("q_qry", "k_qry", "v_qry"):
+        out[name] = f(_randn_bf16((w.query_len, d), seed, name, d, "cpu"))
+    for name in ("q_dec", "k_dec", "v_dec"):
+        out[name] = f(_randn_bf16((d,), seed, name, d, "cpu"))
     return out
 
 
