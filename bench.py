@@ -75,21 +75,28 @@ def sources_sha256(kind: str) -> str:
 
 
 def recorded_traffic(kind: str, w, algorithmic_bytes: float):
-    """DRAM bytes per launch for this workload: the ncu figure if it was captured on
-    this workload, else the captured workload's bytes per algorithmic byte times
-    this workload's algorithmic bytes (both kernels move each byte once, so their
-    traffic grows in proportion). None when the kernel's sources changed since."""
+    """DRAM bytes per launch for this workload from the ncu captures whose kernel
+    sources are unchanged: the capture with this workload's block size (scaled by
+    algorithmic bytes to this context length: every block i > 0 reads the anchor
+    and its own block the same way, so traffic grows in proportion), else one of
+    the same workload. (None, reason) when no capture applies."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            entry = json.load(f)[kind]
+            entries = json.load(f)[kind]
     except Exception:
         return None, None
-    if entry.get("sources_sha256") != sources_sha256(kind):
+    entries = [e for e in entries if e.get("sources_sha256") == sources_sha256(kind)]
+    if not entries:
         return None, "kernel sources changed since the capture"
-    if entry.get("workload") == w.name:
-        return entry["dram_bytes_per_launch"], f"ncu on {w.name}"
-    ratio = entry["dram_bytes_per_launch"] / entry["algorithmic_bytes_per_launch"]
-    return ratio * algorithmic_bytes, f"scaled from the ncu capture on {entry.get('workload')}"
+    for e in entries:
+        if e.get("workload") == w.name:
+            return e["dram_bytes_per_launch"], f"ncu on {w.name}"
+    for e in entries:
+        if e.get("block_size") == w.block_size:
+            ratio = e["dram_bytes_per_launch"] / e["algorithmic_bytes_per_launch"]
+            return ratio * algorithmic_bytes, (f"ncu on {e['workload']} (same block size), scaled by "
+                                               f"algorithmic bytes ({ratio:.3f} x)")
+    return None, "no capture with this workload or block size"
 
 
 # ------------------------------------------------------------------ clocks
@@ -237,8 +244,7 @@ def read_peak_gbs(device, nbytes: int = 4 << 30, reps: int = 5):
     over a buffer far larger than L2 (best of `reps` launches, CUDA events): the
     ceiling of a kernel that only reads."""
     import block_sparse_attention_phase_b200 as sa
-    sms = torch.cuda.get_device_properties(device).multi_processor_count
-    ctas = sms * 4
+    ctas = torch.cuda.get_device_properties(device).multi_processor_count
     buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
     buf.fill_(7)
     sink = torch.empty(ctas, dtype=torch.int32, device=device)

@@ -47,26 +47,26 @@
 namespace star {
 namespace {
 
-// Threads per softmax row: 1 (a warpgroup per Q tile) or 2 (two warpgroups per Q
-// tile, each owning 64 of a row's 128 scores and d/2 of its output columns; the
-// two halves of a row trade their partial maxima through shared memory).
-#ifndef STAR_SOFTMAX_HALVES
-#define STAR_SOFTMAX_HALVES 1
+// Softmax layout. 0: warpgroup 1 takes Q tile 0 and warpgroup 2 Q tile 1, one
+// thread per row with all 128 scores of a K/V tile. 1 (column halves): each
+// warpgroup takes one half (64 columns) of both tiles' scores, the tiles in turn,
+// so that the two warps on an SMSP work on the same tile and a tile's softmax
+// takes about half as long; the two halves of a row trade their partial maxima
+// through shared memory.
+#ifndef STAR_SOFTMAX_COLHALVES
+#define STAR_SOFTMAX_COLHALVES 1
 #endif
-constexpr int kHalves = STAR_SOFTMAX_HALVES;
-static_assert(kHalves == 1 || kHalves == 2, "one or two threads per softmax row");
-constexpr int kThreads = 128 * (1 + 2 * kHalves);
+constexpr bool kColHalves = STAR_SOFTMAX_COLHALVES != 0;
+constexpr int kThreads = 384;
 constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle row each)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;          // lazy-rescale threshold (log2 units)
-// Register split. One thread per row: 384 threads launch with 168 registers
-// (64512); warpgroup 0 gives back down to 104, the two softmax warpgroups take 200.
-// Two per row: 640 threads launch with 96 (61440); warpgroup 0 drops to 56 and the
-// four softmax warpgroups take 104.
-constexpr int kLaunchRegs = kHalves == 1 ? 168 : 96;
-constexpr int kRegsLow = kHalves == 1 ? 104 : 56;
-constexpr int kRegsHigh = kHalves == 1 ? 200 : 104;
-static_assert(128 * kRegsLow + 256 * kHalves * kRegsHigh <= kThreads * kLaunchRegs, "register split");
+// Register split: 384 threads launch with 168 registers (64512); warpgroup 0
+// gives back down to 104, the two softmax warpgroups take 200.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsLow = 104;
+constexpr int kRegsHigh = 200;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
 static_assert(kThreads * kLaunchRegs <= 65536, "register file");
 // Of every 8 pairs of scores, this many take the FMA-pipe exponential; the MUFU
 // (16 results per clock per SM) would otherwise pace the softmax at the same
@@ -107,11 +107,10 @@ struct Bars {
   uint64_t o_bar[2];   // per Q tile: the last O_q += P V complete
   uint64_t drain;
   uint64_t q_free;     // the last anchor S MMAs are done: Q may be reloaded
-  uint64_t xchg[2][4]; // per Q tile and TMEM lane quarter: both halves posted a value
   uint32_t tmem_base;
   int abort;
-  float pmax[2][2][2][128];  // [tile][step parity][half][row] partial row maxima
-  float psum[2][2][128];     // [tile][half][row] partial row sums at the end
+  float pmax[2][2][2][128];  // column halves: [tile][step parity][half][row] partial row maxima
+  float psum[2][2][128];     // column halves: [tile][half][row] partial row sums at the end
 };
 
 // What one CTA computes.
@@ -363,9 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], 4 * kHalves);  // one arrival per softmax warp
-#pragma unroll
-      for (int w4 = 0; w4 < 4; ++w4) mbar_init(&bars->xchg[s][w4], 64);
+      mbar_init(&bars->p_full[s], kColHalves ? 8 : 4);  // one arrival per softmax warp
       mbar_init(&bars->o_bar[s], 1);
     }
     mbar_init(&bars->drain, 1);
@@ -549,157 +546,180 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
     // ------------------------------------------------------------ softmax warpgroups
     setmaxnreg_inc<kRegsHigh>();
     const int sw = wg - 1;
-    const int q = sw / kHalves;   // the Q tile this warpgroup works on
-    const int hf = sw % kHalves;  // which half of each row (with two threads per row)
-    constexpr int kCols = 128 / kHalves;  // scores per thread and tile
-    constexpr int kChunks = kCols / 32;
-    constexpr int kOCols = D / kHalves;   // output columns per thread
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    const uint32_t s_col = q * 128 + hf * kCols;     // this thread's scores
-    const uint32_t p_col = q * 128 + hf * kCols / 2; // its bf16 pairs of P
-    const uint32_t o_col = 256 + q * D + hf * kOCols;
-    uint64_t* xbar = &bars->xchg[q][q4];
-    // This tile's scalars (selected, so that Item stays in registers).
-    int64_t row_tok;  // Phase 1: context position of this row; query: query-token index
-    int head, rows_valid;
-    if constexpr (M == Mode::kPhase1) {
-      row_tok = (q ? it.t0[1] : it.t0[0]) + row;
-      head = q ? it.h[1] : it.h[0];
-      rows_valid = q ? it.rows_valid[1] : it.rows_valid[0];
-    } else {
-      row_tok = (q ? it.tok0[1] : it.tok0[0]) + row / a.G;
-      head = it.kvh * a.G + row % a.G;
-      rows_valid = 0;
-    }
+    // Layout: with column halves, warpgroup sw takes columns [64 sw, 64 sw + 64) of
+    // both Q tiles' scores (and d/2 output columns), the tiles in turn; otherwise
+    // warpgroup sw owns Q tile sw whole.
+    constexpr int kCols = kColHalves ? 64 : 128;  // scores per thread and tile
+    constexpr int kChunks = kCols / 32;
+    constexpr int kOCols = kColHalves ? D / 2 : D;  // output columns per thread
+    constexpr int kTilesPerWarp = kColHalves ? 2 : 1;
+    const int hf = kColHalves ? sw : 0;
     const float sl2 = a.scale_log2;
-    float m_run = -INFINITY;
-    float l_run = 0.f;
+    // This row's token and head in each of the warp's tiles (selected, so that Item
+    // stays in registers). Phase 1: context position; query: query-token index.
+    int64_t row_tok[kTilesPerWarp];
+    int head[kTilesPerWarp], rows_valid[kTilesPerWarp];
+#pragma unroll
+    for (int i = 0; i < kTilesPerWarp; ++i) {
+      const int q = kColHalves ? i : sw;
+      if constexpr (M == Mode::kPhase1) {
+        row_tok[i] = (q ? it.t0[1] : it.t0[0]) + row;
+        head[i] = q ? it.h[1] : it.h[0];
+        rows_valid[i] = q ? it.rows_valid[1] : it.rows_valid[0];
+      } else {
+        row_tok[i] = (q ? it.tok0[1] : it.tok0[0]) + row / a.G;
+        head[i] = it.kvh * a.G + row % a.G;
+        rows_valid[i] = 0;
+      }
+    }
+    float m_run[kTilesPerWarp], l_run[kTilesPerWarp];
+#pragma unroll
+    for (int i = 0; i < kTilesPerWarp; ++i) {
+      m_run[i] = -INFINITY;
+      l_run[i] = 0.f;
+    }
+    // The two warps holding the two halves of the same 32 rows meet on named barrier
+    // 1 + q4 (64 threads). Both take every barrier of the loop even after a wait has
+    // given up, so neither can be left waiting for the other.
+    auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(1 + q4) : "memory"); };
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      // Waits are per thread; the tcgen05 loads/stores below are warp-wide, so
-      // the warp proceeds only if every lane's wait succeeded.
-      ok = __all_sync(0xffffffffu, wait_or_abort(&bars->s_full[q], j & 1, bars, a.status));
-      if (!ok) break;
-      tc_fence_after();
-      const int limit = visible_prefix<M>(it, a, row_tok, j) - hf * kCols;  // in this half
-      // Most tiles are fully visible: mask only when some row of the warp needs it.
-      const bool masked = __any_sync(0xffffffffu, limit < kCols);
-      // S in pieces of 32: the max over the first pieces overlaps the TMEM read of
-      // the later ones. Row max with independent 3-input max chains.
-      uint32_t sr[kChunks][32];
-      float mc[kChunks];
-      tmem_ld32(lane_addr + s_col, sr[0]);
-      tmem_ld32(lane_addr + s_col + 32, sr[1]);
-      tmem_wait_ld();
-      if constexpr (kChunks == 4) {
-        tmem_ld32(lane_addr + s_col + 64, sr[2 % kChunks]);
-        tmem_ld32(lane_addr + s_col + 96, sr[3 % kChunks]);
-      }
 #pragma unroll
-      for (int half = 0; half < kChunks / 2; ++half) {
-        if (half == 1) tmem_wait_ld();
-#pragma unroll
-        for (int c = 2 * half; c < 2 * half + 2; ++c) {
-          if (masked) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (c * 32 + e >= limit) sr[c][e] = __float_as_uint(-INFINITY);
-          }
-          mc[c] = fmaxf(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]));
-#pragma unroll
-          for (int e = 2; e < 32; e += 2)
-            mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
-        }
-      }
-      float mt = fmaxf(mc[0], mc[1]);
-      if constexpr (kChunks == 4) mt = fmaxf(mt, fmaxf(mc[2 % kChunks], mc[3 % kChunks]));
-      if constexpr (kHalves == 2) {
-        // Trade partial maxima with the other half of the row. Both halves have
-        // their scores in registers before either arrives, so P (which the halves
-        // write over S's first 64 columns) cannot overwrite unread scores.
-        bars->pmax[q][j & 1][hf][row] = mt;
-        mbar_arrive(xbar);
-        ok = __all_sync(0xffffffffu, wait_or_abort(xbar, j & 1, bars, a.status));
-        if (!ok) break;
-        mt = fmaxf(mt, bars->pmax[q][j & 1][hf ^ 1][row]);
-      }
-      const bool need = (m_run == -INFINITY) || ((mt - m_run) * sl2 > kRescaleLog2);
-      const float m_new = need ? mt : m_run;
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;  // a row with nothing visible yet
-      const float alpha = need ? ex2_approx((m_run - m_use) * sl2) : 1.f;
-      m_run = m_new;
-      const float ms = m_use * sl2;
-      // p = 2^(s * scale * log2(e) - m'), two lanes per packed fp32 FMA / add.
-      const float2 sl2v = make_float2(sl2, sl2);
-      const float2 nms = make_float2(-ms, -ms);
-      float2 ps[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int c = 0; c < kChunks; ++c) {
-        // Chunk c (32 scores) -> 16 bf16 pairs, stored to TMEM at once (S is all
-        // in registers already), so few P words are ever live.
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float2 x = ffma2(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])),
-                                 sl2v, nms);
-          float p0, p1;
-          if (((e >> 1) & 7) < kPolyPairs) {
-            // a share of the exponentials on the FMA pipe, the rest on the MUFU
-            const float2 pp = exp2_poly2(x);
-            p0 = pp.x;
-            p1 = pp.y;
-          } else {
-            p0 = ex2_approx(x.x);
-            p1 = ex2_approx(x.y);
-          }
-          ps[(e >> 1) & 1] = fadd2(ps[(e >> 1) & 1], make_float2(p0, p1));
-          pk[e / 2] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(lane_addr + p_col + c * 16, pk);
-      }
-      const float psum = (ps[0].x + ps[0].y) + (ps[1].x + ps[1].y);
-      l_run = l_run * alpha + psum;
-      // S_q(j) complete implies O_q += P_q(j-1) V complete: O may be rescaled now.
-      if (j >= 1 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
-        for (int c = 0; c < kOCols / 32; ++c) {
-          uint32_t ob[32];
-          tmem_ld32(lane_addr + o_col + c * 32, ob);
+      for (int i = 0; i < kTilesPerWarp; ++i) {
+        const int q = kColHalves ? i : sw;
+        const uint32_t s_col = q * 128 + hf * kCols;      // this thread's scores
+        const uint32_t p_col = q * 128 + hf * kCols / 2;  // its bf16 pairs of P
+        const uint32_t o_col = 256 + q * D + hf * kOCols;
+        // Waits are per thread; the tcgen05 loads/stores below are warp-wide, so
+        // the warp proceeds only if every lane's wait succeeded.
+        if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&bars->s_full[q], j & 1, bars, a.status));
+        uint32_t sr[kChunks][32];
+        float mt = -INFINITY;
+        if (ok) {
+          tc_fence_after();
+          const int limit = visible_prefix<M>(it, a, row_tok[i], j) - hf * kCols;  // in this half
+          // Most tiles are fully visible: mask only when some row of the warp needs it.
+          const bool masked = __any_sync(0xffffffffu, limit < kCols);
+          // S in pieces of 32: the max over the first pieces overlaps the TMEM read of
+          // the later ones. Row max with independent 3-input max chains.
+          float mc[kChunks];
+          tmem_ld32(lane_addr + s_col, sr[0]);
+          tmem_ld32(lane_addr + s_col + 32, sr[1]);
           tmem_wait_ld();
+          if constexpr (kChunks == 4) {
+            tmem_ld32(lane_addr + s_col + 64, sr[2 % kChunks]);
+            tmem_ld32(lane_addr + s_col + 96, sr[3 % kChunks]);
+          }
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * alpha);
-          tmem_st32(lane_addr + o_col + c * 32, ob);
+          for (int half = 0; half < kChunks / 2; ++half) {
+            if (half == 1) tmem_wait_ld();
+#pragma unroll
+            for (int c = 2 * half; c < 2 * half + 2; ++c) {
+              if (masked) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  if (c * 32 + e >= limit) sr[c][e] = __float_as_uint(-INFINITY);
+              }
+              mc[c] = fmaxf(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]));
+#pragma unroll
+              for (int e = 2; e < 32; e += 2)
+                mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+            }
+          }
+          mt = fmaxf(mc[0], mc[1]);
+          if constexpr (kChunks == 4) mt = fmaxf(mt, fmaxf(mc[2 % kChunks], mc[3 % kChunks]));
         }
+        if constexpr (kColHalves) {
+          // Trade partial maxima with the other half of the row. Both halves have
+          // their scores in registers before either passes the barrier, so P (which
+          // the halves write over S's first 64 columns) cannot overwrite unread scores.
+          bars->pmax[q][j & 1][hf][row] = mt;
+          pair_sync();
+          mt = fmaxf(mt, bars->pmax[q][j & 1][hf ^ 1][row]);
+        }
+        if (!ok) continue;
+        const bool need = (m_run[i] == -INFINITY) || ((mt - m_run[i]) * sl2 > kRescaleLog2);
+        const float m_new = need ? mt : m_run[i];
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;  // a row with nothing visible yet
+        const float alpha = need ? ex2_approx((m_run[i] - m_use) * sl2) : 1.f;
+        m_run[i] = m_new;
+        const float ms = m_use * sl2;
+        // p = 2^(s * scale * log2(e) - m'), two lanes per packed fp32 FMA / add.
+        const float2 sl2v = make_float2(sl2, sl2);
+        const float2 nms = make_float2(-ms, -ms);
+        float2 ps[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          // Chunk c (32 scores) -> 16 bf16 pairs, stored to TMEM at once (S is all
+          // in registers already), so few P words are ever live.
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float2 x = ffma2(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])),
+                                   sl2v, nms);
+            float p0, p1;
+            if (((e >> 1) & 7) < kPolyPairs) {
+              // a share of the exponentials on the FMA pipe, the rest on the MUFU
+              const float2 pp = exp2_poly2(x);
+              p0 = pp.x;
+              p1 = pp.y;
+            } else {
+              p0 = ex2_approx(x.x);
+              p1 = ex2_approx(x.y);
+            }
+            ps[(e >> 1) & 1] = fadd2(ps[(e >> 1) & 1], make_float2(p0, p1));
+            pk[e / 2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(lane_addr + p_col + c * 16, pk);
+        }
+        const float psum = (ps[0].x + ps[0].y) + (ps[1].x + ps[1].y);
+        l_run[i] = l_run[i] * alpha + psum;
+        // S_q(j) complete implies O_q += P_q(j-1) V complete: O may be rescaled now.
+        if (j >= 1 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int c = 0; c < kOCols / 32; ++c) {
+            uint32_t ob[32];
+            tmem_ld32(lane_addr + o_col + c * 32, ob);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * alpha);
+            tmem_st32(lane_addr + o_col + c * 32, ob);
+          }
+        }
+        // Every lane's P (and O rescale) stores are complete; one lane per warp tells
+        // the MMA thread (32x fewer arrivals on the barrier than one per thread).
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[q]);
       }
-      // Every lane's P (and O rescale) stores are complete; one lane per warp tells
-      // the MMA thread (32x fewer arrivals on the barrier than one per thread).
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[q]);
     }
-    if constexpr (kHalves == 2) {
+    if constexpr (kColHalves) {
       // The row sum is the two halves' sums (same running max in both).
-      if (ok) {
-        bars->psum[q][hf][row] = l_run;
-        mbar_arrive(xbar);
-        ok = __all_sync(0xffffffffu, wait_or_abort(xbar, n_tiles & 1, bars, a.status));
-        if (ok) l_run += bars->psum[q][hf ^ 1][row];
-      }
+#pragma unroll
+      for (int i = 0; i < kTilesPerWarp; ++i) bars->psum[i][hf][row] = l_run[i];
+      pair_sync();
+#pragma unroll
+      for (int i = 0; i < kTilesPerWarp; ++i) l_run[i] += bars->psum[i][hf ^ 1][row];
     }
-    if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&bars->o_bar[q], 0, bars, a.status));
-    tc_fence_after();
-    if (ok) {
-      const bool has = l_run > 0.f;
-      const float inv = has ? 1.f / l_run : 0.f;
-      const float lse2 = has ? m_run * sl2 + log2f(l_run) : -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kTilesPerWarp; ++i) {
+      const int q = kColHalves ? i : sw;
+      const uint32_t o_col = 256 + q * D + hf * kOCols;
+      if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&bars->o_bar[q], 0, bars, a.status));
+      tc_fence_after();
+      if (!ok) continue;
+      const bool has = l_run[i] > 0.f;
+      const float inv = has ? 1.f / l_run[i] : 0.f;
+      const float lse2 = has ? m_run[i] * sl2 + log2f(l_run[i]) : -INFINITY;
       if constexpr (M == Mode::kPhase1) {
-        const int64_t t = row_tok;
-        const bool valid = row < rows_valid;
+        const int64_t t = row_tok[i];
+        const bool valid = row < rows_valid[i];
         // uniform: row bb * L + t of [b, L, Hq, d]; varlen: row tok_base + t of [total, Hq, d]
-        __nv_bfloat16* dst = a.o + ((static_cast<int64_t>(it.bb) * a.L + it.tok_base + t) * a.hq + head) * D +
+        __nv_bfloat16* dst = a.o + ((static_cast<int64_t>(it.bb) * a.L + it.tok_base + t) * a.hq + head[i]) * D +
                              hf * kOCols;
 #pragma unroll
         for (int c = 0; c < kOCols / 32; ++c) {
@@ -718,11 +738,11 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
           }
         }
         if (a.lse && valid && hf == 0)
-          a.lse[(static_cast<int64_t>(it.bb) * a.hq + head) * a.L + it.tok_base + t] =
+          a.lse[(static_cast<int64_t>(it.bb) * a.hq + head[i]) * a.L + it.tok_base + t] =
               lse2 * 0.69314718055994531f;
       } else {
-        const int tok = static_cast<int>(row_tok);
-        const int hq = head;
+        const int tok = static_cast<int>(row_tok[i]);
+        const int hq = head[i];
         const bool valid = tok < it.lq;
         float* dst = a.o_parts + ((it.rbase + tok) * a.hq + hq) * D + hf * kOCols;
 #pragma unroll

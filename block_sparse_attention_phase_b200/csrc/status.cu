@@ -50,39 +50,54 @@ __global__ void selftest_exp2_kernel(const float* x, float* y, int64_t n) {
   }
 }
 
-// Reads every 16-byte word of src once (streaming loads that bypass L1) and
-// writes one XOR per CTA to sink, so that no load can be optimised away. A
+// Reads every byte of src once with 1-D bulk asynchronous copies (the copy engine
+// the attention kernels stream K/V with) into a ring of shared-memory buffers, and
+// writes one XOR per CTA of the first word of every chunk it received to sink. A
 // measure of how fast this GPU streams bytes out of HBM when nothing is written
 // back: the ceiling for a kernel that only reads, such as the decode step.
-__global__ void __launch_bounds__(512) selftest_read_kernel(const uint4* src, int64_t n16,
-                                                            uint32_t* sink) {
-  constexpr int kUnroll = 4;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+constexpr int kReadStages = 4;
+constexpr uint32_t kReadChunk = 32768;
+
+__global__ void __launch_bounds__(32) selftest_read_kernel(const uint8_t* src, int64_t bytes,
+                                                           uint32_t* sink, uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* buf = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                            ~uintptr_t(127));
+  __shared__ alignas(8) uint64_t full[kReadStages];
+  if (threadIdx.x != 0) return;
+  for (int s = 0; s < kReadStages; ++s) mbar_init(&full[s], 1);
+  fence_barrier_init();
+  const int64_t n_chunks = (bytes + kReadChunk - 1) / kReadChunk;
+  auto issue = [&](int64_t c, int s) {
+    const int64_t off = c * kReadChunk;
+    const uint32_t n = static_cast<uint32_t>(bytes - off < kReadChunk ? bytes - off : kReadChunk);
+    mbar_arrive_expect_tx(&full[s], n);
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(buf + s * kReadChunk)),
+        "l"(src + off), "r"(n), "r"(smem_u32(&full[s]))
+        : "memory");
+  };
+  // Chunk i of this CTA is blockIdx.x + i * gridDim.x, in stage i % kReadStages.
+  const int64_t mine = blockIdx.x < n_chunks ? (n_chunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  for (int64_t i = 0; i < kReadStages && i < mine; ++i)
+    issue(blockIdx.x + i * gridDim.x, static_cast<int>(i));
   uint32_t acc = 0;
-  for (; i + (kUnroll - 1) * stride < n16; i += kUnroll * stride) {
-    uint4 v[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u)
-      asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                   : "=r"(v[u].x), "=r"(v[u].y), "=r"(v[u].z), "=r"(v[u].w)
-                   : "l"(src + i + u * stride));
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) acc ^= v[u].x ^ v[u].y ^ v[u].z ^ v[u].w;
+  int64_t i = 0;
+  for (; i < mine; ++i) {
+    const int s = static_cast<int>(i % kReadStages);
+    if (!mbar_wait(&full[s], static_cast<uint32_t>((i / kReadStages) & 1), status)) break;
+    acc ^= *reinterpret_cast<const uint32_t*>(buf + s * kReadChunk);
+    if (i + kReadStages < mine) {
+      fence_proxy_async_smem();  // the read above precedes the copy that overwrites the buffer
+      issue(blockIdx.x + (i + kReadStages) * gridDim.x, s);
+    }
   }
-  for (; i < n16; i += stride) {
-    const uint4 v = src[i];
-    acc ^= v.x ^ v.y ^ v.z ^ v.w;
-  }
-  for (int o = 16; o >= 1; o >>= 1) acc ^= __shfl_xor_sync(0xffffffffu, acc, o);
-  __shared__ uint32_t warp_acc[16];
-  if ((threadIdx.x & 31) == 0) warp_acc[threadIdx.x >> 5] = acc;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    uint32_t x = 0;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) x ^= warp_acc[w];
-    sink[blockIdx.x] = x;
-  }
+  // After a wait gave up, the copies still in flight land before the CTA exits
+  // (each wait bounded again).
+  for (int64_t k = i; k < mine && k < i + kReadStages; ++k)
+    mbar_wait(&full[k % kReadStages], static_cast<uint32_t>((k / kReadStages) & 1), status);
+  sink[blockIdx.x] = acc;
 }
 
 }  // namespace
@@ -90,8 +105,15 @@ __global__ void __launch_bounds__(512) selftest_read_kernel(const uint4* src, in
 cudaError_t launch_selftest_read(const void* src, int64_t bytes, uint32_t* sink, int32_t ctas,
                                  cudaStream_t st) {
   if (bytes <= 0 || ctas <= 0) return cudaSuccess;
-  selftest_read_kernel<<<static_cast<unsigned>(ctas), 512, 0, st>>>(
-      static_cast<const uint4*>(src), bytes / 16, sink);
+  uint32_t* status = device_status_word();
+  if (!status) return cudaErrorInvalidDevice;
+  const size_t smem = size_t{kReadStages} * kReadChunk + 128;
+  cudaError_t e = cudaFuncSetAttribute(selftest_read_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  selftest_read_kernel<<<static_cast<unsigned>(ctas), 32, smem, st>>>(
+      static_cast<const uint8_t*>(src), bytes, sink, status);
   count_launch();
   return cudaGetLastError();
 }

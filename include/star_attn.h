@@ -427,10 +427,11 @@ STAR_ATTN_API star_status_t star_attn_selftest_exp2(const float* x, float* y, in
                                                     star_stream_t stream);
 
 /*
- * Read-only streaming probe: reads every byte of `src` once (16-byte streaming
- * loads that bypass L1), spread over `ctas` blocks of 512 threads, and writes one
- * 32-bit XOR of the bytes each block read to sink[block] so that no load can be
- * dropped. Timing it over a buffer much larger than L2 gives the rate at which
+ * Read-only streaming probe: reads every byte of `src` once with 1-D bulk
+ * asynchronous copies (32 KB chunks, four in flight per block) into shared
+ * memory, spread over `ctas` blocks of one warp (one block per SM is enough), and
+ * writes one 32-bit XOR of the first word of each chunk a block received to
+ * sink[block]. Timing it over a buffer much larger than L2 gives the rate at which
  * this GPU reads HBM when nothing is written back, the ceiling of a read-only
  * kernel such as the decode step (a copy-based bandwidth figure counts a read
  * and a write per byte). Measurement infrastructure; no counterpart on the Star

@@ -137,6 +137,23 @@ def test_fma_pipe_exp2_accuracy():
     assert torch.isfinite(lo).all() and (lo >= 0).all() and (lo < 1.2e-38).all()
 
 
+@pytest.mark.parametrize("nbytes,ctas", [(16, 1), (32768 * 5 + 48, 2), (32768 * 37, 3),
+                                         (32768 * 64 - 16, 148)])
+def test_read_probe_reads_every_chunk(nbytes, ctas):
+    """The read-only bandwidth probe visits every 32 KB chunk (block b takes chunks
+    b, b + ctas, ...; a short last chunk included): each block's XOR of its
+    chunks' first words matches the host's."""
+    g = torch.Generator().manual_seed(nbytes)
+    words = torch.randint(0, 2 ** 31 - 1, (nbytes // 4,), generator=g, dtype=torch.int32)
+    sink = torch.full((ctas,), -1, dtype=torch.int32, device="cuda")
+    sa().selftest_read(words.cuda(), sink, ctas)
+    assert sa().device_status() == 0
+    first = words[::32768 // 4].numpy()  # first word of every chunk
+    want = [int(np.bitwise_xor.reduce(first[b::ctas])) if b < len(first) else 0
+            for b in range(ctas)]
+    assert sink.cpu().numpy().tolist() == want
+
+
 def test_wait_timeout_is_reported_not_trapped():
     m = sa()
     assert m.device_status() == 0
