@@ -47,26 +47,31 @@
 namespace star {
 namespace {
 
-// Softmax layout. 0: warpgroup 1 takes Q tile 0 and warpgroup 2 Q tile 1, one
-// thread per row with all 128 scores of a K/V tile. 1 (column halves): each
-// warpgroup takes one half (64 columns) of both tiles' scores, the tiles in turn,
-// so that the two warps on an SMSP work on the same tile and a tile's softmax
-// takes about half as long; the two halves of a row trade their partial maxima
-// through shared memory.
-#ifndef STAR_SOFTMAX_COLHALVES
-#define STAR_SOFTMAX_COLHALVES 1
+// Softmax layout: the number of parts each tile's 128 key columns are split into.
+// 1: warpgroup 1 takes Q tile 0 and warpgroup 2 Q tile 1, one thread per row with
+// all 128 scores of a K/V tile. 2 or 4: each of 2 or 4 softmax warpgroups takes
+// one part (64 or 32 columns) of both tiles' scores, the tiles in turn, so that
+// all softmax warps of an SMSP work on the same tile and a tile's softmax takes
+// less time; the parts of a row trade their partial maxima through shared memory.
+#ifndef STAR_SOFTMAX_PARTS
+#define STAR_SOFTMAX_PARTS 2
 #endif
-constexpr bool kColHalves = STAR_SOFTMAX_COLHALVES != 0;
-constexpr int kThreads = 384;
+constexpr int kParts = STAR_SOFTMAX_PARTS;
+static_assert(kParts == 1 || kParts == 2 || kParts == 4, "softmax parts: 1, 2 or 4");
+constexpr int kSoftmaxWarpgroups = kParts == 4 ? 4 : 2;
+constexpr int kThreads = 128 * (1 + kSoftmaxWarpgroups);
 constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle row each)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;          // lazy-rescale threshold (log2 units)
-// Register split: 384 threads launch with 168 registers (64512); warpgroup 0
-// gives back down to 104, the two softmax warpgroups take 200.
-constexpr int kLaunchRegs = 168;
-constexpr int kRegsLow = 104;
-constexpr int kRegsHigh = 200;
-static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
+// Register split. Two softmax warpgroups: 384 threads launch with 168 registers
+// (64512); warpgroup 0 gives back down to 104, the softmax warpgroups take 200.
+// Four: 640 threads launch with 96 (61440); warpgroup 0 drops to 56 and the
+// softmax warpgroups take 104.
+constexpr int kLaunchRegs = kSoftmaxWarpgroups == 2 ? 168 : 96;
+constexpr int kRegsLow = kSoftmaxWarpgroups == 2 ? 104 : 56;
+constexpr int kRegsHigh = kSoftmaxWarpgroups == 2 ? 200 : 104;
+static_assert(128 * kRegsLow + 128 * kSoftmaxWarpgroups * kRegsHigh <= kThreads * kLaunchRegs,
+              "register split");
 static_assert(kThreads * kLaunchRegs <= 65536, "register file");
 // Of every 8 pairs of scores, this many take the FMA-pipe exponential; the MUFU
 // (16 results per clock per SM) would otherwise pace the softmax at the same
@@ -109,8 +114,8 @@ struct Bars {
   uint64_t q_free;     // the last anchor S MMAs are done: Q may be reloaded
   uint32_t tmem_base;
   int abort;
-  float pmax[2][2][2][128];  // column halves: [tile][step parity][half][row] partial row maxima
-  float psum[2][2][128];     // column halves: [tile][half][row] partial row sums at the end
+  float pmax[2][2][kParts][128];  // split columns: [tile][step parity][part][row] partial row maxima
+  float psum[2][kParts][128];     // split columns: [tile][part][row] partial row sums at the end
 };
 
 // What one CTA computes.
@@ -362,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], kColHalves ? 8 : 4);  // one arrival per softmax warp
+      mbar_init(&bars->p_full[s], 4 * kSoftmaxWarpgroups);  // one arrival per softmax warp
       mbar_init(&bars->o_bar[s], 1);
     }
     mbar_init(&bars->drain, 1);
@@ -549,14 +554,16 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    // Layout: with column halves, warpgroup sw takes columns [64 sw, 64 sw + 64) of
-    // both Q tiles' scores (and d/2 output columns), the tiles in turn; otherwise
-    // warpgroup sw owns Q tile sw whole.
-    constexpr int kCols = kColHalves ? 64 : 128;  // scores per thread and tile
-    constexpr int kChunks = kCols / 32;
-    constexpr int kOCols = kColHalves ? D / 2 : D;  // output columns per thread
-    constexpr int kTilesPerWarp = kColHalves ? 2 : 1;
-    const int hf = kColHalves ? sw : 0;
+    // Layout: with the columns split (kParts > 1), warpgroup sw takes columns
+    // [sw * 128 / kParts, (sw + 1) * 128 / kParts) of both Q tiles' scores (and D /
+    // kParts output columns), the tiles in turn; with kParts = 1 warpgroup sw owns
+    // Q tile sw whole.
+    constexpr int kCols = 128 / kParts;         // scores per thread and tile
+    constexpr int kChunks = kCols / 32;         // 32-column pieces of them
+    constexpr int kOCols = D / kParts;          // output columns per thread
+    constexpr int kOP = kOCols < 32 ? kOCols : 32;  // output columns per TMEM access
+    constexpr int kTilesPerWarp = kParts > 1 ? 2 : 1;
+    const int part = kParts > 1 ? sw : 0;
     const float sl2 = a.scale_log2;
     // This row's token and head in each of the warp's tiles (selected, so that Item
     // stays in registers). Phase 1: context position; query: query-token index.
@@ -564,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
     int head[kTilesPerWarp], rows_valid[kTilesPerWarp];
 #pragma unroll
     for (int i = 0; i < kTilesPerWarp; ++i) {
-      const int q = kColHalves ? i : sw;
+      const int q = kParts > 1 ? i : sw;
       if constexpr (M == Mode::kPhase1) {
         row_tok[i] = (q ? it.t0[1] : it.t0[0]) + row;
         head[i] = q ? it.h[1] : it.h[0];
@@ -581,18 +588,18 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       m_run[i] = -INFINITY;
       l_run[i] = 0.f;
     }
-    // The two warps holding the two halves of the same 32 rows meet on named barrier
-    // 1 + q4 (64 threads). Both take every barrier of the loop even after a wait has
-    // given up, so neither can be left waiting for the other.
-    auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(1 + q4) : "memory"); };
+    // The kParts warps holding the parts of the same 32 rows meet on named barrier
+    // 1 + q4. All of them take every barrier of the loop even after a wait has given
+    // up, so none can be left waiting for another.
+    auto parts_sync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + q4), "n"(32 * kParts) : "memory"); };
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
 #pragma unroll
       for (int i = 0; i < kTilesPerWarp; ++i) {
-        const int q = kColHalves ? i : sw;
-        const uint32_t s_col = q * 128 + hf * kCols;      // this thread's scores
-        const uint32_t p_col = q * 128 + hf * kCols / 2;  // its bf16 pairs of P
-        const uint32_t o_col = 256 + q * D + hf * kOCols;
+        const int q = kParts > 1 ? i : sw;
+        const uint32_t s_col = q * 128 + part * kCols;      // this thread's scores
+        const uint32_t p_col = q * 128 + part * kCols / 2;  // its bf16 pairs of P
+        const uint32_t o_col = 256 + q * D + part * kOCols;
         // Waits are per thread; the tcgen05 loads/stores below are warp-wide, so
         // the warp proceeds only if every lane's wait succeeded.
         if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&bars->s_full[q], j & 1, bars, a.status));
@@ -600,45 +607,44 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         float mt = -INFINITY;
         if (ok) {
           tc_fence_after();
-          const int limit = visible_prefix<M>(it, a, row_tok[i], j) - hf * kCols;  // in this half
+          const int limit = visible_prefix<M>(it, a, row_tok[i], j) - part * kCols;  // in this part
           // Most tiles are fully visible: mask only when some row of the warp needs it.
           const bool masked = __any_sync(0xffffffffu, limit < kCols);
           // S in pieces of 32: the max over the first pieces overlaps the TMEM read of
           // the later ones. Row max with independent 3-input max chains.
           float mc[kChunks];
           tmem_ld32(lane_addr + s_col, sr[0]);
-          tmem_ld32(lane_addr + s_col + 32, sr[1]);
+          if constexpr (kChunks >= 2) tmem_ld32(lane_addr + s_col + 32, sr[1 % kChunks]);
           tmem_wait_ld();
           if constexpr (kChunks == 4) {
             tmem_ld32(lane_addr + s_col + 64, sr[2 % kChunks]);
             tmem_ld32(lane_addr + s_col + 96, sr[3 % kChunks]);
           }
 #pragma unroll
-          for (int half = 0; half < kChunks / 2; ++half) {
-            if (half == 1) tmem_wait_ld();
+          for (int c = 0; c < kChunks; ++c) {
+            if (c == 2) tmem_wait_ld();
+            if (masked) {
 #pragma unroll
-            for (int c = 2 * half; c < 2 * half + 2; ++c) {
-              if (masked) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  if (c * 32 + e >= limit) sr[c][e] = __float_as_uint(-INFINITY);
-              }
-              mc[c] = fmaxf(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]));
-#pragma unroll
-              for (int e = 2; e < 32; e += 2)
-                mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+              for (int e = 0; e < 32; ++e)
+                if (c * 32 + e >= limit) sr[c][e] = __float_as_uint(-INFINITY);
             }
+            mc[c] = fmaxf(__uint_as_float(sr[c][0]), __uint_as_float(sr[c][1]));
+#pragma unroll
+            for (int e = 2; e < 32; e += 2)
+              mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
           }
-          mt = fmaxf(mc[0], mc[1]);
-          if constexpr (kChunks == 4) mt = fmaxf(mt, fmaxf(mc[2 % kChunks], mc[3 % kChunks]));
+          mt = mc[0];
+#pragma unroll
+          for (int c = 1; c < kChunks; ++c) mt = fmaxf(mt, mc[c]);
         }
-        if constexpr (kColHalves) {
-          // Trade partial maxima with the other half of the row. Both halves have
-          // their scores in registers before either passes the barrier, so P (which
-          // the halves write over S's first 64 columns) cannot overwrite unread scores.
-          bars->pmax[q][j & 1][hf][row] = mt;
-          pair_sync();
-          mt = fmaxf(mt, bars->pmax[q][j & 1][hf ^ 1][row]);
+        if constexpr (kParts > 1) {
+          // Trade partial maxima with the other parts of the row. Every part has its
+          // scores in registers before any passes the barrier, so P (which the parts
+          // write over S's first 64 columns) cannot overwrite unread scores.
+          bars->pmax[q][j & 1][part][row] = mt;
+          parts_sync();
+#pragma unroll
+          for (int o = 1; o < kParts; ++o) mt = fmaxf(mt, bars->pmax[q][j & 1][(part + o) % kParts][row]);
         }
         if (!ok) continue;
         const bool need = (m_run[i] == -INFINITY) || ((mt - m_run[i]) * sl2 > kRescaleLog2);
@@ -680,13 +686,22 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         // S_q(j) complete implies O_q += P_q(j-1) V complete: O may be rescaled now.
         if (j >= 1 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
-          for (int c = 0; c < kOCols / 32; ++c) {
-            uint32_t ob[32];
-            tmem_ld32(lane_addr + o_col + c * 32, ob);
-            tmem_wait_ld();
+          for (int c = 0; c < kOCols / kOP; ++c) {
+            if constexpr (kOP == 32) {
+              uint32_t ob[32];
+              tmem_ld32(lane_addr + o_col + c * 32, ob);
+              tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * alpha);
-            tmem_st32(lane_addr + o_col + c * 32, ob);
+              for (int e = 0; e < 32; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * alpha);
+              tmem_st32(lane_addr + o_col + c * 32, ob);
+            } else {
+              uint32_t ob[16];
+              tmem_ld16(lane_addr + o_col + c * 16, ob);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * alpha);
+              tmem_st16(lane_addr + o_col + c * 16, ob);
+            }
           }
         }
         // Every lane's P (and O rescale) stores are complete; one lane per warp tells
@@ -697,68 +712,74 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         if (lane == 0) mbar_arrive(&bars->p_full[q]);
       }
     }
-    if constexpr (kColHalves) {
-      // The row sum is the two halves' sums (same running max in both).
+    if constexpr (kParts > 1) {
+      // The row sum is the parts' sums (same running max in all of them).
 #pragma unroll
-      for (int i = 0; i < kTilesPerWarp; ++i) bars->psum[i][hf][row] = l_run[i];
-      pair_sync();
+      for (int i = 0; i < kTilesPerWarp; ++i) bars->psum[i][part][row] = l_run[i];
+      parts_sync();
 #pragma unroll
-      for (int i = 0; i < kTilesPerWarp; ++i) l_run[i] += bars->psum[i][hf ^ 1][row];
+      for (int i = 0; i < kTilesPerWarp; ++i)
+#pragma unroll
+        for (int o = 1; o < kParts; ++o) l_run[i] += bars->psum[i][(part + o) % kParts][row];
     }
 #pragma unroll
     for (int i = 0; i < kTilesPerWarp; ++i) {
-      const int q = kColHalves ? i : sw;
-      const uint32_t o_col = 256 + q * D + hf * kOCols;
+      const int q = kParts > 1 ? i : sw;
+      const uint32_t o_col = 256 + q * D + part * kOCols;
       if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&bars->o_bar[q], 0, bars, a.status));
       tc_fence_after();
       if (!ok) continue;
       const bool has = l_run[i] > 0.f;
       const float inv = has ? 1.f / l_run[i] : 0.f;
       const float lse2 = has ? m_run[i] * sl2 + log2f(l_run[i]) : -INFINITY;
+      // This thread's kOCols output columns, kOP at a time from TMEM, scaled by 1/l.
+      auto load_scaled = [&](int c, float (&v)[kOP]) {
+        uint32_t ob[kOP];
+        if constexpr (kOP == 32) tmem_ld32(lane_addr + o_col + c * 32, ob);
+        else tmem_ld16(lane_addr + o_col + c * 16, ob);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < kOP; ++e) v[e] = __uint_as_float(ob[e]) * inv;
+      };
       if constexpr (M == Mode::kPhase1) {
         const int64_t t = row_tok[i];
         const bool valid = row < rows_valid[i];
         // uniform: row bb * L + t of [b, L, Hq, d]; varlen: row tok_base + t of [total, Hq, d]
         __nv_bfloat16* dst = a.o + ((static_cast<int64_t>(it.bb) * a.L + it.tok_base + t) * a.hq + head[i]) * D +
-                             hf * kOCols;
+                             part * kOCols;
 #pragma unroll
-        for (int c = 0; c < kOCols / 32; ++c) {
-          uint32_t ob[32];
-          tmem_ld32(lane_addr + o_col + c * 32, ob);
-          tmem_wait_ld();
-          uint32_t w[16];
+        for (int c = 0; c < kOCols / kOP; ++c) {
+          float v[kOP];
+          load_scaled(c, v);
+          uint32_t w[kOP / 2];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(ob[2 * e]) * inv, __uint_as_float(ob[2 * e + 1]) * inv);
+          for (int e = 0; e < kOP / 2; ++e) w[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
           if (valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * kOP);
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < kOP / 8; ++u)
               d4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
           }
         }
-        if (a.lse && valid && hf == 0)
+        if (a.lse && valid && part == 0)
           a.lse[(static_cast<int64_t>(it.bb) * a.hq + head[i]) * a.L + it.tok_base + t] =
               lse2 * 0.69314718055994531f;
       } else {
         const int tok = static_cast<int>(row_tok[i]);
         const int hq = head[i];
         const bool valid = tok < it.lq;
-        float* dst = a.o_parts + ((it.rbase + tok) * a.hq + hq) * D + hf * kOCols;
+        float* dst = a.o_parts + ((it.rbase + tok) * a.hq + hq) * D + part * kOCols;
 #pragma unroll
-        for (int c = 0; c < kOCols / 32; ++c) {
-          uint32_t ob[32];
-          tmem_ld32(lane_addr + o_col + c * 32, ob);
-          tmem_wait_ld();
+        for (int c = 0; c < kOCols / kOP; ++c) {
+          float v[kOP];
+          load_scaled(c, v);
           if (valid) {
-            float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+            float4* d4 = reinterpret_cast<float4*>(dst + c * kOP);
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-              d4[u] = make_float4(__uint_as_float(ob[4 * u]) * inv, __uint_as_float(ob[4 * u + 1]) * inv,
-                                  __uint_as_float(ob[4 * u + 2]) * inv, __uint_as_float(ob[4 * u + 3]) * inv);
+            for (int u = 0; u < kOP / 4; ++u) d4[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
           }
         }
-        if (valid && hf == 0)
+        if (valid && part == 0)
           a.lse_parts[it.rbase * a.hq + static_cast<int64_t>(hq) * it.lq + tok] = lse2 * 0.69314718055994531f;
       }
     }
