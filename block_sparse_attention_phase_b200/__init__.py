@@ -24,7 +24,9 @@ from typing import Optional, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libstarattn.so")
+# STAR_ATTN_LIBRARY may name another build of the same library (the debug build,
+# libstarattn_debug.so next to this file); there is no other fallback.
+LIB_PATH = os.environ.get("STAR_ATTN_LIBRARY") or os.path.join(_HERE, "libstarattn.so")
 
 STAR_PHASE1, STAR_PHASE2_QUERY, STAR_PHASE2_DECODE, STAR_PHASE2_DECODE_FUSED = 1, 2, 3, 4
 STATUS_NAMES = {0: "STAR_OK", 1: "STAR_ERR_INVALID_ARG", 2: "STAR_ERR_UNSUPPORTED",
@@ -33,6 +35,7 @@ STATUS_NAMES = {0: "STAR_OK", 1: "STAR_ERR_INVALID_ARG", 2: "STAR_ERR_UNSUPPORTE
 
 # Every symbol the header declares; tests check that the library exports them all.
 EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase1_varlen",
+            "star_attn_phase1_anchored",
             "star_attn_rope", "star_attn_phase1_anchor_q",
             "star_attn_phase2_query",
             "star_attn_phase2_decode", "star_attn_phase2_decode_fused",
@@ -44,6 +47,7 @@ EXPORTED = ["star_attn_workspace_bytes", "star_attn_phase1", "star_attn_phase1_v
             "star_attn_lse_merge", "star_attn_simple_phase1",
             "star_attn_simple_phase2", "star_attn_get_device_status",
             "star_attn_selftest_wait_timeout", "star_attn_selftest_exp2", "star_attn_selftest_read",
+            "star_attn_debug_build", "star_attn_debug_record", "star_attn_selftest_bounds",
             "star_attn_launch_count",
             "star_attn_status_string", "star_attn_version"]
 
@@ -79,6 +83,7 @@ def lib() -> ctypes.CDLL:
         "star_attn_workspace_bytes": (SZ, [SP, I32, I64]),
         "star_attn_phase1": (I32, [SP, P, P, P, P, P, P]),
         "star_attn_phase1_varlen": (I32, [SP, ctypes.POINTER(I64), P, P, P, P, P, P]),
+        "star_attn_phase1_anchored": (I32, [SP, P, P, P, P, P, P, P, P]),
         "star_attn_rope": (I32, [SP, ctypes.POINTER(ctypes.c_float), I64, P, P, P, P, P, P]),
         "star_attn_phase1_anchor_q": (I32, [SP, P, P, P, P, P, P, P]),
         "star_attn_phase2_query": (I32, [SP, P, P, P, I64, P, P, P, P, I64, P, P, P, SZ, P]),
@@ -108,6 +113,9 @@ def lib() -> ctypes.CDLL:
         "star_attn_selftest_wait_timeout": (I32, [ctypes.c_uint64, P]),
         "star_attn_selftest_exp2": (I32, [P, P, I64, P]),
         "star_attn_selftest_read": (I32, [P, SZ, P, I32, P]),
+        "star_attn_debug_build": (I32, []),
+        "star_attn_debug_record": (I32, [ctypes.POINTER(I64), P]),
+        "star_attn_selftest_bounds": (I32, [P, I64, P]),
         "star_attn_launch_count": (ctypes.c_uint64, []),
         "star_attn_status_string": (ctypes.c_char_p, [I32]),
         "star_attn_version": (ctypes.c_char_p, []),
@@ -171,6 +179,27 @@ def phase1(q, k, v, block_size: int, scale: Optional[float] = None, o=None, lse=
         lse = torch.empty((b, hq, L), dtype=torch.float32, device=q.device)
     _check(lib().star_attn_phase1(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                   _ptr(lse), _stream()), "star_attn_phase1")
+    return o, lse
+
+
+def phase1_anchored(q, k, v, k_anchor, v_anchor, block_size: int, scale: Optional[float] = None,
+                    o=None, lse=None, want_lse: bool = True):
+    """One host's share of Phase 1: q [b, L, Hq, d], k/v [b, L, Hkv, d] are whole blocks
+    b_i.. (i > 0) of a longer context; k_anchor/v_anchor [b, B, Hkv, d] are b_0's K/V.
+    Every local block attends to the anchor and causally to itself. Returns (o, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (k_anchor, "k_anchor"), (v_anchor, "v_anchor")):
+        _bf16(t, n, 4)
+    if k_anchor.shape[1] != block_size or k_anchor.shape != v_anchor.shape:
+        raise ValueError("the anchor holds block_size tokens of K and of V")
+    shape = _ctx_shape(q, k, block_size, scale)
+    b, L, hq, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((b, hq, L), dtype=torch.float32, device=q.device)
+    _check(lib().star_attn_phase1_anchored(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(k_anchor), _ptr(v_anchor), _ptr(o), _ptr(lse),
+                                           _stream()), "star_attn_phase1_anchored")
     return o, lse
 
 
@@ -585,6 +614,27 @@ def selftest_read(buf: torch.Tensor, sink: torch.Tensor, ctas: int) -> None:
         raise TypeError("sink must be an int32 CUDA tensor with ctas elements")
     _check(lib().star_attn_selftest_read(_ptr(buf), buf.numel() * buf.element_size(), _ptr(sink),
                                          int(ctas), _stream()), "star_attn_selftest_read")
+
+
+def debug_build() -> bool:
+    """Whether the loaded library was built with -DSTAR_DEBUG (index checks)."""
+    return bool(lib().star_attn_debug_build())
+
+
+def debug_record():
+    """(refusals, source line, index, limit) of the first index a debug build's
+    checks refused since the last call (zeros if none); synchronises the stream."""
+    out = (ctypes.c_int64 * 4)()
+    _check(lib().star_attn_debug_record(out, _stream()), "star_attn_debug_record")
+    return tuple(int(v) for v in out)
+
+
+def selftest_bounds(out: torch.Tensor, n: int) -> None:
+    """Check index n against limit n with the kernels' store check (out: int32 CUDA
+    tensor with at least n + 1 elements)."""
+    if out.dtype != torch.int32 or not out.is_cuda or out.numel() < n + 1:
+        raise TypeError("out must be an int32 CUDA tensor with n + 1 elements")
+    _check(lib().star_attn_selftest_bounds(_ptr(out), int(n), _stream()), "star_attn_selftest_bounds")
 
 
 def launch_count() -> int:

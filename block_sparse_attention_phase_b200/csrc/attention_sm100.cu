@@ -92,6 +92,8 @@ struct AttnArgs {
   int32_t n_blocks, mt;   // blocks; 128-row q-tiles per block
   int32_t n_anchor;       // 128-column tiles covering the anchor b_0
   int32_t anchor_q;       // 1: the anchor tiles are scored with a second Q (map tk2)
+  int32_t anchor_sep;     // 1: the anchor's K/V come from maps tk2/tv2 ([b, B, Hkv, d]) and
+                          //    every block of this context is a block i > 0 (a host's share)
   __nv_bfloat16* o;       // [b, L, Hq, d]
   float* lse;             // [b, Hq, L] or null
   // Phase-2 query
@@ -198,7 +200,7 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, const VarSeqs& vs
     for (int q = 0; q < 2; ++q)
       it.rows_valid[q] = it.t0[q] >= bend ? 0 : static_cast<int>(bend - it.t0[q] < 128 ? bend - it.t0[q] : 128);
     const int m_last = it.rows_valid[1] > 0 ? m1 : m0;
-    it.n_anchor = i > 0 ? n_anchor : 0;
+    it.n_anchor = (i > 0 || a.anchor_sep) ? n_anchor : 0;
     it.n_tiles = it.rows_valid[0] > 0 ? it.n_anchor + m_last + 1 : 0;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -338,16 +340,32 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
   Bars* bars = reinterpret_cast<Bars*>(sv + 2 * kTileBytes);
 
   const Item it = decode_item<M>(a, vs);
+  // Sizes of the buffers this CTA stores to (the debug build's index checks).
+  // Phase 1: o [b, L, Hq, D] or [total, Hq, D], lse [b, Hq, L] or [Hq, total];
+  // query: o_parts [rows, Hq, D], lse_parts [rows, Hq] with rows = all partial token-rows.
+  const int64_t out_rows = M == Mode::kPhase1 ? (vs.n > 0 ? a.L : static_cast<int64_t>(a.b) * a.L)
+                                              : (vs.n > 0 ? static_cast<int64_t>(vs.rbase[vs.n])
+                                                          : static_cast<int64_t>(a.n_splits) * a.b * a.lq);
+  if constexpr (M == Mode::kQuery) {
+    // The query pass is launched programmatically after the cache write: the merge
+    // that follows may be scheduled now (it waits for this grid to finish). This
+    // kernel waits for the previous one before it reads the cache rows or writes
+    // the partials (the previous kernel may be a merge still reading them).
+    pdl_launch_dependents();
+  }
   if (it.n_tiles == 0) {
     if constexpr (M == Mode::kQuery) {
       // A chunk past the end of a short last block: an empty partial.
+      pdl_wait();
       for (int idx = threadIdx.x; idx < 256 * D; idx += kThreads) {
         const int row = idx / D, e = idx % D;
         const int tok = it.tok0[row >> 7] + (row & 127) / a.G;
         if (tok >= it.lq) continue;
         const int hq = it.kvh * a.G + (row & 127) % a.G;
-        a.o_parts[((it.rbase + tok) * a.hq + hq) * D + e] = 0.f;
-        if (e == 0) a.lse_parts[it.rbase * a.hq + static_cast<int64_t>(hq) * it.lq + tok] = -INFINITY;
+        const int64_t oi = ((it.rbase + tok) * a.hq + hq) * D + e;
+        if (STAR_IN_BOUNDS(a.status, oi, out_rows * a.hq * D)) a.o_parts[oi] = 0.f;
+        const int64_t li = it.rbase * a.hq + static_cast<int64_t>(hq) * it.lq + tok;
+        if (e == 0 && STAR_IN_BOUNDS(a.status, li, out_rows * a.hq)) a.lse_parts[li] = -INFINITY;
       }
     }
     return;  // before any barrier or TMEM allocation
@@ -399,6 +417,15 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(mk);
       tma_prefetch_desc(mv);
+      if constexpr (M == Mode::kPhase1) {
+        if (a.anchor_sep) {
+          tma_prefetch_desc(&tk2);
+          tma_prefetch_desc(&tv2);
+        }
+      }
+      if constexpr (M == Mode::kQuery) {
+        if (it.cache) pdl_wait();  // the cache rows this pass reads were just written
+      }
       // Anchor-position variant: the anchor tiles see Q rotated at the anchor
       // positions (map tk2); after them, Q is reloaded from tq for the own block.
       bool reload_q = false;
@@ -423,9 +450,16 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         const int s = j & 1;
         const uint32_t ph = (j >> 1) & 1;
         int32_t kv0;
+        const CUtensorMap* tkm = mk;
+        const CUtensorMap* tvm = mv;
         if constexpr (M == Mode::kPhase1) {
           kv0 = static_cast<int32_t>(it.tok_base) +
                 (j < it.n_anchor ? j * 128 : static_cast<int32_t>(it.bstart + 128 * (j - it.n_anchor)));
+          if (a.anchor_sep && j < it.n_anchor) {  // the anchor's own buffer, rows [0, B)
+            kv0 = j * 128;
+            tkm = &tk2;
+            tvm = &tv2;
+          }
         } else {
           kv0 = static_cast<int32_t>(it.k0 + 128 * j);
         }
@@ -445,13 +479,13 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         mbar_arrive_expect_tx(&bars->k_full[s], kTileBytes);
 #pragma unroll
         for (int c = 0; c < CH; ++c)
-          tma_load_4d(sk + s * kTileBytes + c * kChunkBytes, mk, &bars->k_full[s], c * 64, it.kvh, kv0, c3);
+          tma_load_4d(sk + s * kTileBytes + c * kChunkBytes, tkm, &bars->k_full[s], c * 64, it.kvh, kv0, c3);
         last_k[s] = j;
         if (j >= 2 && !wait_or_abort(&bars->v_empty[s], ph ^ 1, bars, a.status)) break;
         mbar_arrive_expect_tx(&bars->v_full[s], kTileBytes);
 #pragma unroll
         for (int c = 0; c < CH; ++c)
-          tma_load_4d(sv + s * kTileBytes + c * kChunkBytes, mv, &bars->v_full[s], c * 64, it.kvh, kv0, c3);
+          tma_load_4d(sv + s * kTileBytes + c * kChunkBytes, tvm, &bars->v_full[s], c * 64, it.kvh, kv0, c3);
         last_v[s] = j;
         if (reload_q && j == it.n_anchor) {
           if (!wait_or_abort(&bars->q_free, 0, bars, a.status)) break;
@@ -729,6 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&bars->o_bar[q], 0, bars, a.status));
       tc_fence_after();
       if (!ok) continue;
+      if constexpr (M == Mode::kQuery) pdl_wait();  // the partials may still be read by the previous kernel
       const bool has = l_run[i] > 0.f;
       const float inv = has ? 1.f / l_run[i] : 0.f;
       const float lse2 = has ? m_run[i] * sl2 + log2f(l_run[i]) : -INFINITY;
@@ -743,10 +778,12 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       };
       if constexpr (M == Mode::kPhase1) {
         const int64_t t = row_tok[i];
-        const bool valid = row < rows_valid[i];
         // uniform: row bb * L + t of [b, L, Hq, d]; varlen: row tok_base + t of [total, Hq, d]
-        __nv_bfloat16* dst = a.o + ((static_cast<int64_t>(it.bb) * a.L + it.tok_base + t) * a.hq + head[i]) * D +
-                             part * kOCols;
+        const int64_t o_off = ((static_cast<int64_t>(it.bb) * a.L + it.tok_base + t) * a.hq + head[i]) * D +
+                              part * kOCols;
+        const bool valid = row < rows_valid[i] &&
+                           STAR_IN_BOUNDS(a.status, o_off + kOCols - 1, out_rows * a.hq * D);
+        __nv_bfloat16* dst = a.o + o_off;
 #pragma unroll
         for (int c = 0; c < kOCols / kOP; ++c) {
           float v[kOP];
@@ -761,14 +798,16 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
               d4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
           }
         }
-        if (a.lse && valid && part == 0)
-          a.lse[(static_cast<int64_t>(it.bb) * a.hq + head[i]) * a.L + it.tok_base + t] =
-              lse2 * 0.69314718055994531f;
+        const int64_t l_off = (static_cast<int64_t>(it.bb) * a.hq + head[i]) * a.L + it.tok_base + t;
+        if (a.lse && valid && part == 0 &&
+            STAR_IN_BOUNDS(a.status, l_off, (vs.n > 0 ? 1 : static_cast<int64_t>(a.b)) * a.hq * a.L))
+          a.lse[l_off] = lse2 * 0.69314718055994531f;
       } else {
         const int tok = static_cast<int>(row_tok[i]);
         const int hq = head[i];
-        const bool valid = tok < it.lq;
-        float* dst = a.o_parts + ((it.rbase + tok) * a.hq + hq) * D + part * kOCols;
+        const int64_t o_off = ((it.rbase + tok) * a.hq + hq) * D + part * kOCols;
+        const bool valid = tok < it.lq && STAR_IN_BOUNDS(a.status, o_off + kOCols - 1, out_rows * a.hq * D);
+        float* dst = a.o_parts + o_off;
 #pragma unroll
         for (int c = 0; c < kOCols / kOP; ++c) {
           float v[kOP];
@@ -779,8 +818,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
             for (int u = 0; u < kOP / 4; ++u) d4[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
           }
         }
-        if (valid && part == 0)
-          a.lse_parts[it.rbase * a.hq + static_cast<int64_t>(hq) * it.lq + tok] = lse2 * 0.69314718055994531f;
+        const int64_t l_off = it.rbase * a.hq + static_cast<int64_t>(hq) * it.lq + tok;
+        if (valid && part == 0 && STAR_IN_BOUNDS(a.status, l_off, out_rows * a.hq))
+          a.lse_parts[l_off] = lse2 * 0.69314718055994531f;
       }
     }
   }
@@ -820,7 +860,13 @@ cudaError_t launch(const AttnArgs& a, const CUtensorMap (&m)[5], int64_t items, 
   if (e != cudaSuccess) return e;
   if (items <= 0) return cudaSuccess;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
-  kern<<<static_cast<unsigned>(items), kThreads, smem, st>>>(m[0], m[1], m[2], m[3], m[4], a, vs);
+  if constexpr (M == Mode::kQuery) {
+    e = launch_programmatic(kern, dim3(static_cast<unsigned>(items)), dim3(kThreads), smem, st, m[0],
+                            m[1], m[2], m[3], m[4], a, vs);
+    if (e != cudaSuccess) return e;
+  } else {
+    kern<<<static_cast<unsigned>(items), kThreads, smem, st>>>(m[0], m[1], m[2], m[3], m[4], a, vs);
+  }
   count_launch();
   return cudaGetLastError();
 }
@@ -863,6 +909,36 @@ cudaError_t launch_phase1_anchor_q_t(const Shape& s, const void* q, const void* 
   a.mt = static_cast<int32_t>((s.B + 127) / 128);
   a.n_anchor = a.mt;
   a.anchor_q = 1;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  const int64_t pairs_per_block = a.G >= 2 ? static_cast<int64_t>(a.mt) * (a.G / 2) : (a.mt + 1) / 2;
+  const int64_t items = static_cast<int64_t>(s.b) * s.hkv * a.n_blocks * pairs_per_block;
+  VarSeqs vs;
+  vs.n = 0;
+  return launch<D, Mode::kPhase1>(a, m, items, vs, st);
+}
+
+// A host's share of Phase 1 in the multi-host form: the context holds blocks
+// b_i .. b_k (i > 0) of the global context, and the anchor b_0's K/V [b, B, Hkv, d]
+// is a separate buffer (received from the host holding b_0). Every local block
+// attends to the anchor and causally to itself; s.B is the global block size (also
+// the anchor's length), not clamped to the local context.
+template <int D>
+cudaError_t launch_phase1_anchored_t(const Shape& s, const void* q, const void* k, const void* v,
+                                     const void* ka, const void* va, void* o, float* lse,
+                                     cudaStream_t st) {
+  alignas(64) CUtensorMap m[5];
+  if (!encode_tma_bf16_4d(&m[0], q, D, s.hq, s.L, s.L, s.b, 64, 1, 128, true) ||
+      !encode_tma_bf16_4d(&m[1], k, D, s.hkv, s.L, s.L, s.b, 64, 1, 128, true) ||
+      !encode_tma_bf16_4d(&m[2], v, D, s.hkv, s.L, s.L, s.b, 64, 1, 128, true) ||
+      !encode_tma_bf16_4d(&m[3], ka, D, s.hkv, s.B, s.B, s.b, 64, 1, 128, true) ||
+      !encode_tma_bf16_4d(&m[4], va, D, s.hkv, s.B, s.B, s.b, 64, 1, 128, true))
+    return cudaErrorInvalidValue;
+  AttnArgs a = base_args(s);
+  a.n_blocks = static_cast<int32_t>(s.n_blocks());
+  a.mt = static_cast<int32_t>((s.B + 127) / 128);
+  a.n_anchor = a.mt;
+  a.anchor_sep = 1;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   const int64_t pairs_per_block = a.G >= 2 ? static_cast<int64_t>(a.mt) * (a.G / 2) : (a.mt + 1) / 2;
@@ -1049,6 +1125,13 @@ cudaError_t launch_phase1_anchor_q(const Shape& s, const void* q, const void* q_
                                    cudaStream_t st) {
   if (s.d == 128) return launch_phase1_anchor_q_t<128>(s, q, q_anchor, k, v, o, lse, st);
   return launch_phase1_anchor_q_t<64>(s, q, q_anchor, k, v, o, lse, st);
+}
+
+cudaError_t launch_phase1_anchored(const Shape& s, const void* q, const void* k, const void* v,
+                                   const void* k_anchor, const void* v_anchor, void* o, float* lse,
+                                   cudaStream_t st) {
+  if (s.d == 128) return launch_phase1_anchored_t<128>(s, q, k, v, k_anchor, v_anchor, o, lse, st);
+  return launch_phase1_anchored_t<64>(s, q, k, v, k_anchor, v_anchor, o, lse, st);
 }
 
 cudaError_t launch_phase1_varlen(const Shape& s, const int64_t* cu_seqlens, const void* q,

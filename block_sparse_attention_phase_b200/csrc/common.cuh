@@ -30,6 +30,37 @@ __device__ __forceinline__ void report(uint32_t* status, uint32_t bit) {
   if (status) atomicOr(status, bit);
 }
 
+// ------------------------------------------------------------------ debug index checks
+// Builds with -DSTAR_DEBUG check the index of every global store the kernels
+// compute against the size of the buffer it lands in. A refused index is not
+// stored; the first one is recorded (source line, index, limit) after the status
+// word, and kBoundsFlag is raised. Nothing traps. Without STAR_DEBUG the checks
+// compile to `true`.
+__device__ __forceinline__ void debug_violation(uint32_t* status, int line, int64_t index,
+                                                int64_t limit) {
+  if (!status) return;
+  atomicOr(status, kBoundsFlag);
+  if (atomicAdd(status + 1, 1u) == 0u) {
+    status[2] = static_cast<uint32_t>(line);
+    status[4] = static_cast<uint32_t>(static_cast<uint64_t>(index));
+    status[5] = static_cast<uint32_t>(static_cast<uint64_t>(index) >> 32);
+    status[6] = static_cast<uint32_t>(static_cast<uint64_t>(limit));
+    status[7] = static_cast<uint32_t>(static_cast<uint64_t>(limit) >> 32);
+  }
+}
+__device__ __forceinline__ bool debug_in_bounds(uint32_t* status, int line, int64_t index,
+                                                int64_t limit) {
+  if (index >= 0 && index < limit) return true;
+  debug_violation(status, line, index, limit);
+  return false;
+}
+#ifdef STAR_DEBUG
+#define STAR_IN_BOUNDS(status, index, limit) \
+  (::star::debug_in_bounds((status), __LINE__, static_cast<int64_t>(index), static_cast<int64_t>(limit)))
+#else
+#define STAR_IN_BOUNDS(status, index, limit) true
+#endif
+
 __device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 

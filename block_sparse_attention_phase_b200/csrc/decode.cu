@@ -302,6 +302,9 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const VL& dv,
       stage(sp0 + nb);
     }
   }
+  // outputs [b, 1, Hq, D] and [b, Hq, 1]
+  const int64_t out_rows = static_cast<int64_t>(kIsVarlen<VL> ? dv.n : a.b) * a.hq;
+  if (!STAR_IN_BOUNDS(a.status, orow0 + G - 1, out_rows)) return;
   if (tid < G && a.lse) a.lse[orow0 + tid] = s_w[tid] > 0.f ? s_m[tid] + logf(s_w[tid]) : -INFINITY;
 #pragma unroll
   for (int k = 0; k < KPT; ++k) {
@@ -397,7 +400,11 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
                                           : static_cast<int64_t>(bb) * a.cap + r;
         return (prow * a.hkv + kvh) * D + lane * 8;
       };
-      if (page >= 0) {
+      // cache elements: the pool [num_pages, P, Hkv, D] or [b, cap, Hkv, D]
+      const int64_t cache_elems =
+          (a.page_table ? static_cast<int64_t>(a.num_pages) * a.page_size : static_cast<int64_t>(a.b) * a.cap) *
+          a.hkv * D;
+      if (page >= 0 && STAR_IN_BOUNDS(a.status, row_off(cache_len) + 7, cache_elems)) {
         const int64_t src = (static_cast<int64_t>(bb) * a.hkv + kvh) * D + lane * 8;
         const int64_t dst = row_off(cache_len);
         *reinterpret_cast<uint4*>(a.k_cache + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
@@ -408,6 +415,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
           const uint4 z = make_uint4(0u, 0u, 0u, 0u);
           for (int64_t r = cache_len + 1; r < cache_len + a.page_size; ++r) {
             const int64_t off = row_off(r);
+            if (!STAR_IN_BOUNDS(a.status, off + 7, cache_elems)) break;
             *reinterpret_cast<uint4*>(a.k_cache + off) = z;
             *reinterpret_cast<uint4*>(a.v_cache + off) = z;
           }
@@ -613,7 +621,12 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
     const int64_t prow = part_row(a, dv, w, w.split) * a.hq + kvh * G;  // first head's row
     const float4* cacc4 = reinterpret_cast<const float4*>(cacc);
     float4* dst = reinterpret_cast<float4*>(a.o_parts + prow * D);
-    for (int f = threadIdx.x; f < G * D / 4; f += kWarps * 32) {
+    // partial rows of the launch: [S, b] (uniform) or the varlen splits; Hq rows of D each
+    int64_t part_rows;
+    if constexpr (kIsVarlen<VL>) part_rows = dv.split0[dv.n];
+    else part_rows = static_cast<int64_t>(gridDim.x) * a.b;
+    const bool part_ok = STAR_IN_BOUNDS(a.status, (prow + G) * D - 1, part_rows * a.hq * D);
+    for (int f = threadIdx.x; part_ok && f < G * D / 4; f += kWarps * 32) {
       const int h = f / (D / 4);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -627,7 +640,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, kStages <= 2 ? 3 : 2) decod
       }
       dst[f] = acc;
     }
-    if (threadIdx.x < G) a.lse_parts[prow + threadIdx.x] = s_plse[threadIdx.x];
+    if (threadIdx.x < G && part_ok) a.lse_parts[prow + threadIdx.x] = s_plse[threadIdx.x];
     if (a.counters) merge_if_last<D, G>(a, dv, w, base);
   }
 }

@@ -7,11 +7,11 @@
 //   o = sum_s exp(lse_s - M) o_s / W
 // A split whose lse_s is -inf (it saw no key) contributes nothing.
 //
-// One CTA of 8 warps per (batch, token, head). The warps take the splits in
-// turn (warp w: splits w, w+8, ...), each lane owning d/32 contiguous elements of
-// every partial row (coalesced 128-/256-byte reads), so the S partial rows are
-// read with 8-way parallelism instead of one after another; the warps' sums meet
-// in shared memory.
+// One warp per output row (batch, token, head), eight rows per CTA. The lanes
+// first take the splits' LSEs (32 at a time) for the maximum M and the weights
+// exp(lse_s - M); then each lane owns d/32 contiguous elements of the row and sums
+// the splits' partial rows (coalesced 512- or 256-byte warp reads), with the loads
+// of several splits in flight at once. Every partial is read once.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -20,24 +20,27 @@
 namespace star {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kRowsPerCta = 8;
 
 // Varlen query pass: one row per (packed query token, head); the token's sequence
 // (binary search in vs.start) gives its split count and partial rows: split s of
 // sequence i holds token-rows rbase[i] + s * lq_i .. (o: [rows, H, D]; lse: H x lq_i
 // per split). Outputs are packed: o [total, H, D], lse [H, total].
 template <int D, bool kVarlen, class OutT>
-__global__ void __launch_bounds__(kWarps * 32) merge_kernel(
+__global__ void __launch_bounds__(kRowsPerCta * 32) merge_kernel(
     const float* __restrict__ o_parts, const float* __restrict__ lse_parts, int32_t S, int32_t b,
     int64_t T, int32_t H, OutT* __restrict__ o, float* __restrict__ lse,
-    const __grid_constant__ VarSeqs vs, int64_t block_size) {
+    const __grid_constant__ VarSeqs vs, int64_t block_size, int64_t rows, uint32_t* status) {
   constexpr int E = D / 32;
-  __shared__ float red[kWarps];
-  __shared__ float acc_s[kWarps][D];
-  __shared__ float wsum_s[kWarps];
   const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int64_t row = blockIdx.x;  // (bb, t, h) with h fastest; varlen: (packed token, h)
+  // Launched programmatically: wait until the kernel that wrote the partials has
+  // finished, then let the next kernel in the stream start being scheduled (the
+  // next decode step writes this workspace only after its own pdl_wait()).
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  // (bb, t, h) with h fastest; varlen: (packed token, h)
   const int h = static_cast<int>(row % H);
   int64_t lse_stride, lse_off, o_stride, o_off, out_o, out_lse;
   if constexpr (kVarlen) {
@@ -71,62 +74,65 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(
     out_lse = lse_off;
   }
 
-  // Launched programmatically: wait until the kernel that wrote the partials has
-  // finished, then let the next kernel in the stream start being scheduled (the
-  // next decode step writes this workspace only after its own pdl_wait()).
-  pdl_wait();
-  pdl_launch_dependents();
-
-  // M = max over splits
+  // M = max over splits (lanes over splits)
   float M = -INFINITY;
-  for (int s = threadIdx.x; s < S; s += kWarps * 32) M = fmaxf(M, lse_parts[s * lse_stride + lse_off]);
+  for (int s = lane; s < S; s += 32) M = fmaxf(M, lse_parts[s * lse_stride + lse_off]);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  if (lane == 0) red[warp] = M;
-  __syncthreads();
-  M = red[0];
-#pragma unroll
-  for (int w = 1; w < kWarps; ++w) M = fmaxf(M, red[w]);
 
-  float W = 0.f;
+  float W = 0.f;  // this lane's share of sum_s exp(lse_s - M)
   float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
   if (M != -INFINITY) {
-#pragma unroll 2
-    for (int s = warp; s < S; s += kWarps) {
-      const float w = expf(lse_parts[s * lse_stride + lse_off] - M);  // 0 for an empty split
+    for (int s0 = 0; s0 < S; s0 += 32) {
+      const int cnt = S - s0 < 32 ? S - s0 : 32;
+      // lane k holds the weight of split s0 + k (0 for an empty split)
+      const float w = lane < cnt ? expf(lse_parts[(s0 + lane) * lse_stride + lse_off] - M) : 0.f;
       W += w;
-      const float* src = o_parts + s * o_stride + o_off;
-      if constexpr (E == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(src);
-        acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
-      } else {
-        const float2 x = *reinterpret_cast<const float2*>(src);
-        acc[0] += w * x.x; acc[1] += w * x.y;
+      const float* src = o_parts + static_cast<int64_t>(s0) * o_stride + o_off;
+      int k = 0;
+      for (; k + 4 <= cnt; k += 4) {  // four splits' rows in flight
+        float x[4][E];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if constexpr (E == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(src + (k + u) * o_stride);
+            x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
+          } else {
+            const float2 v = *reinterpret_cast<const float2*>(src + (k + u) * o_stride);
+            x[u][0] = v.x; x[u][1] = v.y;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float wu = __shfl_sync(0xffffffffu, w, k + u);
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[e] += wu * x[u][e];
+        }
+      }
+      for (; k < cnt; ++k) {
+        const float wk = __shfl_sync(0xffffffffu, w, k);
+        const float* r = src + k * o_stride;
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] += wk * r[e];
       }
     }
   }
 #pragma unroll
-  for (int e = 0; e < E; ++e) acc_s[warp][lane * E + e] = acc[e];
-  if (lane == 0) wsum_s[warp] = W;
-  __syncthreads();
-  if (warp == 0) {
-    float Wt = 0.f;
+  for (int off = 16; off >= 1; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+  const float inv = W > 0.f ? 1.f / W : 0.f;
+  // outputs: o [b, T, H, D] or [total, H, D]; lse [b, H, T] or [H, total]
+  const int64_t out_tokens = kVarlen ? T : static_cast<int64_t>(b) * T;
+  if (!STAR_IN_BOUNDS(status, out_o + E - 1, out_tokens * H * D)) return;
+  OutT* dst = o + out_o;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) Wt += wsum_s[w];
-    const float inv = Wt > 0.f ? 1.f / Wt : 0.f;
-    OutT* dst = o + out_o;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      float x = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) x += acc_s[w][lane * E + e];
-      if constexpr (sizeof(OutT) == 4) dst[e] = x * inv;
-      else dst[e] = __float2bfloat16_rn(x * inv);
-    }
-    if (lse && lane == 0) lse[out_lse] = Wt > 0.f ? M + logf(Wt) : -INFINITY;
+  for (int e = 0; e < E; ++e) {
+    if constexpr (sizeof(OutT) == 4) dst[e] = acc[e] * inv;
+    else dst[e] = __float2bfloat16_rn(acc[e] * inv);
   }
+  if (lse && lane == 0 && STAR_IN_BOUNDS(status, out_lse, out_tokens * H))
+    lse[out_lse] = W > 0.f ? M + logf(W) : -INFINITY;
 }
 
 }  // namespace
@@ -137,26 +143,27 @@ cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int32_t n
   const int64_t rows = static_cast<int64_t>(b) * tokens * heads;
   if (rows == 0) return cudaSuccess;
   if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
-  const dim3 grid(static_cast<unsigned>(rows));
+  const dim3 grid(static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta));
   auto* oo = static_cast<__nv_bfloat16*>(o);
   auto* of = static_cast<float*>(o);
   VarSeqs vs;
   vs.n = 0;
-  const dim3 blk(kWarps * 32);
+  const dim3 blk(kRowsPerCta * 32);
+  uint32_t* status = device_status_word();
   const int64_t none = 0;
   cudaError_t e;
   if (o_fp32)
     e = d == 128 ? launch_programmatic(merge_kernel<128, false, float>, grid, blk, 0, st, o_parts,
-                                       lse_parts, n_splits, b, tokens, heads, of, lse, vs, none)
+                                       lse_parts, n_splits, b, tokens, heads, of, lse, vs, none, rows, status)
                  : launch_programmatic(merge_kernel<64, false, float>, grid, blk, 0, st, o_parts,
-                                       lse_parts, n_splits, b, tokens, heads, of, lse, vs, none);
+                                       lse_parts, n_splits, b, tokens, heads, of, lse, vs, none, rows, status);
   else
     e = d == 128 ? launch_programmatic(merge_kernel<128, false, __nv_bfloat16>, grid, blk, 0, st,
                                        o_parts, lse_parts, n_splits, b, tokens, heads, oo, lse, vs,
-                                       none)
+                                       none, rows, status)
                  : launch_programmatic(merge_kernel<64, false, __nv_bfloat16>, grid, blk, 0, st,
                                        o_parts, lse_parts, n_splits, b, tokens, heads, oo, lse, vs,
-                                       none);
+                                       none, rows, status);
   if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();
@@ -169,13 +176,14 @@ cudaError_t launch_merge_varlen(const float* o_parts, const float* lse_parts, co
   const int64_t rows = total * heads;
   if (rows == 0) return cudaSuccess;
   if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;
-  const dim3 grid(static_cast<unsigned>(rows));
+  const dim3 grid(static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta));
   auto* oo = static_cast<__nv_bfloat16*>(o);
+  uint32_t* status = device_status_word();
   const cudaError_t e =
-      d == 128 ? launch_programmatic(merge_kernel<128, true, __nv_bfloat16>, grid, dim3(kWarps * 32), 0,
-                                     st, o_parts, lse_parts, 0, 1, total, heads, oo, lse, vs, block_size)
-               : launch_programmatic(merge_kernel<64, true, __nv_bfloat16>, grid, dim3(kWarps * 32), 0,
-                                     st, o_parts, lse_parts, 0, 1, total, heads, oo, lse, vs, block_size);
+      d == 128 ? launch_programmatic(merge_kernel<128, true, __nv_bfloat16>, grid, dim3(kRowsPerCta * 32), 0,
+                                     st, o_parts, lse_parts, 0, 1, total, heads, oo, lse, vs, block_size, rows, status)
+               : launch_programmatic(merge_kernel<64, true, __nv_bfloat16>, grid, dim3(kRowsPerCta * 32), 0,
+                                     st, o_parts, lse_parts, 0, 1, total, heads, oo, lse, vs, block_size, rows, status);
   if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();

@@ -192,10 +192,12 @@ star_status_t check_shape(const star_attn_shape_t* shape) {
 SplitPlan decode_plan(const Shape& s) { return make_plan(s, int64_t{sm_count()} * kDecodeCtasPerSM); }
 
 SplitPlan query_plan(const Shape& s, int64_t lq) {
-  // One tensor-core CTA per SM, each taking two q-tiles; aim at about two waves
-  // over (splits x pairs of q-tiles).
+  // One tensor-core CTA per SM, each taking two q-tiles; aim at about one wave
+  // over (splits x pairs of q-tiles): a CTA's time is set by its K/V tiles, so
+  // longer chunks in one wave beat shorter ones in two, and the fp32 partials
+  // (one per split) halve.
   const int64_t pairs = (query_tiles(s, lq) + 1) / 2;
-  return make_plan(s, 2 * int64_t{sm_count()} / pairs);
+  return make_plan(s, int64_t{sm_count()} / pairs);
 }
 
 size_t partial_bytes(const Shape& s, const SplitPlan& p, int64_t rows) {
@@ -255,6 +257,24 @@ STAR_ATTN_API star_status_t star_attn_phase1(const star_attn_shape_t* shape, con
     return STAR_ERR_INVALID_ARG;
   return star::cuda_status(
       star::launch_phase1_sm100(s, q, k, v, o, lse, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+STAR_ATTN_API star_status_t star_attn_phase1_anchored(const star_attn_shape_t* shape,
+                                                      const void* q, const void* k, const void* v,
+                                                      const void* k_anchor, const void* v_anchor,
+                                                      void* o, float* lse, star_stream_t stream) {
+  Shape s;
+  star_status_t st = star::resolve(shape, &s);
+  if (st != STAR_OK) return st;
+  s.B = shape->block_size;  // the global block size: also the anchor's length
+  if (s.B > (int64_t{1} << 31) - 1) return STAR_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !k_anchor || !v_anchor || !o) return STAR_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, k_anchor, v_anchor, o};
+  for (const void* p : ptrs)
+    if (!star::aligned16(p)) return STAR_ERR_INVALID_ARG;
+  if (!star::aligned4(lse)) return STAR_ERR_INVALID_ARG;
+  return star::cuda_status(star::launch_phase1_anchored(s, q, k, v, k_anchor, v_anchor, o, lse,
+                                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
 STAR_ATTN_API star_status_t star_attn_rope(const star_attn_shape_t* shape,
@@ -679,6 +699,34 @@ STAR_ATTN_API star_status_t star_attn_get_device_status(star_stream_t stream) {
   if (flags & star::kTimeoutFlag) return STAR_ERR_TIMEOUT;
   if (flags) return STAR_ERR_CUDA;
   return STAR_OK;
+}
+
+STAR_ATTN_API int32_t star_attn_debug_build(void) { return star::debug_build() ? 1 : 0; }
+
+STAR_ATTN_API star_status_t star_attn_debug_record(int64_t* out, star_stream_t stream) {
+  if (!out) return STAR_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return STAR_ERR_CUDA;
+  uint32_t* word = star::device_status_word();
+  if (!word) return STAR_ERR_CUDA;
+  uint32_t rec[star::kStatusWords] = {};
+  if (cudaMemcpy(rec, word, sizeof(rec), cudaMemcpyDeviceToHost) != cudaSuccess) return STAR_ERR_CUDA;
+  out[0] = rec[1];
+  out[1] = rec[2];
+  out[2] = static_cast<int64_t>(static_cast<uint64_t>(rec[4]) | (static_cast<uint64_t>(rec[5]) << 32));
+  out[3] = static_cast<int64_t>(static_cast<uint64_t>(rec[6]) | (static_cast<uint64_t>(rec[7]) << 32));
+  if (rec[1]) {  // clear the record (the flags word stays for star_attn_get_device_status)
+    const uint32_t zero[star::kStatusWords - 1] = {};
+    if (cudaMemcpy(word + 1, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return STAR_ERR_CUDA;
+  }
+  return STAR_OK;
+}
+
+STAR_ATTN_API star_status_t star_attn_selftest_bounds(void* out, int64_t n, star_stream_t stream) {
+  if (!out || n < 0 || !star::aligned4(out)) return STAR_ERR_INVALID_ARG;
+  return star::cuda_status(star::launch_selftest_bounds(static_cast<uint32_t*>(out), n,
+                                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
 STAR_ATTN_API star_status_t star_attn_selftest_exp2(const float* x, float* y, int64_t n,

@@ -18,6 +18,12 @@ namespace star {
 constexpr uint32_t kTimeoutFlag = 1u;  // a bounded wait ran out
 constexpr uint32_t kBoundsFlag = 2u;   // a bounds check refused an access
 
+// The status "word" is the first of kStatusWords 32-bit words. The rest hold the
+// record of the first index a debug build's checks refused (builds with
+// -DSTAR_DEBUG): [1] violations so far, [2] source line of the check, [3] unused,
+// [4..5] the index, [6..7] its limit (64-bit, low word first).
+constexpr int kStatusWords = 8;
+
 struct Shape {
   int32_t b, hq, hkv, d;
   int64_t L, B;
@@ -155,6 +161,12 @@ cudaError_t launch_decode_varlen(const Shape& s, const DecVarlen& dv, int64_t ma
                                  const FusedMerge& fm, cudaStream_t st);
 cudaError_t launch_phase1_sm100(const Shape& s, const void* q, const void* k, const void* v,
                                 void* o, float* lse, cudaStream_t st);
+// A host's share of Phase 1: q/k/v [b, L, H, d] hold whole blocks b_i.. (i > 0) of a
+// longer context, the anchor b_0's K/V [b, B, Hkv, d] is a separate buffer; every
+// local block attends to the anchor and causally to itself. s.B is not clamped to s.L.
+cudaError_t launch_phase1_anchored(const Shape& s, const void* q, const void* k, const void* v,
+                                   const void* k_anchor, const void* v_anchor, void* o, float* lse,
+                                   cudaStream_t st);
 // Phase 1 over a varlen batch: s.b sequences packed along tokens, s.L = total tokens,
 // cu_seqlens (host) [s.b + 1]; o [total, Hq, d], lse [Hq, total].
 cudaError_t launch_phase1_varlen(const Shape& s, const int64_t* cu_seqlens, const void* q,
@@ -190,6 +202,10 @@ cudaError_t launch_merge_varlen(const float* o_parts, const float* lse_parts, co
                                 int64_t block_size, int32_t heads, int32_t d, void* o, float* lse,
                                 cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t wait_ns, cudaStream_t st);
+// Whether this library was built with -DSTAR_DEBUG (index checks on every store).
+bool debug_build();
+// Checks index n against limit n in a tiny kernel (out: device, n + 1 words).
+cudaError_t launch_selftest_bounds(uint32_t* out, int64_t n, cudaStream_t st);
 cudaError_t launch_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t st);
 cudaError_t launch_selftest_read(const void* src, int64_t bytes, uint32_t* sink, int32_t ctas,
                                  cudaStream_t st);

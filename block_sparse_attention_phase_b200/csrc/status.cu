@@ -12,10 +12,18 @@
 namespace star {
 namespace {
 
-__device__ uint32_t g_status_word;
+__device__ uint32_t g_status_word[kStatusWords];
 
 constexpr int kMaxDevices = 64;
 std::atomic<uint32_t*> g_status_addr[kMaxDevices];
+
+// Debug-check self-test: one thread checks index n against limit n (one past the
+// end) with the same check the kernels' stores use, so a debug build records it
+// and skips the store (the store itself would be in bounds anyway: the buffer has
+// n + 1 elements and the kernel writes element n only when the check lets it).
+__global__ void selftest_bounds_kernel(uint32_t* out, int64_t n, uint32_t* status) {
+  if (threadIdx.x == 0 && blockIdx.x == 0 && STAR_IN_BOUNDS(status, n, n)) out[n] = 1u;
+}
 
 // One warp waits on a barrier that no thread arrives at; the wait runs out
 // after wait_ns, records the timeout and the block returns normally.
@@ -137,6 +145,22 @@ uint32_t* device_status_word() {
   p = static_cast<uint32_t*>(addr);
   g_status_addr[dev].store(p, std::memory_order_release);
   return p;
+}
+
+bool debug_build() {
+#ifdef STAR_DEBUG
+  return true;
+#else
+  return false;
+#endif
+}
+
+cudaError_t launch_selftest_bounds(uint32_t* out, int64_t n, cudaStream_t st) {
+  uint32_t* status = device_status_word();
+  if (!status) return cudaErrorInvalidDevice;
+  selftest_bounds_kernel<<<1, 32, 0, st>>>(out, n, status);
+  count_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_selftest_wait(uint64_t wait_ns, cudaStream_t st) {

@@ -5,14 +5,16 @@ communication: Phase 1 needs no exchange besides the anchor, Phase 2 one vector
 and one scalar per host and query row.)
 
 - The context's blocks are spread over the ranks in contiguous runs; rank 0 holds
-  b_0. Rank 0 broadcasts b_0's K/V (the anchor) once per layer. Each rank runs
-  Phase 1 on its own blocks: rank 0 directly (its context starts with b_0), the
-  others on [anchor ; their blocks], keeping only their blocks' rows.
+  b_0. Rank 0 broadcasts b_0's K/V (the anchor) once per layer into every rank's
+  own memory. Each rank runs Phase 1 on its own blocks: rank 0 directly (its
+  context starts with b_0), the others with star_attn_phase1_anchored, which reads
+  the received anchor where it lies: no copy of the anchor next to the blocks, no
+  anchor rows computed.
 - Phase 2: the query host (the last rank by default) broadcasts the query rows; every
   rank attends with its own context keys (and the query host also with its
   query-local cache) and returns an fp32 output and an LSE per row
-  (star_attn_phase2_partial); they are gathered to the query host and merged
-  exactly (star_attn_lse_merge).
+  (star_attn_phase2_partial); they are gathered to the query host only and
+  merged exactly there (star_attn_lse_merge).
 
 The collectives go through torch.distributed (NCCL between GPUs); the compute is
 this library's kernels. `backend` lets the host logic run with other compute (the
@@ -30,11 +32,15 @@ class GpuBackend:
     """The library's kernels."""
 
     def __init__(self):
-        from . import lse_merge, phase1, phase2_partial
+        from . import lse_merge, phase1, phase1_anchored, phase2_partial
         self._phase1, self._partial, self._merge = phase1, phase2_partial, lse_merge
+        self._anchored = phase1_anchored
 
     def phase1(self, q, k, v, block_size):
         return self._phase1(q, k, v, block_size)
+
+    def phase1_anchored(self, q, k, v, k_anchor, v_anchor, block_size):
+        return self._anchored(q, k, v, k_anchor, v_anchor, block_size)
 
     def partial(self, q, block_size, k_ctx, v_ctx, k, v, k_cache, v_cache, cache_len):
         return self._partial(q, block_size, k_ctx=k_ctx, v_ctx=v_ctx, k=k, v=v, k_cache=k_cache,
@@ -92,20 +98,17 @@ class ShardedStarAttention:
             anchor_k.copy_(k[:, :B])
             anchor_v.copy_(v[:, :B])
         if self.dist and self.world > 1:
-            self.dist.broadcast(anchor_k, src=0, group=self.group)
-            self.dist.broadcast(anchor_v, src=0, group=self.group)
+            src = self.dist.get_global_rank(self.group, 0) if self.group else 0
+            self.dist.broadcast(anchor_k, src=src, group=self.group)
+            self.dist.broadcast(anchor_v, src=src, group=self.group)
         if self.t1 == self.t0:
             return None, None
         self.k_ctx, self.v_ctx = k, v
         if self.t0 == 0:
             return self.backend.phase1(q, k, v, B)
-        # [anchor ; own blocks]: block 0 of this local context is the anchor copy
-        # (its rows are computed and dropped), every other block sees the anchor.
-        qa = torch.cat([torch.zeros((self.b, B, self.hq, self.d), dtype=q.dtype, device=q.device),
-                        q], dim=1)
-        o, lse = self.backend.phase1(qa, torch.cat([anchor_k, k], dim=1),
-                                     torch.cat([anchor_v, v], dim=1), B)
-        return o[:, B:], (lse[..., B:] if lse is not None else None)
+        # Every block here is a block i > 0: it attends to the received anchor and
+        # causally to itself.
+        return self.backend.phase1_anchored(q, k, v, anchor_k, anchor_v, B)
 
     # ------------------------------------------------------------------ Phase 2
     def _partial(self, q, k, v, cache_len):
@@ -122,21 +125,26 @@ class ShardedStarAttention:
                                     self.v_cache if on_host else None, cache_len)
 
     def _combine(self, o, lse):
+        """Gather every rank's (o, lse) to the query rank (one vector and one scalar
+        per row and head from each host) and merge them there."""
+        on_host = self.rank == self.query_rank
         if self.dist and self.world > 1:
-            os_ = [torch.empty_like(o) for _ in range(self.world)]
-            ls = [torch.empty_like(lse) for _ in range(self.world)]
-            self.dist.all_gather(os_, o.contiguous(), group=self.group)
-            self.dist.all_gather(ls, lse.contiguous(), group=self.group)
+            dst = self.dist.get_global_rank(self.group, self.query_rank) if self.group else self.query_rank
+            os_ = [torch.empty_like(o) for _ in range(self.world)] if on_host else None
+            ls = [torch.empty_like(lse) for _ in range(self.world)] if on_host else None
+            self.dist.gather(o.contiguous(), os_, dst=dst, group=self.group)
+            self.dist.gather(lse.contiguous(), ls, dst=dst, group=self.group)
         else:
             os_, ls = [o], [lse]
-        if self.rank != self.query_rank:
+        if not on_host:
             return None, None
         return self.backend.lse_merge(torch.stack(os_), torch.stack(ls))
 
     def _broadcast_query(self, q):
         if self.dist and self.world > 1:
             q = q.contiguous()
-            self.dist.broadcast(q, src=self.query_rank, group=self.group)
+            src = self.dist.get_global_rank(self.group, self.query_rank) if self.group else self.query_rank
+            self.dist.broadcast(q, src=src, group=self.group)
         return q
 
     def query(self, q, k, v):

@@ -107,6 +107,28 @@ STAR_ATTN_API star_status_t star_attn_phase1(const star_attn_shape_t* shape, con
                                              star_stream_t stream);
 
 /*
+ * One host's share of Phase 1 in the multi-host form (hotaipapers.com page,
+ * Phase 1 paragraph: every host runs its blocks with the anchor b_0 in front;
+ * rebuttal to reviewer dnhh: no communication in Phase 1 beyond giving every
+ * host the anchor). The caller's context is a run of whole blocks b_i .. b_k of
+ * a longer context with i > 0 (the last may be short), and b_0's K/V arrive as
+ * separate buffers. Every local block attends to the whole anchor and causally to
+ * itself, exactly the rows star_attn_phase1() computes for those blocks over the
+ * whole context; the anchor is read where it lies and never copied next to the
+ * blocks, and no anchor row is computed.
+ *   shape->ctx_len: this host's tokens L; shape->block_size: the global block size
+ *     B, which is also the anchor's length (B may exceed L: one short block).
+ *   q [batch, L, Hq, d]; k, v [batch, L, Hkv, d]: this host's blocks.
+ *   k_anchor, v_anchor [batch, B, Hkv, d]: b_0's K and V (read only).
+ *   o [batch, L, Hq, d] bf16; lse [batch, Hq, L] fp32 or NULL.
+ * Needs no workspace. Errors as star_attn_phase1().
+ */
+STAR_ATTN_API star_status_t star_attn_phase1_anchored(const star_attn_shape_t* shape,
+                                                      const void* q, const void* k, const void* v,
+                                                      const void* k_anchor, const void* v_anchor,
+                                                      void* o, float* lse, star_stream_t stream);
+
+/*
  * Rotary position embedding of a layer's projected q [batch, L, Hq, d] and
  * k [batch, L, Hkv, d] (the model step before Phase 1 and Phase 2), at positions
  * pos0 + t for token t (Phase 1: pos0 = 0; the query tokens: pos0 = L; decode step
@@ -404,6 +426,28 @@ STAR_ATTN_API star_status_t star_attn_simple_phase2(
  * STAR_OK.
  */
 STAR_ATTN_API star_status_t star_attn_get_device_status(star_stream_t stream);
+
+/*
+ * Debug builds. A library built with -DSTAR_DEBUG checks the index of every
+ * global store its kernels compute against the size of the buffer it lands in
+ * (outputs, partials, LSEs, cache rows). A refused index is not stored: the
+ * kernel raises the bounds flag (star_attn_get_device_status() then returns
+ * STAR_ERR_CUDA) and the first refusal is recorded. Nothing traps.
+ *   star_attn_debug_build(): 1 for such a build, else 0.
+ *   star_attn_debug_record(out, stream): synchronises `stream`, then returns the
+ *     record of the current device and clears it: out[0] = refusals since the
+ *     last call, out[1] = the source line of the check, out[2] = the index,
+ *     out[3] = its limit (all 0 when nothing was refused, always so in other
+ *     builds). out: HOST array of 4 int64.
+ *   star_attn_selftest_bounds(out, n, stream): one thread checks index n against
+ *     limit n (one past the end) with the kernels' check; a debug build records
+ *     it and skips the store, another build stores out[n] = 1. out: device,
+ *     n + 1 uint32 (4-byte aligned).
+ * No counterpart on the Star Attention pages (the library's own test tooling).
+ */
+STAR_ATTN_API int32_t star_attn_debug_build(void);
+STAR_ATTN_API star_status_t star_attn_debug_record(int64_t* out, star_stream_t stream);
+STAR_ATTN_API star_status_t star_attn_selftest_bounds(void* out, int64_t n, star_stream_t stream);
 
 /*
  * Self-test of the bounded-wait path: launches one block that waits on a

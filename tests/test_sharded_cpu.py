@@ -39,6 +39,15 @@ class OracleBackend:
         o, lse = self.oracle.phase1(q.numpy(), k.numpy(), v.numpy(), block_size)
         return torch.from_numpy(o), torch.from_numpy(lse)
 
+    def phase1_anchored(self, q, k, v, k_anchor, v_anchor, block_size):
+        # The definition: this host's blocks are blocks i > 0 of a context that starts
+        # with the anchor, so their rows are those of Phase 1 over [anchor ; blocks].
+        B = block_size
+        qa = np.concatenate([np.zeros((q.shape[0], B) + tuple(q.shape[2:])), q.numpy()], axis=1)
+        o, lse = self.oracle.phase1(qa, np.concatenate([k_anchor.numpy(), k.numpy()], axis=1),
+                                    np.concatenate([v_anchor.numpy(), v.numpy()], axis=1), B)
+        return torch.from_numpy(o[:, B:]), torch.from_numpy(lse[..., B:])
+
     def partial(self, q, block_size, k_ctx, v_ctx, k, v, k_cache, v_cache, cache_len):
         o, lse, kc, vc = self.oracle.phase2_partial(
             q.numpy(), self._np(k_ctx), self._np(v_ctx), self._np(k), self._np(v),
@@ -132,3 +141,54 @@ def test_sharded_layer_matches_single_host(tmp_path, world):
         od, ld, kc, vc = oracle.phase2_decode(qd, kd, vd, k.numpy(), v.numpy(), kc, vc, s["lq"] + t)
         np.testing.assert_allclose(np.array(host["dec"][t][0]), od, atol=1e-12)
         np.testing.assert_allclose(np.array(host["dec"][t][1]), ld, atol=1e-12)
+
+
+def _bench_worker(rank, world, port, out_dir):
+    """bench.py's sharded step (the multi-GPU bench form) on gloo ranks with the
+    oracle as compute: every phase runs, and the query rank's merged outputs equal
+    the single-host oracle."""
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = workloads.Workload("bench-sharded", 1, 4, 2, 16, 70, 16, 3, 2, 0, 5)
+        x = {k: t.double() for k, t in workloads.make_inputs(w, device="cpu").items()}
+        step = bench.ShardedStep(w, x, "cpu", backend=OracleBackend(), dtype=torch.float64)
+        step.run()
+        step.run()  # a second pass over the same state (the bench's repeated steps)
+        res = {"range": [step.t0, step.t1]}
+        oq, lq = step.out["qry"]
+        res["oq"] = None if oq is None else oq.tolist()
+        res["dec"] = [None if od is None else od.tolist() for od, _ in step.out["dec"]]
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump(res, f)
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+def test_bench_sharded_step_on_gloo_ranks(tmp_path):
+    world = 3
+    mp.start_processes(_bench_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    sys.path.insert(0, ROOT)
+    import oracle
+    import workloads
+    w = workloads.Workload("bench-sharded", 1, 4, 2, 16, 70, 16, 3, 2, 0, 5)
+    x = {k: t.double().numpy() for k, t in workloads.make_inputs(w, device="cpu").items()}
+    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    assert [r["range"] for r in res][0][0] == 0 and res[-1]["range"][1] == w.ctx_len
+    host = res[-1]
+    rq, _ = oracle.phase2_query(x["q_qry"], x["k_qry"], x["v_qry"], x["k_ctx"], x["v_ctx"])
+    np.testing.assert_allclose(np.array(host["oq"]), rq, atol=1e-12)
+    cap = w.cache_capacity
+    kc = np.zeros((1, cap, w.num_kv_heads, w.head_dim))
+    vc = np.zeros_like(kc)
+    kc[:, :w.query_len], vc[:, :w.query_len] = x["k_qry"], x["v_qry"]
+    for t in range(w.decode_steps):
+        od, _, kc, vc = oracle.phase2_decode(x["q_dec"][t], x["k_dec"][t], x["v_dec"][t],
+                                             x["k_ctx"], x["v_ctx"], kc, vc, w.query_len + t)
+        np.testing.assert_allclose(np.array(host["dec"][t]), od, atol=1e-12)
+    assert all(r["oq"] is None for r in res[:-1])

@@ -33,14 +33,13 @@ def test_emulated_ranks_match_single_gpu(P):
     n = math.ceil(L / B)
     ranges = [(min(r * n // P * B, L), min((r + 1) * n // P * B, L)) for r in range(P)]
     # ---- Phase 1 per rank
+    ka, va = k[:, :B].contiguous(), v[:, :B].contiguous()  # what the anchor broadcast delivers
     for t0, t1 in ranges:
+        sl = lambda t: t[:, t0:t1].contiguous()  # noqa: E731
         if t0 == 0:
-            o, l = m.phase1(q[:, t0:t1].contiguous(), k[:, t0:t1].contiguous(), v[:, t0:t1].contiguous(), B)
+            o, l = m.phase1(sl(q), sl(k), sl(v), B)
         else:
-            qa = torch.cat([torch.zeros_like(q[:, :B]), q[:, t0:t1]], dim=1)
-            o, l = m.phase1(qa, torch.cat([k[:, :B], k[:, t0:t1]], dim=1),
-                            torch.cat([v[:, :B], v[:, t0:t1]], dim=1), B)
-            o, l = o[:, B:], l[..., B:]
+            o, l = m.phase1_anchored(sl(q), sl(k), sl(v), ka, va, B)
         assert torch.equal(o, o_full[:, t0:t1]) and torch.equal(l, l_full[..., t0:t1])
     # ---- Phase 2: the last rank is the query host
     cap = lq + T
@@ -71,6 +70,35 @@ def test_emulated_ranks_match_single_gpu(P):
         check_rows(to_np(od), to_np(rd).astype(np.float64), to_np(ld), to_np(rdl).astype(np.float64),
                    f"decode P={P} t={t}")
     assert torch.equal(kc, kref) and torch.equal(vc, vref)
+    assert m.device_status() == 0
+
+
+@pytest.mark.parametrize("b,hq,hkv,d,L,B,t0", [
+    (1, 8, 2, 128, 9000, 1024, 3072),   # G = 4; the last local block is ragged
+    (2, 4, 4, 64, 2600, 640, 640),      # G = 1 (pairs of q-tiles of one head), batch 2
+    (1, 4, 2, 128, 2100, 1024, 2048),   # a host holding only a short last block (52 < B rows)
+    (1, 16, 2, 128, 1500, 300, 900),    # G = 8, B not a multiple of 128
+])
+def test_phase1_anchored_rows_equal_the_single_launch(b, hq, hkv, d, L, B, t0):
+    """A host's blocks b_i.. (i > 0) with the anchor passed as its own buffer give
+    exactly the rows the whole-context launch gives for them (same tiles, same
+    order), and they match the oracle."""
+    m = sa()
+    w = workloads.Workload("anch", b, hq, hkv, d, L, B, 1, 1, 0, 11)
+    x = workloads.make_inputs(w, device="cuda", parts=("ctx",))
+    q, k, v = x["q_ctx"], x["k_ctx"], x["v_ctx"]
+    o_full, l_full = m.phase1(q, k, v, B)
+    ka, va = k[:, :B].contiguous(), v[:, :B].contiguous()
+    o, l = m.phase1_anchored(q[:, t0:].contiguous(), k[:, t0:].contiguous(), v[:, t0:].contiguous(),
+                             ka, va, B)
+    assert torch.equal(o, o_full[:, t0:]) and torch.equal(l, l_full[..., t0:])
+    rows = np.arange(t0, L)
+    for bi in range(b):
+        for h in (0, hq - 1):
+            g = h // (hq // hkv)
+            ro, rl = oracle.phase1_head(to_np(q[bi, :, h]), to_np(k[bi, :, g]), to_np(v[bi, :, g]), B,
+                                        1.0 / math.sqrt(d), rows)
+            check_rows(to_np(o[bi, :, h]), ro, to_np(l[bi, h]), rl, f"anchored b={bi} h={h}")
     assert m.device_status() == 0
 
 
