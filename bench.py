@@ -7,9 +7,12 @@ in HBM when timing starts. Prints one JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl star|reference]
 
-Multi-GPU runs (torchrun, one process per GPU) execute independent replicas of
-the workload (the path has no data-path exchange on one node's problem; each
-rank draws its own seeded inputs): weak scaling, timed as the max over ranks.
+Multi-GPU runs (torchrun, one process per GPU) run the pages' own multi-host
+form by default: one context of the workload split over the ranks in runs of
+whole blocks, the anchor broadcast from rank 0, each rank's Phase-2 partials
+gathered to the query rank and merged there (strong scaling, timed as the max
+over ranks; `--sharded` forces this form on one GPU too). `--replicas` runs
+independent single-GPU replicas instead (weak scaling).
 `--impl reference` times the CPU oracle instead, on bounded samples of the same
 workload, extrapolated to the same metric.
 """
@@ -262,6 +265,190 @@ def read_peak_gbs(device, nbytes: int = 4 << 30, reps: int = 5):
     del buf, sink
     torch.cuda.empty_cache()
     return nbytes / (best / 1e3) / 1e9
+
+
+class ShardedStep:
+    """One whole hot-path pass of the pages' multi-host form on this rank: its share
+    of the context (a contiguous run of blocks; rank 0 holds b_0, the last rank is
+    the query host), the anchor broadcast and Phase 1 on its own blocks, then the
+    query tokens and every decode step with each rank's partials gathered to the
+    query rank and merged there (block_sparse_attention_phase_b200.sharded).
+    `backend` None = the library's kernels; tests pass a CPU stand-in."""
+
+    def __init__(self, w, x, device, backend=None, dtype=torch.bfloat16):
+        from block_sparse_attention_phase_b200.sharded import ShardedStarAttention
+        self.w = w
+        self.att = ShardedStarAttention(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                        w.ctx_len, w.block_size, w.cache_capacity, backend=backend,
+                                        device=device, dtype=dtype)
+        t0, t1 = self.att.token_range()
+        self.t0, self.t1 = t0, t1
+        self.x = {k: (v[:, t0:t1].contiguous() if k.endswith("_ctx") else v) for k, v in x.items()}
+        self.events = None
+        self.out = {}
+
+    def phases(self):
+        x, att, w = self.x, self.att, self.w
+        yield lambda: self.out.__setitem__("ctx", att.prefill(x["q_ctx"], x["k_ctx"], x["v_ctx"]))
+        yield lambda: self.out.__setitem__("qry", att.query(x["q_qry"], x["k_qry"], x["v_qry"]))
+
+        def decode_all():
+            dec = []
+            for t in range(w.decode_steps):
+                dec.append(att.decode(x["q_dec"][t], x["k_dec"][t], x["v_dec"][t]))
+            self.out["dec"] = dec
+        yield decode_all
+
+    def run(self, record: bool = False):
+        ev = []
+
+        def mark():
+            if record:
+                e = torch.cuda.Event(enable_timing=True)
+                e.record()
+                ev.append(e)
+
+        mark()
+        for fn in self.phases():
+            fn()
+            mark()
+        if record:
+            self.events = ev
+
+    def phase_times_ms(self):
+        ev = self.events
+        return (ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]),
+                ev[2].elapsed_time(ev[3]) / self.w.decode_steps)
+
+
+def sharded_e2e(step: ShardedStep, steps: int, world: int, device):
+    """The sharded step through the public API with host buffers: every step each
+    rank copies its inputs from pinned host memory, runs, and copies its outputs
+    back (the query rank: the merged query and decode outputs too), all inside the
+    timed region; the max over ranks. Returns the e2e object of the JSON line."""
+    host_in = {k: v.cpu().pin_memory() for k, v in step.x.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    step.run()  # outputs exist: their shapes size the host buffers
+    torch.cuda.synchronize()
+
+    def outputs():
+        o = [t for t in step.out["ctx"] if t is not None]
+        for key in ("qry",):
+            o += [t for t in step.out[key] if t is not None]
+        for pair in step.out["dec"]:
+            o += [t for t in pair if t is not None]
+        return o
+
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outputs()]
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    barrier(world)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        for k, v in host_in.items():
+            step.x[k].copy_(v, non_blocking=True)
+        step.run()
+        for h, t in zip(host_out, outputs()):
+            h.copy_(t, non_blocking=True)
+    b.record()
+    b.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world, device)
+    barrier(world)
+    return {"value": step.w.batch * step.w.ctx_len / (ms / 1e3), "unit": "tok/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "bytes_are": "this rank's (rank 0)"}
+
+
+def run_sharded(args, w, world, rank, local):
+    """The pages' multi-host form across the ranks of this job (strong scaling: one
+    context of the workload split over all GPUs). Prints one JSON line on rank 0."""
+    import block_sparse_attention_phase_b200 as sa
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    x = workloads.make_inputs(w, device=device, seed=w.seed)  # identical on every rank
+    step = ShardedStep(w, x, device)
+    del x
+    torch.cuda.empty_cache()
+    peaks = load_peaks()
+    flush = torch.empty(workloads.l2_flush_bytes(), dtype=torch.uint8, device=device)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step.run()
+    torch.cuda.synchronize()
+    barrier(world)
+    n0 = sa.launch_count()
+    recorded = []
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    wall0 = time.time()
+    t0.record()
+    for _ in range(args.steps):
+        flush.fill_(1)  # evict L2 between steps (buffer > 126 MB L2)
+        step.run(record=True)
+        recorded.append(step.events)
+    t1.record()
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier(world)
+    launches = sa.launch_count() - n0
+    clk = clocks.stop(wall0, wall1)
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world, device)
+    phases = []
+    for evs in recorded:
+        step.events = evs
+        phases.append(step.phase_times_ms())
+    p1_ms = max_over_ranks(statistics.mean(p[0] for p in phases), world, device)
+    q_ms = max_over_ranks(statistics.mean(p[1] for p in phases), world, device)
+    dec_ms = max_over_ranks(statistics.mean(p[2] for p in phases), world, device)
+    if world > 1:
+        t = torch.tensor([float(launches)], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t)
+        launches = int(t.item())
+    tokens = w.batch * w.ctx_len
+    value = tokens * args.steps / (elapsed_ms / 1e3)
+    flops = w.phase1_flops()
+    p1_tflops = flops / (p1_ms / 1e3) / 1e12  # whole context over the slowest rank's time
+    sustained = sum(p[0] for p in phases) / 1e3 >= SUSTAINED_AFTER_S
+    peak = (peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]) * world
+    kv = statistics.mean(w.decode_kv_bytes(t) for t in range(w.decode_steps))
+    dec_gbs = kv / (dec_ms / 1e3) / 1e9
+    e2e = None
+    if not args.no_e2e:
+        e2e = sharded_e2e(step, min(args.steps, 8), world, device)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads,
+                       "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                       "ctx_len": w.ctx_len, "block_size": w.block_size,
+                       "query_len": w.query_len, "decode_steps": w.decode_steps,
+                       "planted_pairs": w.planted_pairs, "parallelism": f"star-sharded{world}",
+                       "launch": "eager (collectives between the kernels)",
+                       "l2": "256 MiB write before every step",
+                       "sharding": "contiguous runs of blocks per rank; anchor broadcast from "
+                                   "rank 0; partials gathered to the last rank"},
+            "phase1": {"ms": p1_ms, "tflops": p1_tflops, "frac": p1_tflops / peak},
+            "query": {"ms": q_ms},
+            "decode": {"ms_per_token_in_step": dec_ms, "gbs_in_step": dec_gbs,
+                       "frac_hbm_in_step": dec_gbs / (peaks["hbm_gbs"] * world)},
+            "roofline": {"bound": "tensor", "achieved": p1_tflops / world, "peak": peak / world,
+                         "unit": "TFLOP/s", "frac": p1_tflops / peak, "traffic": None},
+            "roofline_kernel": "phase1 (slowest rank, per GPU)",
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "cpu_baseline": None,
+            "peaks": peaks,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
 
 
 COLD_SPIN_CYCLES = 400_000  # ~0.2 ms of GPU time at 1.9 GHz
@@ -587,6 +774,10 @@ def main(argv=None):
                     help="time Phase 1 against block size and dense causal attention instead")
     ap.add_argument("--decode-merge", default="fused", choices=["fused", "separate"],
                     help="decode step as one kernel (last-CTA merge) or partials + merge kernel")
+    ap.add_argument("--sharded", action="store_true",
+                    help="the pages' multi-host form (also on one GPU); the default with several GPUs")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with several GPUs: independent replicas of the single-GPU step instead")
     ap.add_argument("--phase1-only", action="store_true",
                     help="time Phase 1 alone (launch by launch) instead of the whole step")
     ap.add_argument("--ctx-len", type=int, default=None,
@@ -609,6 +800,11 @@ def main(argv=None):
         return block_sweep(args) if rank == 0 else 0
     if args.impl == "reference":
         return run_reference(args, w, world, rank)
+    if args.sharded or (world > 1 and not args.replicas):
+        rc = run_sharded(args, w, world, rank, local)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return rc
 
     import block_sparse_attention_phase_b200 as sa
     device = torch.device("cuda", local)
