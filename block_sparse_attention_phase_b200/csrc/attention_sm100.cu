@@ -133,6 +133,7 @@ struct Item {
   // query
   int split, tok0[2];
   bool cache;
+  bool dual;           // both Q tiles hold the same rows; tile q takes K/V tiles 2j + q of the chunk
   int64_t k0, k1;
   int32_t lq;          // this sequence's query tokens
   int32_t q_c3;        // outer Q coordinate: the sequence, or 0 for packed queries
@@ -265,7 +266,15 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, const VarSeqs& vs
       it.k0 = 0;
       it.k1 = it.lq;
     }
-    it.n_tiles = static_cast<int>((it.k1 - it.k0 + 127) / 128);
+    const int n_kv = static_cast<int>((it.k1 - it.k0 + 127) / 128);
+    // A context split whose second Q tile has no rows (all query rows fit one tile)
+    // gives that tile the same rows and half of the chunk's K/V tiles: tile q takes
+    // tiles 2j + q, so each step processes two K/V tiles for the one real Q tile and
+    // the two partial softmaxes are combined in the epilogue. (Needs the column-part
+    // layout, where each thread holds both tiles' state for its row.)
+    it.dual = kParts > 1 && !it.cache && it.tok0[1] >= it.lq;
+    if (it.dual) it.tok0[1] = it.tok0[0];
+    it.n_tiles = it.dual ? (n_kv + 1) / 2 : n_kv;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       it.qc1[q] = it.kvh * a.G;
@@ -305,7 +314,7 @@ __device__ __forceinline__ void setmaxnreg_inc() {
 // `tok` (Phase 1: absolute context position; query: query-token index).
 template <Mode M>
 __device__ __forceinline__ int visible_prefix(const Item& it, const AttnArgs& a, int64_t tok,
-                                              int j) {
+                                              int j, int q) {
   int64_t lim;
   if constexpr (M == Mode::kPhase1) {
     if (j < it.n_anchor) {
@@ -318,7 +327,7 @@ __device__ __forceinline__ int visible_prefix(const Item& it, const AttnArgs& a,
     if (it.cache)
       lim = tok - 128 * static_cast<int64_t>(j) + 1;  // query token sees cache rows <= itself
     else
-      lim = it.k1 - it.k0 - 128 * static_cast<int64_t>(j);  // end of the chunk
+      lim = it.k1 - it.k0 - 128 * static_cast<int64_t>(it.dual ? 2 * j + q : j);  // end of the chunk
   }
   return lim < 0 ? 0 : (lim > 128 ? 128 : static_cast<int>(lim));
 }
@@ -446,7 +455,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       load_q(mq);
       int q_loads = 1;
       int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
-      for (int j = 0; j < n_tiles; ++j) {
+      // Tile j goes to ring stage j & 1 (dual: stage q holds Q tile q's K/V tiles).
+      const int n_loads = it.dual ? 2 * n_tiles : n_tiles;
+      for (int j = 0; j < n_loads; ++j) {
         const int s = j & 1;
         const uint32_t ph = (j >> 1) & 1;
         int32_t kv0;
@@ -522,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       if constexpr (M == Mode::kPhase1) reload_q = a.anchor_q && it.n_anchor > 0;
       auto issue_s = [&](int q, int j) {
         const uint32_t qd = q ? qd1 : qd0;
-        const uint32_t kd = (j & 1) ? kd1 : kd0;
+        const uint32_t kd = (it.dual ? q : (j & 1)) ? kd1 : kd0;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off16 = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
@@ -535,46 +546,79 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       // (d contiguous): 16 kv rows a step, the next 64 columns of d one chunk (LBO)
       // away, the next 8 kv rows 1024 B (SBO) away.
       auto issue_pv = [&](int q, int j) {
-        const uint32_t vd = (j & 1) ? vd1 : vd0;
+        const uint32_t vd = (it.dual ? q : (j & 1)) ? vd1 : vd0;
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
           tc_mma_ts_lo(tmem + 256 + q * D, tmem + q * 128 + kk * 8, vd + kk * (2048 >> 4), kDescHi,
                        kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
       };
-      bool ok = wait_or_abort(&bars->q_full, 0, bars, a.status) &&
-                wait_or_abort(&bars->k_full[0], 0, bars, a.status);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        tc_commit(&bars->k_empty[0]);
-      }
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j & 1;
-        const bool more = j + 1 < n_tiles;
-        ok = wait_or_abort(&bars->v_full[s], (j >> 1) & 1, bars, a.status) &&
-             wait_or_abort(&bars->p_full[0], j & 1, bars, a.status);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(0, j);
-        if (!more) tc_commit(&bars->o_bar[0]);
-        if (more) {
-          ok = wait_or_abort(&bars->k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, bars, a.status);
-          // the first own-block tile needs the reloaded Q
-          if (ok && reload_q && j + 1 == it.n_anchor) ok = wait_or_abort(&bars->q_full, 1, bars, a.status);
+      bool ok;
+      if (it.dual) {
+        // Both Q tiles hold the same rows; Q tile q's K/V tiles (2j + q) sit in ring
+        // stage q, round j: S_q and PV_q each free their own stage.
+        ok = wait_or_abort(&bars->q_full, 0, bars, a.status);
+        for (int q = 0; ok && q < 2; ++q) {
+          ok = wait_or_abort(&bars->k_full[q], 0, bars, a.status);
           if (!ok) break;
           tc_fence_after();
-          issue_s(0, j + 1);
+          issue_s(q, 0);
+          tc_commit(&bars->k_empty[q]);
         }
-        ok = wait_or_abort(&bars->p_full[1], j & 1, bars, a.status);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(1, j);
-        tc_commit(&bars->v_empty[s]);
-        if (!more) tc_commit(&bars->o_bar[1]);
-        if (more) {
-          issue_s(1, j + 1);
-          tc_commit(&bars->k_empty[(j + 1) & 1]);
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const bool more = j + 1 < n_tiles;
+          for (int q = 0; ok && q < 2; ++q) {
+            ok = wait_or_abort(&bars->v_full[q], j & 1, bars, a.status) &&
+                 wait_or_abort(&bars->p_full[q], j & 1, bars, a.status);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(q, j);
+            tc_commit(&bars->v_empty[q]);
+            if (!more) tc_commit(&bars->o_bar[q]);
+            if (more) {
+              ok = wait_or_abort(&bars->k_full[q], (j + 1) & 1, bars, a.status);
+              if (!ok) break;
+              tc_fence_after();
+              issue_s(q, j + 1);
+              tc_commit(&bars->k_empty[q]);
+            }
+          }
+        }
+      } else {
+        ok = wait_or_abort(&bars->q_full, 0, bars, a.status) &&
+             wait_or_abort(&bars->k_full[0], 0, bars, a.status);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          issue_s(1, 0);
+          tc_commit(&bars->k_empty[0]);
+        }
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int s = j & 1;
+          const bool more = j + 1 < n_tiles;
+          ok = wait_or_abort(&bars->v_full[s], (j >> 1) & 1, bars, a.status) &&
+               wait_or_abort(&bars->p_full[0], j & 1, bars, a.status);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(0, j);
+          if (!more) tc_commit(&bars->o_bar[0]);
+          if (more) {
+            ok = wait_or_abort(&bars->k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, bars, a.status);
+            // the first own-block tile needs the reloaded Q
+            if (ok && reload_q && j + 1 == it.n_anchor) ok = wait_or_abort(&bars->q_full, 1, bars, a.status);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(0, j + 1);
+          }
+          ok = wait_or_abort(&bars->p_full[1], j & 1, bars, a.status);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(1, j);
+          tc_commit(&bars->v_empty[s]);
+          if (!more) tc_commit(&bars->o_bar[1]);
+          if (more) {
+            issue_s(1, j + 1);
+            tc_commit(&bars->k_empty[(j + 1) & 1]);
+          }
         }
       }
       // Every MMA this thread issued has completed before TMEM is released.
@@ -641,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         float mt = -INFINITY;
         if (ok) {
           tc_fence_after();
-          const int limit = visible_prefix<M>(it, a, row_tok[i], j) - part * kCols;  // in this part
+          const int limit = visible_prefix<M>(it, a, row_tok[i], j, q) - part * kCols;  // in this part
           // Most tiles are fully visible: mask only when some row of the warp needs it.
           const bool masked = __any_sync(0xffffffffu, limit < kCols);
           // S in pieces of 32: the max over the first pieces overlaps the TMEM read of
@@ -756,8 +800,61 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
 #pragma unroll
         for (int o = 1; o < kParts; ++o) l_run[i] += bars->psum[i][(part + o) % kParts][row];
     }
+    bool dual = false;
+    if constexpr (M == Mode::kQuery && kParts > 1) dual = it.dual;
+    if (dual) {
+      // Both tiles hold this row over disjoint halves of the chunk's keys: combine
+      // the two partial softmaxes exactly (the Phase-2 merge within one CTA) and
+      // store one partial.
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&bars->o_bar[q], 0, bars, a.status));
+      tc_fence_after();
+      if (ok) {
+        pdl_wait();  // the partials may still be read by the previous kernel
+        const float M2 = fmaxf(m_run[0], m_run[kTilesPerWarp - 1]);
+        float wq[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          wq[q] = (M2 == -INFINITY || m_run[q % kTilesPerWarp] == -INFINITY)
+                      ? 0.f : ex2_approx((m_run[q % kTilesPerWarp] - M2) * sl2);
+        const float l = l_run[0] * wq[0] + l_run[kTilesPerWarp - 1] * wq[1];
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float lse2 = l > 0.f ? M2 * sl2 + log2f(l) : -INFINITY;
+        const int tok = static_cast<int>(row_tok[0]);
+        const int hq = head[0];
+        const int64_t o_off = ((it.rbase + tok) * a.hq + hq) * D + part * kOCols;
+        const bool valid = tok < it.lq && STAR_IN_BOUNDS(a.status, o_off + kOCols - 1, out_rows * a.hq * D);
+        float* dst = a.o_parts + o_off;
+#pragma unroll
+        for (int c = 0; c < kOCols / kOP; ++c) {
+          uint32_t o0[kOP], o1[kOP];
+          if constexpr (kOP == 32) {
+            tmem_ld32(lane_addr + 256 + part * kOCols + c * 32, o0);
+            tmem_ld32(lane_addr + 256 + D + part * kOCols + c * 32, o1);
+          } else {
+            tmem_ld16(lane_addr + 256 + part * kOCols + c * 16, o0);
+            tmem_ld16(lane_addr + 256 + D + part * kOCols + c * 16, o1);
+          }
+          tmem_wait_ld();
+          float v[kOP];
+#pragma unroll
+          for (int e = 0; e < kOP; ++e)
+            v[e] = (__uint_as_float(o0[e]) * wq[0] + __uint_as_float(o1[e]) * wq[1]) * inv;
+          if (valid) {
+            float4* d4 = reinterpret_cast<float4*>(dst + c * kOP);
+#pragma unroll
+            for (int u = 0; u < kOP / 4; ++u) d4[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+          }
+        }
+        const int64_t l_off = it.rbase * a.hq + static_cast<int64_t>(hq) * it.lq + tok;
+        if (valid && part == 0 && STAR_IN_BOUNDS(a.status, l_off, out_rows * a.hq))
+          a.lse_parts[l_off] = lse2 * 0.69314718055994531f;
+      }
+    }
 #pragma unroll
     for (int i = 0; i < kTilesPerWarp; ++i) {
+      if (dual) break;
       const int q = kParts > 1 ? i : sw;
       const uint32_t o_col = 256 + q * D + part * kOCols;
       if (ok) ok = __all_sync(0xffffffffu, wait_or_abort(&bars->o_bar[q], 0, bars, a.status));

@@ -272,3 +272,30 @@ def test_phase1_score_jumps_in_later_tiles(boost):
     ro, rl = oracle.phase1(to_np(q), to_np(k), to_np(v), B)
     check_rows(to_np(o), ro, to_np(lse), rl, f"score jump x{boost}")
     assert m.device_status() == 0
+
+
+@pytest.mark.parametrize("peak_tile", [0, 3, 6])
+def test_query_single_q_tile_combines_two_key_streams(peak_tile):
+    """When all query rows fit one 128-row tile, a context split runs the tile twice,
+    over the chunk's even and odd K/V tiles, and combines the two softmaxes: a key
+    that dominates the row may sit in either stream (tile 3 is odd, 0 and 6 even;
+    7 tiles in the chunk, so the odd stream's last step has no keys)."""
+    m = sa()
+    # 80 blocks of 896 keys: the split plan gives one 7-tile chunk per block
+    b, hq, hkv, d, B, lq = 1, 8, 2, 128, 896, 5
+    L = 80 * B
+    w, x = make(b, hq, hkv, d, L, B, lq, 1, seed=7)
+    g = torch.Generator(device="cpu").manual_seed(peak_tile)
+    u = torch.randn(d, generator=g)
+    u = u / u.norm() * 11.0
+    key = peak_tile * 128 + 17
+    x["k_ctx"][0, key, 1] = u.to(torch.bfloat16).cuda()
+    x["q_qry"][0, 2, 5] = u.to(torch.bfloat16).cuda()  # q-head 5 reads kv-head 1
+    kc = torch.zeros((b, lq, hkv, d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    oq, lse = m.phase2_query(x["q_qry"], x["k_qry"], x["v_qry"], x["k_ctx"], x["v_ctx"], kc, vc, B)
+    rq, rl = oracle.phase2_query(to_np(x["q_qry"]), to_np(x["k_qry"]), to_np(x["v_qry"]),
+                                 to_np(x["k_ctx"]), to_np(x["v_ctx"]))
+    check_rows(to_np(oq), rq, to_np(lse), rl, f"single-tile query, peak in tile {peak_tile}")
+    assert float(rl[0, 5, 2]) > 10.0  # the planted key dominates that row
+    assert m.device_status() == 0
