@@ -95,9 +95,12 @@ def recorded_traffic(kind: str, w, algorithmic_bytes: float):
         if e.get("workload") == w.name:
             return e["dram_bytes_per_launch"], f"ncu on {w.name}"
     for e in entries:
-        if e.get("block_size") == w.block_size:
+        # Phase 1 scales between captures of one block size; a decode step reads every
+        # KV byte once whatever the block size, so any decode capture scales.
+        if e.get("block_size") == w.block_size or kind.startswith("decode"):
             ratio = e["dram_bytes_per_launch"] / e["algorithmic_bytes_per_launch"]
-            return ratio * algorithmic_bytes, (f"ncu on {e['workload']} (same block size), scaled by "
+            same = "same block size" if e.get("block_size") == w.block_size else "every KV byte once"
+            return ratio * algorithmic_bytes, (f"ncu on {e['workload']} ({same}), scaled by "
                                                f"algorithmic bytes ({ratio:.3f} x)")
     return None, "no capture with this workload or block size"
 
