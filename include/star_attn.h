@@ -55,7 +55,7 @@ typedef struct CUstream_st* star_stream_t;
 typedef enum {
   STAR_OK = 0,
   STAR_ERR_INVALID_ARG = 1,  /* null or misaligned pointer, inconsistent shape */
-  STAR_ERR_UNSUPPORTED = 2,  /* a shape this build does not implement (head_dim not 64/128) */
+  STAR_ERR_UNSUPPORTED = 2,  /* a shape the library does not implement (head_dim not 64/128, GQA group not 1/2/4/8) */
   STAR_ERR_WORKSPACE = 3,    /* workspace missing or smaller than star_attn_workspace_bytes() */
   STAR_ERR_CACHE_FULL = 4,   /* the query-local cache has no room for the rows to append */
   STAR_ERR_CUDA = 5,         /* a CUDA runtime call or a kernel launch failed */
