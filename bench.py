@@ -342,7 +342,7 @@ def sharded_e2e(step: ShardedStep, steps: int, world: int, device):
             o += [t for t in pair if t is not None]
         return o
 
-    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outputs()]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outputs()]
     d2h = sum(t.numel() * t.element_size() for t in host_out)
     barrier(world)
     torch.cuda.synchronize()
@@ -364,11 +364,12 @@ def sharded_e2e(step: ShardedStep, steps: int, world: int, device):
             "bytes_are": "this rank's (rank 0)"}
 
 
-def run_sharded(args, w, world, rank, local):
+def run_sharded(args, w, world, rank, local, device=None):
     """The pages' multi-host form across the ranks of this job (strong scaling: one
-    context of the workload split over all GPUs). Prints one JSON line on rank 0."""
+    context of the workload split over all GPUs). Prints one JSON line on rank 0.
+    `device` defaults to this rank's GPU."""
     import block_sparse_attention_phase_b200 as sa
-    device = torch.device("cuda", local)
+    device = torch.device("cuda", local) if device is None else device
     torch.cuda.set_device(device)
     x = workloads.make_inputs(w, device=device, seed=w.seed)  # identical on every rank
     step = ShardedStep(w, x, device)

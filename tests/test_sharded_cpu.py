@@ -192,3 +192,80 @@ def test_bench_sharded_step_on_gloo_ranks(tmp_path):
                                              x["k_ctx"], x["v_ctx"], kc, vc, w.query_len + t)
         np.testing.assert_allclose(np.array(host["dec"][t]), od, atol=1e-12)
     assert all(r["oq"] is None for r in res[:-1])
+
+
+class _HostEvent:
+    """Stand-in for torch.cuda.Event on the host: wall-clock stamps."""
+
+    def __init__(self, enable_timing=False):
+        self.t = None
+
+    def record(self, stream=None):
+        import time
+        self.t = time.perf_counter()
+
+    def synchronize(self):
+        pass
+
+    def elapsed_time(self, other):
+        return (other.t - self.t) * 1e3
+
+
+class _Float64Step:
+    """bench.ShardedStep with the oracle as compute on float64 copies of the inputs."""
+
+    def __new__(cls, w, x, device):
+        import bench
+        return bench._RealShardedStep(w, {k: t.double() for k, t in x.items()}, device,
+                                      backend=OracleBackend(), dtype=torch.float64)
+
+
+def _run_sharded_worker(rank, world, port, out_dir):
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "RANK": str(rank),
+                       "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank)})
+    sys.path.insert(0, ROOT)
+    import contextlib
+    import io
+    import bench
+    import workloads
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # the CUDA calls of the timing harness, replaced by host stand-ins
+        torch.cuda.Event = _HostEvent
+        torch.cuda.synchronize = lambda *a, **k: None
+        torch.cuda.set_device = lambda *a, **k: None
+        torch.cuda.empty_cache = lambda *a, **k: None
+        torch.cuda.current_device = lambda: 0
+        torch.Tensor.pin_memory = lambda self: self
+        bench._RealShardedStep = bench.ShardedStep
+        bench.ShardedStep = _Float64Step
+        w = workloads.Workload("bench-sharded", 1, 4, 2, 16, 70, 16, 3, 2, 0, 5)
+
+        class Args:
+            steps, warmup, no_e2e = 2, 3, False
+        buf = io.StringIO()
+        with contextlib.redirect_stdout(buf):
+            rc = bench.run_sharded(Args, w, world, rank, rank, device=torch.device("cpu"))
+        with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
+            f.write(f"{rc}\n{buf.getvalue()}")
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+def test_bench_run_sharded_on_gloo_ranks(tmp_path):
+    """bench.py's multi-GPU mode end to end on 2 gloo ranks (timing calls on the
+    host, the oracle as compute): warm-up, the timed steps with their collectives,
+    the max over ranks, the end-to-end pass and rank 0's JSON line."""
+    world = 2
+    mp.start_processes(_run_sharded_worker, args=(world, _free_port(), str(tmp_path)),
+                       nprocs=world, join=True, start_method="spawn")
+    outs = [open(tmp_path / f"rank{r}.txt").read().split("\n", 1) for r in range(world)]
+    assert all(rc == "0" for rc, _ in outs)
+    assert outs[1][1].strip() == ""  # only rank 0 prints
+    line = json.loads(outs[0][1].strip().splitlines()[-1])
+    assert line["n_gpus"] == 2 and line["scaling"] == "strong" and line["steps"] == 2
+    assert line["config"]["parallelism"] == "star-sharded2" and line["value"] > 0
+    assert line["e2e"]["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] > 0
+    for k in ("phase1", "query", "decode", "roofline", "clocks", "gpu_launches"):
+        assert k in line
