@@ -183,11 +183,11 @@ __device__ __forceinline__ Split locate(const DecodeArgs& a, const VL& dv) {
 //
 // The combine is bound by L2 latency, so it takes as few round trips as possible:
 // one gpu-scope fence and one atomic per CTA (the grid-barrier pattern: the CTA's
-// stores, a CTA barrier, then one thread's fence and count); in the last CTA the
-// splits' partial blocks are copied into shared memory with asynchronous 16-byte
-// copies, issued before the LSEs are read so that both are in flight together.
-// Each thread then owns float4 columns of the G x d output and sums over the
-// staged splits from shared memory.
+// stores, a CTA barrier, then one thread's fence and count); in the last CTA one
+// thread copies each split's partial block (G x d fp32, contiguous) into shared
+// memory with one 1-D bulk copy on an mbarrier, issued before the LSEs are read so
+// that both are in flight together. Each thread then owns float4 columns of the
+// G x d output and sums over the staged splits from shared memory.
 template <int D, int G, class VL>
 __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const VL& dv, const Split& w,
                                               uint8_t* smem) {
@@ -195,6 +195,7 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const VL& dv,
   constexpr int F = G * D / 4;  // float4 columns of one split's G x D block
   __shared__ int s_last;
   __shared__ float s_m[G], s_w[G];
+  __shared__ alignas(8) uint64_t s_staged;  // the bulk copies of one staging pass landed
   const int tid = threadIdx.x;  // 0 .. 127 (the consumer warps)
   asm volatile("bar.sync 1, %0;" ::"r"(kThreads) : "memory");  // every partial store issued
   if (tid == 0) {
@@ -222,17 +223,30 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const VL& dv,
   float4* parts = reinterpret_cast<float4*>(smem + fused_weights_bytes(S, G));  // [nb][F]
   const uint32_t parts_s = smem_u32(parts);
 
-  // Copies of splits sp0 .. sp0 + nb - 1 into the staging area (L2 only: the
-  // partials were written by other SMs).
+  // Copies of splits sp0 .. sp0 + nb - 1 into the staging area, one bulk copy of
+  // G x D floats per split, completing on s_staged (thread 0 issues them).
+  constexpr uint32_t kBlockBytes = G * D * 4;
+  if (tid == 0) {
+    mbar_init(&s_staged, 1);
+    fence_barrier_init();
+    // The partials were written by other CTAs (generic stores, acquired through the
+    // counter above); the bulk copies below read them through the async proxy.
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  }
   auto stage = [&](int sp0) {
-    const int cnt = min(nb, S - sp0) * F;
-    for (int i = tid; i < cnt; i += kThreads) {
-      const float* src = a.o_parts + (row0 + static_cast<int64_t>(sp0 + i / F) * stride) * D + 4 * (i % F);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(parts_s + 16u * i), "l"(src)
-                   : "memory");
+    if (tid != 0) return;
+    const int cnt = min(nb, S - sp0);
+    mbar_arrive_expect_tx(&s_staged, cnt * kBlockBytes);
+    for (int j = 0; j < cnt; ++j) {
+      const float* src = a.o_parts + (row0 + static_cast<int64_t>(sp0 + j) * stride) * D;
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              parts_s + j * kBlockBytes),
+          "l"(src), "r"(kBlockBytes), "r"(smem_u32(&s_staged))
+          : "memory");
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
   };
+  int pass = 0;
   // 1. the LSEs -> shared memory (the first 4 per thread are loaded before the
   //    staging copies are issued, so that they do not queue behind them); per head
   //    (warp h % 4, lanes over the splits) the maximum M, the weights exp(lse_s - M)
@@ -278,9 +292,11 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const VL& dv,
   float4 acc[KPT];
 #pragma unroll
   for (int k = 0; k < KPT; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int sp0 = 0; sp0 < S; sp0 += nb) {
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    asm volatile("bar.sync 1, %0;" ::"r"(kThreads) : "memory");  // staged blocks and weights ready
+  for (int sp0 = 0; sp0 < S; sp0 += nb, ++pass) {
+    // staged blocks landed (a second bounded wait after a timeout: no copy may
+    // still be in flight when the CTA moves on)
+    if (!mbar_wait(&s_staged, pass & 1, a.status)) mbar_wait(&s_staged, pass & 1, a.status);
+    asm volatile("bar.sync 1, %0;" ::"r"(kThreads) : "memory");  // and the weights are ready
     const int cnt = min(nb, S - sp0);
 #pragma unroll
     for (int k = 0; k < KPT; ++k) {
@@ -299,6 +315,7 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const VL& dv,
     }
     if (sp0 + nb < S) {
       asm volatile("bar.sync 1, %0;" ::"r"(kThreads) : "memory");  // staging area free again
+      if (tid == 0) fence_proxy_async_smem();  // the reads above precede the copies that overwrite it
       stage(sp0 + nb);
     }
   }
