@@ -9,9 +9,11 @@
 //
 // One warp per output row (batch, token, head), eight rows per CTA. The lanes
 // first take the splits' LSEs (32 at a time) for the maximum M and the weights
-// exp(lse_s - M); then each lane owns d/32 contiguous elements of the row and sums
-// the splits' partial rows (coalesced 512- or 256-byte warp reads), with the loads
-// of several splits in flight at once. Every partial is read once.
+// exp(lse_s - M); each lane owns d/32 contiguous elements of the row and sums the
+// splits' partial rows (coalesced 512- or 256-byte warp reads) in split order. The
+// reads of the first eight splits go out with the LSE reads and each later group of
+// eight while the one before is summed: the merge is bound by L2 latency, not
+// bandwidth. Every partial is read once.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -21,6 +23,7 @@ namespace star {
 namespace {
 
 constexpr int kRowsPerCta = 8;
+constexpr int kGroup = 8;  // partial rows of a warp in flight per group
 
 // Varlen query pass: one row per (packed query token, head); the token's sequence
 // (binary search in vs.start) gives its split count and partial rows: split s of
@@ -74,9 +77,28 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) merge_kernel(
     out_lse = lse_off;
   }
 
-  // M = max over splits (lanes over splits)
-  float M = -INFINITY;
-  for (int s = lane; s < S; s += 32) M = fmaxf(M, lse_parts[s * lse_stride + lse_off]);
+  // Partial row of split sp: E contiguous floats per lane (one coalesced warp read).
+  auto load_row = [&](int sp, float (&x)[E]) {
+    const float* r = o_parts + static_cast<int64_t>(sp) * o_stride + o_off;
+    if constexpr (E == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(r);
+      x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(r);
+      x[0] = v.x; x[1] = v.y;
+    }
+  };
+  // The partial rows do not depend on the weights: the first kGroup of them are
+  // requested together with the LSEs, and every later group while the previous one
+  // is summed, so a row costs about one L2 round trip per kGroup splits.
+  float xa[kGroup][E];
+#pragma unroll
+  for (int u = 0; u < kGroup; ++u)
+    if (u < S) load_row(u, xa[u]);
+  // M = max over splits (lanes over splits; lane k keeps the LSE of split k)
+  const float lse0 = lane < S ? lse_parts[lane * lse_stride + lse_off] : -INFINITY;
+  float M = lse0;
+  for (int sp = lane + 32; sp < S; sp += 32) M = fmaxf(M, lse_parts[sp * lse_stride + lse_off]);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
 
@@ -88,34 +110,29 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) merge_kernel(
     for (int s0 = 0; s0 < S; s0 += 32) {
       const int cnt = S - s0 < 32 ? S - s0 : 32;
       // lane k holds the weight of split s0 + k (0 for an empty split)
-      const float w = lane < cnt ? expf(lse_parts[(s0 + lane) * lse_stride + lse_off] - M) : 0.f;
+      const float lv = s0 == 0 ? lse0 : (lane < cnt ? lse_parts[(s0 + lane) * lse_stride + lse_off] : 0.f);
+      const float w = lane < cnt ? expf(lv - M) : 0.f;
       W += w;
-      const float* src = o_parts + static_cast<int64_t>(s0) * o_stride + o_off;
-      int k = 0;
-      for (; k + 4 <= cnt; k += 4) {  // four splits' rows in flight
-        float x[4][E];
+      for (int g = 0; g < cnt; g += kGroup) {
+        float xb[kGroup][E];
+        const int nx = s0 + g + kGroup;  // the next group (32 is a multiple of kGroup)
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if constexpr (E == 4) {
-            const float4 v = *reinterpret_cast<const float4*>(src + (k + u) * o_stride);
-            x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
-          } else {
-            const float2 v = *reinterpret_cast<const float2*>(src + (k + u) * o_stride);
-            x[u][0] = v.x; x[u][1] = v.y;
+        for (int u = 0; u < kGroup; ++u)
+          if (nx + u < S) load_row(nx + u, xb[u]);
+#pragma unroll
+        for (int u = 0; u < kGroup; ++u) {
+          if (g + u < cnt) {
+            const float wu = __shfl_sync(0xffffffffu, w, g + u);
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[e] += wu * xa[u][e];
           }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float wu = __shfl_sync(0xffffffffu, w, k + u);
+        for (int u = 0; u < kGroup; ++u)
+          if (nx + u < S) {
 #pragma unroll
-          for (int e = 0; e < E; ++e) acc[e] += wu * x[u][e];
-        }
-      }
-      for (; k < cnt; ++k) {
-        const float wk = __shfl_sync(0xffffffffu, w, k);
-        const float* r = src + k * o_stride;
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] += wk * r[e];
+            for (int e = 0; e < E; ++e) xa[u][e] = xb[u][e];
+          }
       }
     }
   }

@@ -91,16 +91,27 @@ def test_phase1_deterministic():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-def test_lse_merge_kernel_against_oracle():
-    g = torch.Generator(device="cpu").manual_seed(5)
-    S, b, T, H, d = 7, 2, 3, 4, 128
+@pytest.mark.parametrize("S,d", [(7, 128), (1, 128), (8, 128), (9, 128), (17, 128), (33, 128),
+                                 (70, 128), (19, 64), (41, 64)])
+def test_lse_merge_kernel_against_oracle(S, d):
+    """Split counts on both sides of the kernel's groups of 8 partial rows and its
+    32-split LSE chunks, an empty split, and one row every split of which is empty."""
+    g = torch.Generator(device="cpu").manual_seed(5 + S)
+    b, T, H = 2, 3, 4
     o_parts = torch.randn(S, b, T, H, d, generator=g)
     lse_parts = torch.randn(S, b, H, T, generator=g) * 3
-    lse_parts[2] = float("-inf")  # an empty split
+    if S > 1:
+        lse_parts[S // 2] = float("-inf")  # an empty split
+    lse_parts[:, 1, 2, 0] = float("-inf")  # a row that no split saw
     o, lse = sa().lse_merge(o_parts.cuda(), lse_parts.cuda())
     ro, rl = oracle.lse_merge(o_parts.numpy().transpose(0, 1, 3, 2, 4),
                               lse_parts.numpy())  # oracle wants [S, b, H, T, d]
-    check_rows(to_np(o).transpose(0, 2, 1, 3), ro, to_np(lse), rl, "merge")
+    og, lg = to_np(o).transpose(0, 2, 1, 3), to_np(lse).copy()
+    # the empty row: lse -inf and a zero output on both sides
+    assert np.isneginf(lg[1, 2, 0]) and np.isneginf(rl[1, 2, 0]) and not og[1, 2, 0].any()
+    rl = rl.copy()
+    lg[1, 2, 0] = rl[1, 2, 0] = 0.0
+    check_rows(og, ro, lg, rl, "merge")
 
 
 def test_simple_kernels_agree_with_oracle():
