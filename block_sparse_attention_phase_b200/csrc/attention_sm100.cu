@@ -22,12 +22,14 @@
 // Work items are ordered so that the tiles of one block run together (their
 // K/V and the anchor's stay in L2), blocks i > 0 before b_0, longer rows first.
 //
-// CTA = 3 warpgroups (12 warps):
+// CTA = 3 warpgroups (12 warps; 5 with STAR_SOFTMAX_PARTS = 4):
 //   warpgroup 0  warp 0: TMA producer (both Q tiles once, then K and V tiles
 //                into 2-stage rings); warp 1: TMEM allocator and MMA issuer
-//                (one thread); warps 2-3 idle. Registers trimmed to 40.
-//   warpgroups 1, 2  the softmax of Q tile 0 and of Q tile 1, one thread per row
-//                (TMEM lane = row), registers raised to 232.
+//                (one thread); warps 2-3 idle. Registers trimmed to 104.
+//   warpgroups 1, 2  the softmax, one thread per row (TMEM lane = row): each
+//                takes one half (64 key columns) of both Q tiles' scores, tile 0
+//                then tile 1 at every step, the halves of a row trading their
+//                partial maxima through shared memory. Registers raised to 200.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256, 256+d), O_1 [256+d, 256+2d).
 // MMA order (one thread): S_0(0), S_1(0), then for every K/V tile j
 //   O_0 += P_0(j) V_j, S_0(j+1), O_1 += P_1(j) V_j, S_1(j+1),
