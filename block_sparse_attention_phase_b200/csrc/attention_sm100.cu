@@ -106,6 +106,16 @@ struct AttnArgs {
   // paged query-local cache (page_table == null: contiguous)
   const int32_t* page_table;  // [b, max_pages]
   int32_t page_size, max_pages;
+  // Query pass of a uniform batch: the cache split reads the query tokens' K/V from
+  // the inputs (maps tk2/tv2 over [b, Lq, Hkv, d]), and the cache append is done in
+  // this kernel (cw_k == null: the cache was written before, the cache split reads it).
+  const uint4* cw_k;  // [b, Lq, Hkv, d] as 16-byte words
+  const uint4* cw_v;
+  uint4* cw_kc;       // contiguous cache [b, cap, Hkv, d] or page pool [pages, P, Hkv, d]
+  uint4* cw_vc;
+  int64_t cw_cap;
+  const int32_t* cw_table;  // [b, cw_max_pages] or null
+  int32_t cw_page, cw_max_pages, cw_num_pages;
 };
 
 struct Bars {
@@ -435,7 +445,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         }
       }
       if constexpr (M == Mode::kQuery) {
-        if (it.cache) pdl_wait();  // the cache rows this pass reads were just written
+        // the cache rows this pass reads were just written by the previous kernel
+        // (when they come from the inputs, nothing needs to wait)
+        if (it.cache && a.cw_k == nullptr) pdl_wait();
       }
       // Anchor-position variant: the anchor tiles see Q rotated at the anchor
       // positions (map tk2); after them, Q is reloaded from tq for the own block.
@@ -626,6 +638,46 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       // Every MMA this thread issued has completed before TMEM is released.
       tc_commit(&bars->drain);
       mbar_wait(&bars->drain, 0, a.status);
+    } else if (warp >= 2) {
+      if constexpr (M == Mode::kQuery) {
+        // ------------------------------------------------------------ cache append
+        // The cache split's CTA of the first q-tile pair appends its (sequence,
+        // kv-head)'s query K/V rows to the query-local cache: rows [0, Lq), and for
+        // a paged cache zeros up to the end of the last page (later tiles read
+        // those rows). It waits for the previous kernel, which may still read the
+        // cache. A page id outside the pool is refused (bounds flag, no write).
+        if (a.cw_k != nullptr && it.cache && it.tok0[0] == 0) {
+          pdl_wait();
+          constexpr int W = D / 8;  // 16-byte words of one row of one kv-head
+          const int64_t lq = it.lq;
+          const int64_t ext = a.cw_table ? (lq + a.cw_page - 1) / a.cw_page * a.cw_page : lq;
+          const int64_t cache_rows = a.cw_table ? static_cast<int64_t>(a.cw_num_pages) * a.cw_page
+                                                : static_cast<int64_t>(a.b) * a.cw_cap;
+          for (int64_t i = (warp - 2) * 32 + lane; i < ext * W; i += 64) {
+            const int64_t r = i / W;
+            const int e = static_cast<int>(i % W);
+            int64_t drow = static_cast<int64_t>(it.bb) * a.cw_cap + r;
+            if (a.cw_table) {
+              const int64_t page = a.cw_table[static_cast<int64_t>(it.bb) * a.cw_max_pages + r / a.cw_page];
+              if (page < 0 || page >= a.cw_num_pages) {
+                report(a.status, kBoundsFlag);
+                continue;
+              }
+              drow = page * a.cw_page + r % a.cw_page;
+            }
+            if (!STAR_IN_BOUNDS(a.status, drow, cache_rows)) continue;
+            const int64_t dst = (drow * a.hkv + it.kvh) * W + e;
+            if (r < lq) {
+              const int64_t src = ((static_cast<int64_t>(it.bb) * lq + r) * a.hkv + it.kvh) * W + e;
+              a.cw_kc[dst] = a.cw_k[src];
+              a.cw_vc[dst] = a.cw_v[src];
+            } else {
+              a.cw_kc[dst] = make_uint4(0u, 0u, 0u, 0u);
+              a.cw_vc[dst] = make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
+        }
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroups
@@ -1087,31 +1139,37 @@ cudaError_t launch_phase1_varlen_t(const Shape& s, const int64_t* cu, const void
 }
 
 template <int D>
-cudaError_t launch_query_t(const Shape& s, const SplitPlan& p, const void* q, int64_t lq,
-                           const void* kc, const void* vc, const CacheRef& c, float* o_parts,
-                           float* lse_parts, cudaStream_t st) {
+cudaError_t launch_query_t(const Shape& s, const SplitPlan& p, const void* q, const void* k_new,
+                           const void* v_new, int64_t lq, const void* kc, const void* vc,
+                           const CacheRef& c, float* o_parts, float* lse_parts, cudaStream_t st,
+                           bool write_cache) {
   const int G = s.group();
   alignas(64) CUtensorMap m[5];
   bool ok = encode_tma_bf16_4d(&m[0], q, D, s.hq, lq, lq, s.b, 64, G, 128 / G, true) &&
             encode_tma_bf16_4d(&m[1], kc, D, s.hkv, s.L, s.L, s.b, 64, 1, 128, true) &&
             encode_tma_bf16_4d(&m[2], vc, D, s.hkv, s.L, s.L, s.b, 64, 1, 128, true);
-  if (c.paged()) {
-    // the page pool [pages, P, Hkv, d]; rows past Lq in the last page were zeroed
-    // by the cache write of this call
-    ok = ok &&
-         encode_tma_bf16_4d(&m[3], c.k, D, s.hkv, c.page_size, c.page_size, c.num_pages, 64, 1, 128, true) &&
-         encode_tma_bf16_4d(&m[4], c.v, D, s.hkv, c.page_size, c.page_size, c.num_pages, 64, 1, 128, true);
-  } else {
-    // only the Lq rows written by this call are in bounds: rows past them
-    // (unwritten, any bytes) read as zeros, so P = 0 never meets a NaN there
-    ok = ok && encode_tma_bf16_4d(&m[3], c.k, D, s.hkv, lq, c.cap, s.b, 64, 1, 128, true) &&
-         encode_tma_bf16_4d(&m[4], c.v, D, s.hkv, lq, c.cap, s.b, 64, 1, 128, true);
-  }
+  // The cache split's keys are exactly this call's query tokens: it reads them from
+  // the inputs [b, Lq, Hkv, d] (rows past Lq read as zeros, so P = 0 never meets
+  // whatever bytes the cache holds there). Without them (no cache split) the maps
+  // only stand in.
+  const void* ks = k_new ? k_new : kc;
+  const void* vsrc = v_new ? v_new : vc;
+  const int64_t rows = k_new ? lq : s.L;
+  ok = ok && encode_tma_bf16_4d(&m[3], ks, D, s.hkv, rows, rows, s.b, 64, 1, 128, true) &&
+       encode_tma_bf16_4d(&m[4], vsrc, D, s.hkv, rows, rows, s.b, 64, 1, 128, true);
   if (!ok) return cudaErrorInvalidValue;
   AttnArgs a = base_args(s);
-  a.page_table = c.page_table;
-  a.page_size = c.page_size;
-  a.max_pages = c.max_pages;
+  if (write_cache && k_new) {
+    a.cw_k = static_cast<const uint4*>(k_new);
+    a.cw_v = static_cast<const uint4*>(v_new);
+    a.cw_kc = static_cast<uint4*>(c.k);
+    a.cw_vc = static_cast<uint4*>(c.v);
+    a.cw_cap = c.cap;
+    a.cw_table = c.page_table;
+    a.cw_page = c.page_size;
+    a.cw_max_pages = c.max_pages;
+    a.cw_num_pages = c.num_pages;
+  }
   a.lq = lq;
   a.chunk = p.chunk;
   a.spb = p.spb;
@@ -1240,12 +1298,14 @@ cudaError_t launch_phase1_varlen(const Shape& s, const int64_t* cu_seqlens, cons
   return launch_phase1_varlen_t<64>(s, cu_seqlens, q, k, v, o, lse, st);
 }
 
-cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q, int64_t lq,
+cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q,
+                              const void* k_new, const void* v_new, int64_t lq,
                               const void* kc, const void* vc, const CacheRef& c, float* o_parts,
                               float* lse_parts, void* o, float* lse, cudaStream_t st,
-                              bool o_fp32) {
-  cudaError_t e = s.d == 128 ? launch_query_t<128>(s, p, q, lq, kc, vc, c, o_parts, lse_parts, st)
-                             : launch_query_t<64>(s, p, q, lq, kc, vc, c, o_parts, lse_parts, st);
+                              bool o_fp32, bool write_cache) {
+  cudaError_t e =
+      s.d == 128 ? launch_query_t<128>(s, p, q, k_new, v_new, lq, kc, vc, c, o_parts, lse_parts, st, write_cache)
+                 : launch_query_t<64>(s, p, q, k_new, v_new, lq, kc, vc, c, o_parts, lse_parts, st, write_cache);
   if (e != cudaSuccess) return e;
   return launch_merge(o_parts, lse_parts, p.n_splits, s.b, lq, s.hq, s.d, o, lse, st, o_fp32);
 }

@@ -119,48 +119,13 @@ __global__ void __launch_bounds__(kWarps * 32) simple_phase2_kernel(
           lse ? lse + (static_cast<int64_t>(bb) * s.hq + h) * rows + r_tok : nullptr, lane);
 }
 
-// Cache rows [0, rows) <- k, v [b, rows, Hkv, d] with 16-byte copies. A
-// contiguous cache is [b, cap, Hkv, d]; a paged one puts row r of sequence b in
-// row r % P of page table[b * max_pages + r / P] of a [pages, P, Hkv, d] pool, and
-// the rows after `rows` up to the end of that page are written with zeros (`ext`
-// = rows rounded up to P), so that later tiles read zeros there. A page id outside
+// Varlen cache write (the uniform query pass appends its rows inside the partial
+// kernel): sequence i's rows [0, e0[i+1] - e0[i]) of its cache (its query rows,
+// then zeros up to the end of the tile or page) come from packed rows q0[i] .. of
+// k, v [total, Hkv, d]; e0 is the prefix of those row counts. A contiguous cache is
+// [seqs, cap, Hkv, d]; a paged one puts row r of sequence i in row r % P of page
+// table[i * max_pages + r / P] of a [pages, P, Hkv, d] pool. A page id outside
 // [0, num_pages) is refused: the bounds flag is set and nothing is written.
-__global__ void cache_write_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
-                                   int64_t rows, int64_t ext, int32_t b, int32_t hkv, int32_t d,
-                                   uint4* __restrict__ kc, uint4* __restrict__ vc, int64_t cap,
-                                   const int32_t* __restrict__ table, int32_t P,
-                                   int32_t max_pages, int32_t num_pages, uint32_t* status) {
-  const int64_t per_row = static_cast<int64_t>(hkv) * d / 8;  // uint4 per token row
-  const int64_t total = static_cast<int64_t>(b) * ext * per_row;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t e = i % per_row;
-    const int64_t r = (i / per_row) % ext;
-    const int64_t bb = i / (per_row * ext);
-    int64_t drow = bb * cap + r;
-    if (table) {
-      const int64_t page = table[bb * max_pages + r / P];
-      if (page < 0 || page >= num_pages) {
-        atomicOr(status, kBoundsFlag);
-        continue;
-      }
-      drow = page * P + r % P;
-    }
-    const int64_t dst = drow * per_row + e;
-    if (r < rows) {
-      const int64_t src = (bb * rows + r) * per_row + e;
-      kc[dst] = k[src];
-      vc[dst] = v[src];
-    } else {
-      kc[dst] = make_uint4(0u, 0u, 0u, 0u);
-      vc[dst] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-}
-
-// Varlen cache write: sequence i's rows [0, e0[i+1] - e0[i]) of its cache (its
-// query rows, then zeros up to the end of the tile or page) come from packed rows
-// q0[i] .. of k, v [total, Hkv, d]; e0 is the prefix of those row counts.
 struct CacheRows {
   int32_t n;
   int32_t q0[kMaxVarSeqs + 1];
@@ -282,20 +247,5 @@ cudaError_t launch_simple_phase2(const Shape& s, const void* q, int64_t rows, co
   return cudaGetLastError();
 }
 
-cudaError_t launch_cache_write(const Shape& s, const void* k, const void* v, int64_t rows,
-                               const CacheRef& c, cudaStream_t st) {
-  const int64_t ext = c.paged() ? (rows + c.page_size - 1) / c.page_size * c.page_size : rows;
-  const int64_t total = static_cast<int64_t>(s.b) * ext * s.hkv * s.d / 8;
-  if (total == 0) return cudaSuccess;
-  const int threads = 256;
-  const int64_t blocks64 = (total + threads - 1) / threads;
-  const unsigned blocks = static_cast<unsigned>(blocks64 < 4096 ? blocks64 : 4096);
-  cache_write_kernel<<<blocks, threads, 0, st>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), rows, ext, s.b, s.hkv, s.d,
-      static_cast<uint4*>(c.k), static_cast<uint4*>(c.v), c.cap, c.page_table, c.page_size,
-      c.max_pages, c.num_pages, device_status_word());
-  count_launch();
-  return cudaGetLastError();
-}
 
 }  // namespace star

@@ -145,16 +145,16 @@ float* lse_parts_of(void* workspace, const Shape& s, const SplitPlan& p, int64_t
                                   align256(per * s.d * sizeof(float)));
 }
 
-// Phase-2 query pass on validated arguments: cache append, then partials + merge.
+// Phase-2 query pass on validated arguments: partials (whose kernel also appends the
+// query K/V to the cache) + merge.
 star_status_t run_query(const Shape& s, const void* q, const void* k, const void* v,
                         int64_t query_len, const void* k_ctx, const void* v_ctx,
                         const CacheRef& c, void* o, float* lse, void* workspace,
                         cudaStream_t cs) {
   const SplitPlan plan = query_plan(s, query_len);
-  cudaError_t e = launch_cache_write(s, k, v, query_len, c, cs);
-  if (e != cudaSuccess) return STAR_ERR_CUDA;
-  e = launch_query_path(s, plan, q, query_len, k_ctx, v_ctx, c, static_cast<float*>(workspace),
-                        lse_parts_of(workspace, s, plan, query_len), o, lse, cs);
+  const cudaError_t e =
+      launch_query_path(s, plan, q, k, v, query_len, k_ctx, v_ctx, c, static_cast<float*>(workspace),
+                        lse_parts_of(workspace, s, plan, query_len), o, lse, cs, false, true);
   return e == cudaSuccess ? STAR_OK : STAR_ERR_CUDA;
 }
 
@@ -587,11 +587,8 @@ STAR_ATTN_API star_status_t star_attn_phase2_partial(
     if (e != cudaSuccess) return STAR_ERR_CUDA;
     e = star::launch_merge(o_parts, lse_parts, plan.n_splits, s.b, 1, s.hq, s.d, o32, lse, cs, true);
   } else {
-    if (has_cache) {
-      e = star::launch_cache_write(s, k, v, rows, c, cs);
-      if (e != cudaSuccess) return STAR_ERR_CUDA;
-    }
-    e = star::launch_query_path(s, plan, q, rows, kc, vc, c, o_parts, lse_parts, o32, lse, cs, true);
+    e = star::launch_query_path(s, plan, q, has_cache ? k : nullptr, has_cache ? v : nullptr, rows, kc,
+                                vc, c, o_parts, lse_parts, o32, lse, cs, true, has_cache);
   }
   return star::cuda_status(e);
 }

@@ -127,10 +127,6 @@ cudaError_t launch_simple_phase2(const Shape& s, const void* q, int64_t rows, co
 cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int32_t n_splits,
                          int32_t b, int64_t tokens, int32_t heads, int32_t d, void* o,
                          float* lse, cudaStream_t st, bool o_fp32 = false);
-// Cache rows [0, rows) <- k, v [b, rows, Hkv, d]; for a paged cache, also zero
-// the rest of the page holding row rows-1.
-cudaError_t launch_cache_write(const Shape& s, const void* k, const void* v, int64_t rows,
-                               const CacheRef& c, cudaStream_t st);
 // Outputs of a decode step whose partial kernel also merges (the last CTA of each
 // (sequence, kv-head) combines the splits); counters [b * Hkv] must be zero before
 // the launch and are zero again after it.
@@ -172,11 +168,15 @@ cudaError_t launch_phase1_anchored(const Shape& s, const void* q, const void* k,
 cudaError_t launch_phase1_varlen(const Shape& s, const int64_t* cu_seqlens, const void* q,
                                  const void* k, const void* v, void* o, float* lse,
                                  cudaStream_t st);
-// Phase-2 query tokens after their KV is in the cache: partials + merge into o/lse.
-cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q, int64_t lq,
+// Phase-2 query tokens: partials + merge into o/lse. The cache split reads the query
+// tokens' K/V from k_new/v_new [b, lq, Hkv, d]; with write_cache the partial kernel
+// also appends them to the cache c (rows [0, lq), zeros to the end of a paged
+// cache's last page).
+cudaError_t launch_query_path(const Shape& s, const SplitPlan& p, const void* q,
+                              const void* k_new, const void* v_new, int64_t lq,
                               const void* kc, const void* vc, const CacheRef& c, float* o_parts,
                               float* lse_parts, void* o, float* lse, cudaStream_t st,
-                              bool o_fp32 = false);
+                              bool o_fp32, bool write_cache);
 // RoPE on q [b, L, Hq, d] and k [b, L, Hkv, d] at positions pos0 + t (in place
 // allowed); q_anchor (or null) gets q rotated at the anchor-variant positions.
 cudaError_t launch_rope(const Shape& s, const float* inv_freq, int64_t pos0, const void* q_in,
