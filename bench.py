@@ -916,7 +916,7 @@ def main(argv=None):
     t_flop = q_flops / (peaks["bf16_tflops"] * 1e12)
     t_byte = q_bytes / (peaks["hbm_gbs"] * 1e9)
     q_bound = "tensor" if t_flop >= t_byte else "hbm"
-    rl_q = {"bound": q_bound, "kernel": "phase2_query (cache write + partials + merge)",
+    rl_q = {"bound": q_bound, "kernel": "phase2_query (partials with the cache append + merge)",
             "achieved": (q_flops / (q_avg / 1e3) / 1e12 if q_bound == "tensor"
                          else q_bytes / (q_avg / 1e3) / 1e9),
             "peak": peaks["bf16_tflops"] if q_bound == "tensor" else peaks["hbm_gbs"],
