@@ -171,3 +171,43 @@ def test_phase1_varlen_rejects_bad_offsets():
     assert call([0] + list(range(1, 130)), 129) == 2  # 129 sequences: more than 128
     s = sa.make_shape(2, 4, 2, 128, 9, 64)
     assert L.star_attn_phase1_varlen(ctypes.byref(s), None, F, F, F, F, None, None) == 1
+
+
+def _plan(b, hkv, L, B, target):
+    """The split plan the library documents: per (batch, kv-head), the query-local
+    cache split plus context splits that are chunks of one block (at least one per
+    block, at least 64 keys each), as many as bring the CTAs to about `target`."""
+    B = min(B, L)
+    n = -(-L // B)
+    spb = max(1, (target // (b * hkv) - 1) // n)
+    chunk = -(-B // spb)
+    if chunk < 64:
+        chunk = 64
+        spb = -(-B // chunk)
+    return n * spb + 1  # splits: context chunks + the cache
+
+
+def _partial_bytes(splits, b, rows, hq, d):
+    per = splits * b * rows * hq
+    align = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    return align(per * d * 4) + align(per * 4)
+
+
+@pytest.mark.parametrize("b,hq,hkv,d,L,B,lq", [
+    (1, 32, 8, 128, 32768, 4096, 64),        # llama8b-32k: 16 context splits of 2048 + cache
+    (1, 32, 8, 128, 1048576, 32768, 32),     # 1m: 4 x 32 q-rows in one tile pair
+    (2, 64, 8, 128, 131072, 16384, 64),      # 70b-128k shape: G = 8
+    (1, 4, 2, 64, 640, 256, 8),              # small: the 64-key minimum chunk binds
+    (3, 8, 8, 128, 1000, 100000, 300),       # B clamped to L, G = 1, several q-tile pairs
+])
+def test_split_plans_match_their_rule(b, hq, hkv, d, L, B, lq):
+    """Workspace sizes are the fp32 partials of exactly the planned splits: decode
+    aims at 2 CTAs per SM, the query pass at one wave of (splits x q-tile pairs).
+    Without a GPU the library plans for 148 SMs."""
+    sms = 148
+    s = sa.make_shape(b, hq, hkv, d, L, B)
+    dec = _plan(b, hkv, L, B, 2 * sms)
+    assert sa.workspace_bytes(s, sa.STAR_PHASE2_DECODE) == _partial_bytes(dec, b, 1, hq, d)
+    pairs = (-(-(lq * (hq // hkv)) // 128) + 1) // 2
+    qry = _plan(b, hkv, L, B, sms // pairs)
+    assert sa.workspace_bytes(s, sa.STAR_PHASE2_QUERY, lq) == _partial_bytes(qry, b, lq, hq, d)
