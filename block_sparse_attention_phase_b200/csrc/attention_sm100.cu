@@ -368,10 +368,11 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
                                               : (vs.n > 0 ? static_cast<int64_t>(vs.rbase[vs.n])
                                                           : static_cast<int64_t>(a.n_splits) * a.b * a.lq);
   if constexpr (M == Mode::kQuery) {
-    // The query pass is launched programmatically after the cache write: the merge
-    // that follows may be scheduled now (it waits for this grid to finish). This
-    // kernel waits for the previous one before it reads the cache rows or writes
-    // the partials (the previous kernel may be a merge still reading them).
+    // The query pass is launched programmatically: the merge that follows may be
+    // scheduled now (it waits for this grid to finish). This kernel waits for the
+    // previous one before it writes the partials (the previous kernel may be a merge
+    // still reading them), appends to the cache (a decode step may still read it),
+    // or, in the varlen pass, reads the cache rows its separate append just wrote.
     pdl_launch_dependents();
   }
   if (it.n_tiles == 0) {
