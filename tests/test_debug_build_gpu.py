@@ -126,8 +126,11 @@ def test_debug_build_every_kernel_family_stays_in_bounds():
 
 
 def test_normal_build_compiles_the_checks_away():
+    import os
     import torch
     import block_sparse_attention_phase_b200 as sa
+    if os.environ.get("STAR_ATTN_LIBRARY"):
+        pytest.skip("STAR_ATTN_LIBRARY names another build: this test is about the in-tree one")
     assert not sa.debug_build()
     out = torch.zeros(5, dtype=torch.int32, device="cuda")
     sa.selftest_bounds(out, 4)  # no check: the (in-bounds) store of element 4 happens
