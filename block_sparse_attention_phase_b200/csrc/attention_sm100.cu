@@ -407,7 +407,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], 4 * kSoftmaxWarpgroups);  // one arrival per softmax warp
+      // one arrival per softmax warp that holds a part of tile s: all of them when
+      // the columns are split, tile s's own warpgroup otherwise
+      mbar_init(&bars->p_full[s], 4 * (kParts > 1 ? kSoftmaxWarpgroups : 1));
       mbar_init(&bars->o_bar[s], 1);
     }
     mbar_init(&bars->drain, 1);
