@@ -717,6 +717,18 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         rows_valid[i] = 0;
       }
     }
+    // K/V tiles [0, full_upto) are visible in full to every row of this warp, so
+    // they need no mask and no visibility test. Phase 1: the anchor tiles when B is
+    // a multiple of 128, then the own block's tiles wholly below the warp's first
+    // row (row tiles start at multiples of 128 from the block start). Otherwise,
+    // and for the query pass, every tile is tested.
+    int full_upto = 0;
+    if constexpr (M == Mode::kPhase1) {
+      if (it.B % 128 == 0) {
+        const int64_t first = (it.t0[0] < it.t0[1] ? it.t0[0] : it.t0[1]) + q4 * 32 - it.bstart;
+        full_upto = it.n_anchor + static_cast<int>((first + 1) / 128);
+      }
+    }
     float m_run[kTilesPerWarp], l_run[kTilesPerWarp];
 #pragma unroll
     for (int i = 0; i < kTilesPerWarp; ++i) {
@@ -742,9 +754,13 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(
         float mt = -INFINITY;
         if (ok) {
           tc_fence_after();
-          const int limit = visible_prefix<M>(it, a, row_tok[i], j, q) - part * kCols;  // in this part
           // Most tiles are fully visible: mask only when some row of the warp needs it.
-          const bool masked = __any_sync(0xffffffffu, limit < kCols);
+          int limit = kCols;
+          bool masked = false;
+          if (j >= full_upto) {
+            limit = visible_prefix<M>(it, a, row_tok[i], j, q) - part * kCols;  // in this part
+            masked = __any_sync(0xffffffffu, limit < kCols);
+          }
           // S in pieces of 32: the max over the first pieces overlaps the TMEM read of
           // the later ones. Row max with independent 3-input max chains.
           float mc[kChunks];
